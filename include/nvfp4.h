@@ -1,0 +1,200 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so, the B200 (sm_100a) NVFP4 linear-layer training path.
+ *
+ * What the library computes (web pages on NVFP4 training):
+ *  - NVFP4: E2M1 4-bit elements, one E4M3 scale per 16 elements and one FP32 scale
+ *    per tensor, 4.5 bits per element ("Nemotron NVFP4" explainer,
+ *    ai.thesatyajit.com, "What NVFP4 actually is").
+ *  - 1x16 blocks for activations and gradients, 16x16 blocks for weights;
+ *    round-to-nearest-even, stochastic rounding for gradients only; a random
+ *    Hadamard transform on the weight-gradient GEMM inputs; fprop, dgrad and
+ *    wgrad GEMMs in NVFP4 ("NVIDIA's 4-bit floating point pushes AI training
+ *    limits", artiverse.ca; explainer, "Why 4-bit training normally falls apart --
+ *    and the three fixes").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *    allocates device memory.  Host pointers are marked "host".
+ *  - bf16 tensors are row-major [rows][cols] (cols contiguous), 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *    Argument errors are detected on the host before anything is launched and
+ *    returned as a negative nvfp4_status; nothing is written in that case.
+ *  - Errors found on the device (non-finite input, a bounded wait that ran out)
+ *    are recorded in a status word in the caller's workspace; read it with
+ *    nvfp4_read_status() (which synchronizes the stream).
+ *  - No entry point traps, asserts on the device or throws across the ABI.
+ *
+ * Numerics (fixed readings of points the pages leave open):
+ *  - decode scale g = amax / (6 * 448) (fp32), encode factor 2688 / amax.
+ *  - block scale s = E4M3_rne_satfinite((amax_b / 6) * enc); element
+ *    v = x * (1 / (dec(s) * g)) rounded to E2M1 (RNE, or stochastic with a
+ *    16-bit Philox4x32-10 draw keyed by (seed, element index)).
+ *  - scales are stored in the block-scaled MMA layout: 512-byte atoms of
+ *    128 rows x 4 blocks, rows padded to 128 and blocks to 4 with zeros.
+ *  - packed codes: [rows][cols/2] bytes, element 2j in the low nibble.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* identical to cudaStream_t */
+
+typedef enum nvfp4_status {
+    NVFP4_OK = 0,
+    NVFP4_ERR_ARG = -1,       /* null pointer, bad enum value, bad sign vector      */
+    NVFP4_ERR_SHAPE = -2,     /* a size is not a multiple the operation needs       */
+    NVFP4_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned                   */
+    NVFP4_ERR_CUDA = -4,      /* a CUDA runtime call or launch failed               */
+    NVFP4_ERR_NONFINITE = -5, /* device status: the input held Inf or NaN           */
+    NVFP4_ERR_TIMEOUT = -6,   /* device status: a bounded wait in a kernel ran out  */
+    NVFP4_ERR_WORKSPACE = -7, /* workspace pointer null or smaller than required    */
+    NVFP4_ERR_DEVICE = -8     /* the current device is not sm_100 (B200 class)      */
+} nvfp4_status;
+
+enum { NVFP4_BLOCK_1X16 = 0, NVFP4_BLOCK_16X16 = 1 };
+enum { NVFP4_ROUND_RNE = 0, NVFP4_ROUND_SR = 1 };
+
+/* One quantized operand as the GEMM reads it (reduction axis = cols). */
+typedef struct nvfp4_tensor {
+    uint8_t* data;        /* E2M1 codes, nvfp4_packed_bytes(rows, cols) bytes        */
+    uint8_t* scales;      /* E4M3 block scales, nvfp4_scale_bytes(rows, cols) bytes   */
+    float* tensor_scale;  /* one fp32: the decode scale g                            */
+    int64_t rows;
+    int64_t cols;
+} nvfp4_tensor;
+
+/* Sizes (bytes).  packed = rows*cols/2; scales = pad128(rows) * pad4(cols/16). */
+size_t nvfp4_packed_bytes(int64_t rows, int64_t cols);
+size_t nvfp4_scale_bytes(int64_t rows, int64_t cols);
+/* Scratch of nvfp4_quantize / nvfp4_quantize_2d (tensor amax words + status). */
+size_t nvfp4_quantize_workspace_bytes(void);
+
+/*
+ * nvfp4_quantize -- quantize a bf16 tensor along its rows (blocks run along cols).
+ * Defines: the two-level NVFP4 encoding of the explainer's "What NVFP4 actually
+ * is"; 1x16 strips ("activations and gradients") or 16x16 tiles ("weights",
+ * artiverse.ca).
+ *   x            [rows][cols] bf16.  cols % 16 == 0; 16x16 also needs rows % 16 == 0.
+ *   block_mode   NVFP4_BLOCK_1X16 or NVFP4_BLOCK_16X16.
+ *   rounding     NVFP4_ROUND_RNE or NVFP4_ROUND_SR (Philox stream 0, key = seed).
+ *   packed       out, nvfp4_packed_bytes(rows, cols) bytes.
+ *   scales       out, nvfp4_scale_bytes(rows, cols) bytes (padding written as 0).
+ *   tensor_scale out, one float: g = amax / 2688 (NaN if x held Inf/NaN).
+ *   workspace    nvfp4_quantize_workspace_bytes() bytes of device scratch; its status
+ *                word reports NVFP4_ERR_NONFINITE (see nvfp4_read_status).
+ * Launches: one amax pass and one quantize pass (two reads of x).
+ */
+int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int block_mode, int rounding,
+                   uint64_t seed, uint8_t* packed, uint8_t* scales, float* tensor_scale,
+                   void* workspace, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_quantize_2d -- one read of x, up to two quantized orientations.
+ * Defines: the row orientation as nvfp4_quantize; the column orientation quantizes
+ * x^T (blocks run down the rows of x), optionally after the 16-point random
+ * Hadamard transform along the rows ("Random Hadamard transform on the wgrad
+ * inputs", explainer).  With 16x16 blocks both orientations share the tile scales,
+ * so their codes are exact transposes ("consistency between forward and backward",
+ * artiverse.ca).
+ *   row_out  nullable; rows x cols operand (data, scales, tensor_scale filled).
+ *   col_out  nullable; cols x rows operand.  Needs rows % 16 == 0.
+ *   opts     host struct below; rht_signs is a HOST array of 16 entries, each +1/-1.
+ * The column orientation draws from Philox stream 1, the row orientation stream 0.
+ */
+typedef struct nvfp4_quantize_opts {
+    int block_mode;          /* NVFP4_BLOCK_1X16 / NVFP4_BLOCK_16X16                 */
+    int row_rounding;        /* NVFP4_ROUND_RNE / NVFP4_ROUND_SR                      */
+    int col_rounding;        /* NVFP4_ROUND_RNE / NVFP4_ROUND_SR                      */
+    uint64_t seed;           /* Philox key for stochastic rounding                    */
+    int col_rht;             /* 1: transform the column orientation (1x16 only)       */
+    const int8_t* rht_signs; /* host, 16 x (+1|-1); required when col_rht == 1         */
+} nvfp4_quantize_opts;
+int nvfp4_quantize_2d(const void* x, int64_t rows, int64_t cols, const nvfp4_quantize_opts* opts,
+                      nvfp4_tensor* row_out, nvfp4_tensor* col_out, void* workspace,
+                      nvfp4_stream_t stream);
+
+/*
+ * nvfp4_rht -- standalone 16-point random Hadamard transform, fp32 output.
+ * Defines: y = x . diag(signs) . H16 on every 16-element chunk along `axis`, with
+ * the unnormalised Sylvester H16 (H16 H16^T = 16 I), so the transform is undone
+ * analytically by dividing the wgrad product by 16 (explainer, "the three fixes").
+ *   x      [rows][cols] bf16;  y  [rows][cols] fp32 (same layout).
+ *   axis   1: chunks along cols (cols % 16 == 0);  0: chunks along rows (rows % 16 == 0).
+ *   signs  HOST array of n entries, each +1 or -1;  n must be 16.
+ * Each output is the fp32 rounding of the exact sum (exact when the 16 inputs'
+ * exponents span at most 41 binades).
+ */
+int nvfp4_rht(const void* x, int64_t rows, int64_t cols, int axis, const int8_t* signs, int n,
+              float* y, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm -- block-scaled FP4 GEMM with fp32 accumulation.
+ * Defines: D[m][n] = alpha * gA * gB * sum_k a[m][k] * b[n][k], a and b the decoded
+ * E2M1 x E4M3 values (fprop, dgrad and wgrad all have this form; artiverse.ca).
+ *   A, sfA     M x K operand (codes, swizzled scales).   B, sfB   N x K operand.
+ *   scale_a/b  device pointers to the tensor scales gA, gB (nullable: 1.0).
+ *   alpha      host multiplier (1/16 for the RHT-rotated wgrad).
+ *   D_bf16     nullable; [M][N] bf16, rounded to nearest even from the fp32 value.
+ *   D_f32      nullable; [M][N] fp32 (the value before the bf16 rounding).
+ *   status     nullable device int; set to NVFP4_ERR_TIMEOUT if a pipeline wait ran
+ *              out (the output is then incomplete).
+ * Needs K % 64 == 0, N % 8 == 0, at least one of D_bf16 / D_f32, 16-byte alignment.
+ */
+int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+               const float* scale_a, const float* scale_b, float alpha, int64_t M, int64_t N,
+               int64_t K, void* D_bf16, float* D_f32, int* status, nvfp4_stream_t stream);
+
+/*
+ * Linear layer Y = X W^T in NVFP4 (artiverse.ca: forward, backward and weight-gradient
+ * GEMMs in 4 bits; 16x16 weight blocks; RHT on the weight-gradient inputs; stochastic
+ * rounding on gradients only).
+ *   X [M][K], W [N][K], Y [M][N], dY [M][N], dX [M][K], dW [N][K]; all bf16.
+ *   M, K and N multiples of 64 (each is the reduction axis of one of the GEMMs).
+ *   ws / ws_bytes  device workspace of nvfp4_linear_workspace_bytes(M, K, N) bytes.
+ *                  It holds the quantized operands between the three calls.
+ *   rht_signs      HOST array of 16 x (+1|-1); the same vector must be passed to
+ *                  fprop, dgrad and wgrad of one step.
+ * fprop: quantizes X (rows RNE + columns RHT RNE, one read) and W (16x16, both
+ *        orientations, one read); Y = X W^T.
+ * dgrad: quantizes dY (rows SR stream 0 + columns RHT SR stream 1, one read);
+ *        dX = dY W.
+ * wgrad: dW = (dY^T D H)(X^T D H)^T / 16.  dY nullable: NULL reuses the quantized dY
+ *        that dgrad left in ws; non-NULL quantizes dY's columns here.
+ */
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
+int nvfp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* Views of the quantized operands a linear workspace holds (no device access). */
+enum {
+    NVFP4_LIN_X_ROW = 0,  /* X,   M x K, 1x16 RNE                 */
+    NVFP4_LIN_X_COL = 1,  /* X^T, K x M, RHT + 1x16 RNE           */
+    NVFP4_LIN_W_ROW = 2,  /* W,   N x K, 16x16 RNE                */
+    NVFP4_LIN_W_COL = 3,  /* W^T, K x N, 16x16 RNE                */
+    NVFP4_LIN_DY_ROW = 4, /* dY,  M x N, 1x16 SR                  */
+    NVFP4_LIN_DY_COL = 5  /* dY^T, N x M, RHT + 1x16 SR           */
+};
+int nvfp4_linear_operand(void* ws, int64_t M, int64_t K, int64_t N, int which,
+                         nvfp4_tensor* out);
+
+/* Status word of a quantize or linear workspace (synchronizes `stream`, then
+ * clears the word).  *status = NVFP4_OK or the first device error recorded.    */
+int nvfp4_read_status(void* workspace, int* status, nvfp4_stream_t stream);
+
+const char* nvfp4_status_string(int status);
+int nvfp4_version(void); /* major * 10000 + minor * 100 + patch */
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

@@ -1,0 +1,406 @@
+// capi.cu -- the extern "C" boundary of libnvfp4 (declared in include/nvfp4.h).
+//
+// Host-side only: argument validation (before any launch), workspace layout,
+// and the order of kernel launches for each entry point.  Every step of the
+// computation runs in the kernels of quantize.cu and gemm.cu.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/nvfp4.h"
+#include "internal.h"
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr int64_t kCtrlBytes = 256;   // control block at the start of a workspace
+constexpr int kWordStatus = 8;        // int status at byte 32 of every workspace
+constexpr int64_t kClearBytes = 64;   // amax words + status, cleared by every call
+// linear workspace: amax words and tensor-scale slots inside the control block
+constexpr int kWX = 0, kWW = 2, kWDY = 4;                   // word pairs [row, col]
+constexpr int kGxr = 16, kGxc = 17, kGw = 18, kGwc = 19, kGdyr = 20, kGdyc = 21;  // float slots
+
+int64_t pad(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct DevInfo {
+    int sm_count = 0;
+    int status = 0;  // 0 unknown, 1 ok, -1 not sm_100
+};
+
+int device_check(int* sm_count) {
+    static DevInfo info[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+    DevInfo& d = info[dev];
+    if (d.status == 0) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        d.sm_count = sms;
+        d.status = (major == 10) ? 1 : -1;
+    }
+    if (d.status < 0) return NVFP4_ERR_DEVICE;
+    *sm_count = d.sm_count;
+    return NVFP4_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+// Sign vector (+1/-1 x 16, host) -> bit mask of the -1 entries.
+int sign_mask_of(const int8_t* signs, uint32_t* mask) {
+    if (!signs) return NVFP4_ERR_ARG;
+    uint32_t m = 0;
+    for (int i = 0; i < 16; ++i) {
+        if (signs[i] == -1)
+            m |= 1u << i;
+        else if (signs[i] != 1)
+            return NVFP4_ERR_ARG;
+    }
+    *mask = m;
+    return NVFP4_OK;
+}
+
+struct LinLayout {
+    int64_t x_row, x_row_sf, x_col, x_col_sf, w_row, w_row_sf, w_col, w_col_sf;
+    int64_t dy_row, dy_row_sf, dy_col, dy_col_sf, total;
+};
+LinLayout lin_layout(int64_t M, int64_t K, int64_t N) {
+    LinLayout L;
+    int64_t off = kCtrlBytes;
+    auto take = [&](int64_t bytes) {
+        const int64_t o = off;
+        off = pad(off + bytes, 256);
+        return o;
+    };
+    L.x_row = take(M * K / 2);
+    L.x_row_sf = take((int64_t)nvfp4_scale_bytes(M, K));
+    L.x_col = take(K * M / 2);
+    L.x_col_sf = take((int64_t)nvfp4_scale_bytes(K, M));
+    L.w_row = take(N * K / 2);
+    L.w_row_sf = take((int64_t)nvfp4_scale_bytes(N, K));
+    L.w_col = take(K * N / 2);
+    L.w_col_sf = take((int64_t)nvfp4_scale_bytes(K, N));
+    L.dy_row = take(M * N / 2);
+    L.dy_row_sf = take((int64_t)nvfp4_scale_bytes(M, N));
+    L.dy_col = take(N * M / 2);
+    L.dy_col_sf = take((int64_t)nvfp4_scale_bytes(N, M));
+    L.total = off;
+    return L;
+}
+
+int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_sr, int col_sr,
+                 uint64_t seed, int col_rht, uint32_t mask, uint8_t* rd, uint8_t* rsf, float* rg,
+                 uint8_t* cd, uint8_t* csf, float* cg, uint32_t* words, int* status, int sms,
+                 cudaStream_t st, bool rows_only_kernel) {
+    cudaError_t e = launch_amax(static_cast<const uint16_t*>(x), rows, cols, col_rht && cd, mask,
+                                words, sms, st);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    QuantParams p;
+    memset(&p, 0, sizeof p);
+    p.x = static_cast<const uint16_t*>(x);
+    p.rows = rows;
+    p.cols = cols;
+    p.row_data = rd;
+    p.row_sf = rsf;
+    p.row_g = rg;
+    p.col_data = cd;
+    p.col_sf = csf;
+    p.col_g = cg;
+    p.amax_words = words;
+    p.status = status;
+    p.seed = seed;
+    p.row_sr = row_sr;
+    p.col_sr = col_sr;
+    p.col_rht = (col_rht && cd) ? 1 : 0;
+    p.sign_mask = mask;
+    e = rows_only_kernel ? launch_quant_rows(p, sms, st) : launch_quant_tile(p, two_d, st);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (rsf && (e = launch_sf_pad(rsf, rows, cols / 16, sms, st)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (csf && (e = launch_sf_pad(csf, cols, rows / 16, sms, st)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+int gemm_call(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+              const float* sa, const float* sb, float alpha, int64_t M, int64_t N, int64_t K,
+              void* Dbf, float* Df, int* status, int sms, cudaStream_t st) {
+    GemmParams g;
+    g.A = A;
+    g.sfA = sfA;
+    g.B = B;
+    g.sfB = sfB;
+    g.scale_a = sa;
+    g.scale_b = sb;
+    g.alpha = alpha;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.D_bf16 = Dbf;
+    g.D_f32 = Df;
+    g.status = status;
+    return cuda_status(launch_gemm(g, sms, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_version(void) { return 100; }
+
+const char* nvfp4_status_string(int s) {
+    switch (s) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_ARG: return "invalid argument";
+        case NVFP4_ERR_SHAPE: return "unsupported shape";
+        case NVFP4_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case NVFP4_ERR_CUDA: return "CUDA error";
+        case NVFP4_ERR_NONFINITE: return "input holds Inf or NaN";
+        case NVFP4_ERR_TIMEOUT: return "a bounded wait in a kernel ran out";
+        case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+        case NVFP4_ERR_DEVICE: return "device is not sm_100";
+        default: return "unknown status";
+    }
+}
+
+size_t nvfp4_packed_bytes(int64_t rows, int64_t cols) {
+    return (rows <= 0 || cols <= 0) ? 0 : (size_t)(rows * cols / 2);
+}
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t cols) {
+    return (rows <= 0 || cols <= 0) ? 0 : (size_t)(pad(rows, 128) * pad(cols / 16, 4));
+}
+
+size_t nvfp4_quantize_workspace_bytes(void) { return (size_t)kCtrlBytes; }
+
+int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int block_mode, int rounding,
+                   uint64_t seed, uint8_t* packed, uint8_t* scales, float* tensor_scale,
+                   void* workspace, nvfp4_stream_t stream) {
+    if (!x || !packed || !scales || !tensor_scale) return NVFP4_ERR_ARG;
+    if (!workspace) return NVFP4_ERR_WORKSPACE;
+    if (block_mode != NVFP4_BLOCK_1X16 && block_mode != NVFP4_BLOCK_16X16) return NVFP4_ERR_ARG;
+    if (rounding != NVFP4_ROUND_RNE && rounding != NVFP4_ROUND_SR) return NVFP4_ERR_ARG;
+    if (rows < 1 || cols < 16 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (block_mode == NVFP4_BLOCK_16X16 && rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 16) || !aligned(workspace, 16) ||
+        !aligned(tensor_scale, 4))
+        return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* words = static_cast<uint32_t*>(workspace);
+    if (cudaMemsetAsync(words, 0, kClearBytes, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return run_quantize(x, rows, cols, block_mode == NVFP4_BLOCK_16X16, rounding, 0, seed, 0, 0,
+                        packed, scales, tensor_scale, nullptr, nullptr, nullptr, words,
+                        reinterpret_cast<int*>(words + kWordStatus), sms, st,
+                        block_mode == NVFP4_BLOCK_1X16);
+}
+
+int nvfp4_quantize_2d(const void* x, int64_t rows, int64_t cols, const nvfp4_quantize_opts* o,
+                      nvfp4_tensor* row_out, nvfp4_tensor* col_out, void* workspace,
+                      nvfp4_stream_t stream) {
+    if (!x || !o || (!row_out && !col_out)) return NVFP4_ERR_ARG;
+    if (!workspace) return NVFP4_ERR_WORKSPACE;
+    if (o->block_mode != NVFP4_BLOCK_1X16 && o->block_mode != NVFP4_BLOCK_16X16) return NVFP4_ERR_ARG;
+    if ((o->row_rounding != 0 && o->row_rounding != 1) || (o->col_rounding != 0 && o->col_rounding != 1))
+        return NVFP4_ERR_ARG;
+    uint32_t mask = 0;
+    if (o->col_rht) {
+        if (o->block_mode != NVFP4_BLOCK_1X16) return NVFP4_ERR_ARG;
+        if (sign_mask_of(o->rht_signs, &mask)) return NVFP4_ERR_ARG;
+    }
+    if (rows < 1 || cols < 16 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if ((col_out || o->block_mode == NVFP4_BLOCK_16X16) && rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    for (nvfp4_tensor* t : {row_out, col_out}) {
+        if (!t) continue;
+        if (!t->data || !t->scales || !t->tensor_scale) return NVFP4_ERR_ARG;
+        if (!aligned(t->data, 16) || !aligned(t->scales, 16) || !aligned(t->tensor_scale, 4))
+            return NVFP4_ERR_ALIGN;
+    }
+    if (!aligned(x, 16) || !aligned(workspace, 16)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* words = static_cast<uint32_t*>(workspace);
+    if (cudaMemsetAsync(words, 0, kClearBytes, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (row_out) {
+        row_out->rows = rows;
+        row_out->cols = cols;
+    }
+    if (col_out) {
+        col_out->rows = cols;
+        col_out->cols = rows;
+    }
+    return run_quantize(x, rows, cols, o->block_mode == NVFP4_BLOCK_16X16, o->row_rounding,
+                        o->col_rounding, o->seed, o->col_rht, mask,
+                        row_out ? row_out->data : nullptr, row_out ? row_out->scales : nullptr,
+                        row_out ? row_out->tensor_scale : nullptr, col_out ? col_out->data : nullptr,
+                        col_out ? col_out->scales : nullptr,
+                        col_out ? col_out->tensor_scale : nullptr, words,
+                        reinterpret_cast<int*>(words + kWordStatus), sms, st, false);
+}
+
+int nvfp4_rht(const void* x, int64_t rows, int64_t cols, int axis, const int8_t* signs, int n,
+              float* y, nvfp4_stream_t stream) {
+    if (!x || !y) return NVFP4_ERR_ARG;
+    if (n != 16 || (axis != 0 && axis != 1)) return NVFP4_ERR_ARG;
+    uint32_t mask = 0;
+    if (sign_mask_of(signs, &mask)) return NVFP4_ERR_ARG;
+    if (rows < 1 || cols < 1) return NVFP4_ERR_SHAPE;
+    if (axis == 1 && cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (axis == 0 && (rows % 16 != 0 || cols % 8 != 0)) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(y, 16)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    return cuda_status(launch_rht(static_cast<const uint16_t*>(x), y, rows, cols, axis, mask, sms,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+               const float* scale_a, const float* scale_b, float alpha, int64_t M, int64_t N,
+               int64_t K, void* D_bf16, float* D_f32, int* status, nvfp4_stream_t stream) {
+    if (!A || !sfA || !B || !sfB || (!D_bf16 && !D_f32)) return NVFP4_ERR_ARG;
+    if (M < 1 || N < 8 || K < 64 || K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_SHAPE;
+    if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K / 2 > (1ll << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sfA, 16) || !aligned(sfB, 16) ||
+        (D_bf16 && !aligned(D_bf16, 16)) || (D_f32 && !aligned(D_f32, 16)))
+        return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    return gemm_call(A, sfA, B, sfB, scale_a, scale_b, alpha, M, N, K, D_bf16, D_f32, status, sms,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+    if (M <= 0 || K <= 0 || N <= 0) return 0;
+    return (size_t)lin_layout(M, K, N).total;
+}
+
+int nvfp4_linear_operand(void* ws, int64_t M, int64_t K, int64_t N, int which, nvfp4_tensor* out) {
+    if (!ws || !out) return NVFP4_ERR_ARG;
+    if (M <= 0 || K <= 0 || N <= 0) return NVFP4_ERR_SHAPE;
+    const LinLayout L = lin_layout(M, K, N);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    float* g = reinterpret_cast<float*>(b);
+    switch (which) {
+        case NVFP4_LIN_X_ROW: *out = {b + L.x_row, b + L.x_row_sf, g + kGxr, M, K}; break;
+        case NVFP4_LIN_X_COL: *out = {b + L.x_col, b + L.x_col_sf, g + kGxc, K, M}; break;
+        case NVFP4_LIN_W_ROW: *out = {b + L.w_row, b + L.w_row_sf, g + kGw, N, K}; break;
+        case NVFP4_LIN_W_COL: *out = {b + L.w_col, b + L.w_col_sf, g + kGwc, K, N}; break;
+        case NVFP4_LIN_DY_ROW: *out = {b + L.dy_row, b + L.dy_row_sf, g + kGdyr, M, N}; break;
+        case NVFP4_LIN_DY_COL: *out = {b + L.dy_col, b + L.dy_col_sf, g + kGdyc, N, M}; break;
+        default: return NVFP4_ERR_ARG;
+    }
+    return NVFP4_OK;
+}
+
+static int lin_check(int64_t M, int64_t K, int64_t N, void* ws, size_t ws_bytes) {
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (M < 64 || K < 64 || N < 64 || M % 64 || K % 64 || N % 64) return NVFP4_ERR_SHAPE;
+    if (ws_bytes < nvfp4_linear_workspace_bytes(M, K, N)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return NVFP4_ERR_ALIGN;
+    return NVFP4_OK;
+}
+
+int nvfp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!X || !W || !Y) return NVFP4_ERR_ARG;
+    uint32_t mask = 0;
+    if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
+    int rc = lin_check(M, K, N, ws, ws_bytes);
+    if (rc) return rc;
+    if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    if ((rc = device_check(&sms))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    nvfp4_tensor xr, xc, wr, wc;
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_X_ROW, &xr);
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_X_COL, &xc);
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_W_ROW, &wr);
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_W_COL, &wc);
+    uint32_t* words = static_cast<uint32_t*>(ws);
+    int* status = reinterpret_cast<int*>(words + kWordStatus);
+    if (cudaMemsetAsync(words, 0, kClearBytes, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    // X: rows (1x16 RNE) for fprop, RHT columns (1x16 RNE) for wgrad -- one read
+    rc = run_quantize(X, M, K, false, 0, 0, 0, 1, mask, xr.data, xr.scales, xr.tensor_scale, xc.data,
+                      xc.scales, xc.tensor_scale, words + kWX, status, sms, st, false);
+    if (rc) return rc;
+    // W: 16x16 RNE, both orientations -- one read
+    rc = run_quantize(W, N, K, true, 0, 0, 0, 0, 0, wr.data, wr.scales, wr.tensor_scale, wc.data,
+                      wc.scales, wc.tensor_scale, words + kWW, status, sms, st, false);
+    if (rc) return rc;
+    return gemm_call(xr.data, xr.scales, wr.data, wr.scales, xr.tensor_scale, wr.tensor_scale, 1.0f,
+                     M, N, K, Y, nullptr, status, sms, st);
+}
+
+int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!dY || !dX) return NVFP4_ERR_ARG;
+    uint32_t mask = 0;
+    if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
+    int rc = lin_check(M, K, N, ws, ws_bytes);
+    if (rc) return rc;
+    if (!aligned(dY, 16) || !aligned(dX, 16)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    if ((rc = device_check(&sms))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    nvfp4_tensor dr, dc, wc;
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_DY_ROW, &dr);
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_DY_COL, &dc);
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_W_COL, &wc);
+    uint32_t* words = static_cast<uint32_t*>(ws);
+    int* status = reinterpret_cast<int*>(words + kWordStatus);
+    if (cudaMemsetAsync(words, 0, kClearBytes, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    // dY: rows (1x16 SR, stream 0) for dgrad, RHT columns (1x16 SR, stream 1) for wgrad
+    rc = run_quantize(dY, M, N, false, 1, 1, seed, 1, mask, dr.data, dr.scales, dr.tensor_scale,
+                      dc.data, dc.scales, dc.tensor_scale, words + kWDY, status, sms, st, false);
+    if (rc) return rc;
+    return gemm_call(dr.data, dr.scales, wc.data, wc.scales, dr.tensor_scale, wc.tensor_scale, 1.0f,
+                     M, K, N, dX, nullptr, status, sms, st);
+}
+
+int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!dW) return NVFP4_ERR_ARG;
+    uint32_t mask = 0;
+    if (dY && sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
+    int rc = lin_check(M, K, N, ws, ws_bytes);
+    if (rc) return rc;
+    if ((dY && !aligned(dY, 16)) || !aligned(dW, 16)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    if ((rc = device_check(&sms))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    nvfp4_tensor dc, xc;
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_DY_COL, &dc);
+    nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_X_COL, &xc);
+    uint32_t* words = static_cast<uint32_t*>(ws);
+    int* status = reinterpret_cast<int*>(words + kWordStatus);
+    if (cudaMemsetAsync(words, 0, kClearBytes, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dY) {
+        rc = run_quantize(dY, M, N, false, 0, 1, seed, 1, mask, nullptr, nullptr, nullptr, dc.data,
+                          dc.scales, dc.tensor_scale, words + kWDY, status, sms, st, false);
+        if (rc) return rc;
+    }
+    // dW = (dY^T D H)(X^T D H)^T / 16: the rotation cancels, H H^T = 16 I
+    return gemm_call(dc.data, dc.scales, xc.data, xc.scales, dc.tensor_scale, xc.tensor_scale,
+                     1.0f / 16.0f, N, K, M, dW, nullptr, status, sms, st);
+}
+
+int nvfp4_read_status(void* workspace, int* status, nvfp4_stream_t stream) {
+    if (!workspace || !status) return NVFP4_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, static_cast<uint32_t*>(workspace) + kWordStatus, sizeof v,
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    *status = v;
+    return NVFP4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,383 @@
+// gemm.cu -- block-scaled NVFP4 GEMM on the sm_100a 5th-generation tensor cores.
+//
+// D[m][n] = alpha * gA * gB * sum_k a[m][k] * b[n][k], with a, b the decoded
+// E2M1 codes times their E4M3 16-element block scales, fp32 accumulation.  The
+// fprop, dgrad and wgrad GEMMs of the NVFP4 linear layer all take this form
+// ("NVIDIA's 4-bit floating point pushes AI training limits", artiverse.ca).
+//
+// Design (one CTA = one 128 x BN output tile, 128 threads):
+//   warp 0 lane 0   TMA producer: A/B tiles (128-byte swizzled K-major boxes of
+//                   256 FP4 along K) and the matching 512-byte scale atoms
+//                   (bulk copies) into a STAGES-deep shared-memory ring.
+//   warp 1 lane 0   MMA issuer: copies the stage's scale atoms to TMEM with
+//                   tcgen05.cp (32x128b, replicated to the four lane quadrants),
+//                   then four tcgen05.mma kind::mxf4nvf4 block_scale (K = 64 each)
+//                   into the fp32 accumulator in TMEM; tcgen05.commit frees the
+//                   stage, and a final commit signals the epilogue.
+//   warps 0-3       epilogue: tcgen05.ld of their 32 accumulator lanes, scale by
+//                   alpha * gA * gB, store fp32 and/or bf16.
+// Every wait is bounded: after ~1 s the kernel records NVFP4_ERR_TIMEOUT in the
+// status word, stops issuing work, drains its own copies and frees TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+
+constexpr int kBM = 128;         // rows of A per tile (MMA M)
+constexpr int kBKBytes = 128;    // bytes of K per stage per row (256 FP4)
+constexpr int kKStep = 64;       // FP4 elements per MMA
+constexpr long long kWaitCycles = 1ll << 31;
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+// Copy one 512-byte scale atom (32 lines of 16 bytes) into 4 TMEM columns, the
+// 32 lines replicated into each of the four 32-lane quadrants.
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format): start address, leading and
+// stride byte offsets (all >> 4), descriptor version 1, layout type.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                               uint32_t layout) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+// K-major operand with 128-byte swizzle: 8-row x 128-byte atoms, 1024 B apart.
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
+    return make_sdesc(saddr, 16, 1024, 2);
+}
+// Scale atom source of tcgen05.cp: unswizzled 8 x 16-byte core matrices, 128 B apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) { return make_sdesc(saddr, 0, 128, 0); }
+
+// Instruction descriptor of kind::mxf4nvf4 block-scaled MMA: E2M1 A and B
+// (format 1), K-major both, UE4M3 scales (scale format 0), M = 128, N = BN,
+// K = 64 per instruction, dense.
+template <int BN>
+__host__ __device__ constexpr uint32_t nvf4_idesc() {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (0u << 23) |
+           ((uint32_t)(kBM >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- shared memory
+template <int BN, int STAGES>
+struct __align__(1024) GemmSmem {
+    uint8_t a[STAGES][kBM * kBKBytes];          // 16 KB / stage
+    uint8_t b[STAGES][BN * kBKBytes];           // BN * 128 B / stage
+    uint8_t sfa[STAGES][4 * 512];               // 4 atoms: 128 rows x 16 blocks
+    uint8_t sfb[STAGES][(BN / 128) * 4 * 512];  // per 128-row group, 4 atoms
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t acc_full;
+    uint32_t tmem_base;
+};
+
+template <int BN>
+struct TmemLayout {
+    static constexpr int kSfaCols = 16;                   // 4 k-steps x 4 columns
+    static constexpr int kSfbCols = 4 * 4 * (BN / 128);   // 4 k-steps x 4 columns per group
+    static constexpr int kRegion = kSfaCols + kSfbCols;   // scales of one stage
+    static constexpr int kUsed = BN + 2 * kRegion;        // accumulator + two scale regions
+    static constexpr int kAlloc = kUsed <= 32 ? 32 : kUsed <= 64 ? 64 : kUsed <= 128 ? 128
+                                : kUsed <= 256 ? 256 : 512;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(128, 1)
+    gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmParams p) {
+    using Smem = GemmSmem<BN, STAGES>;
+    using TL = TmemLayout<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m0 = (int64_t)blockIdx.y * kBM;
+    const int64_t n0 = (int64_t)blockIdx.x * BN;
+    const int64_t katoms = p.K / 64;                 // scale atoms per 128-row group
+    const int KT = (int)((p.K + 255) / 256);         // k-tiles of 256
+    const int64_t nb_groups = (p.N + 127) / 128;     // 128-row groups of B
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_addr(&S.full[s]), 1);
+            mbar_init(smem_addr(&S.empty[s]), 1);
+        }
+        mbar_init(smem_addr(&S.acc_full), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&S.tmem_base)),
+                     "r"((uint32_t)TL::kAlloc)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    __shared__ int timed_out;
+    if (threadIdx.x == 0) timed_out = 0;
+    __syncthreads();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int armed = 0;  // k-tiles whose full barrier was armed
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t use = (uint32_t)(kt / STAGES);
+                if (kt >= STAGES && !mbar_wait(smem_addr(&S.empty[s]), (use & 1u) ^ 1u)) {
+                    timed_out = 1;
+                    break;
+                }
+                if (*(volatile int*)&timed_out) break;
+                const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
+                const int nks = rem < 4 ? (int)rem : 4;
+                uint32_t sf_bytes = (uint32_t)nks * 512u;
+                uint32_t bytes = kBM * kBKBytes + BN * kBKBytes + sf_bytes;
+                for (int g = 0; g < BN / 128; ++g)
+                    if (n0 / 128 + g < nb_groups) bytes += sf_bytes;
+                const uint32_t fb = smem_addr(&S.full[s]);
+                mbar_expect_tx(fb, bytes);
+                tma_load_2d(smem_addr(S.a[s]), &tmA, kt * kBKBytes, (int)m0, fb);
+                tma_load_2d(smem_addr(S.b[s]), &tmB, kt * kBKBytes, (int)n0, fb);
+                bulk_load(smem_addr(S.sfa[s]), p.sfA + ((m0 / 128) * katoms + (int64_t)kt * 4) * 512,
+                          sf_bytes, fb);
+                for (int g = 0; g < BN / 128; ++g)
+                    if (n0 / 128 + g < nb_groups)
+                        bulk_load(smem_addr(S.sfb[s] + g * 2048),
+                                  p.sfB + ((n0 / 128 + g) * katoms + (int64_t)kt * 4) * 512, sf_bytes,
+                                  fb);
+                armed = kt + 1;
+            }
+            if (*(volatile int*)&timed_out) {
+                // let copies already issued land before the CTA can exit
+                for (int kt = max(0, armed - STAGES); kt < armed; ++kt)
+                    mbar_wait(smem_addr(&S.full[kt % STAGES]), (uint32_t)(kt / STAGES) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = nvf4_idesc<BN>();
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(kt / STAGES) & 1u)) {
+                    timed_out = 1;
+                    break;
+                }
+                tc_fence_after();
+                const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
+                const int nks = rem < 4 ? (int)rem : 4;
+                const uint32_t region = (uint32_t)(BN + (kt & 1) * TL::kRegion);
+                const uint32_t t_sfa = tmem + region;
+                const uint32_t t_sfb = tmem + region + TL::kSfaCols;
+                const uint32_t a_base = smem_addr(S.a[s]), b_base = smem_addr(S.b[s]);
+                for (int j = 0; j < nks; ++j) {
+                    tc_cp_sf(t_sfa + 4 * j, sf_desc(smem_addr(S.sfa[s] + j * 512)));
+                    for (int g = 0; g < BN / 128; ++g)
+                        tc_cp_sf(t_sfb + 4 * (BN / 128) * j + 4 * g,
+                                 sf_desc(smem_addr(S.sfb[s] + g * 2048 + j * 512)));
+                }
+                for (int j = 0; j < nks; ++j) {
+                    tc_mma_nvf4(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                                idesc, t_sfa + 4 * j, t_sfb + 4 * (BN / 128) * j,
+                                (kt > 0 || j > 0) ? 1u : 0u);
+                }
+                tc_commit(smem_addr(&S.empty[s]));
+            }
+            tc_commit(smem_addr(&S.acc_full));
+        }
+        __syncwarp();
+    }
+
+    // ---------------------------------------------------- epilogue (all warps)
+    const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), 0);
+    tc_fence_after();
+    __syncwarp();
+    if (!acc_ok) timed_out = 1;
+    const bool bad = *(volatile int*)&timed_out != 0;
+    float alpha = p.alpha;
+    if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
+    if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
+    const int64_t row = m0 + warp * 32 + lane;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+            "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+              "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+              "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+              "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+              "=r"(r[31])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (bad || row >= p.M) continue;
+        const int64_t col0 = n0 + c * 32;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int64_t col = col0 + 8 * g;
+            if (col >= p.N) break;
+            if (p.D_f32) {
+                float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
+                d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
+                d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+            }
+            if (p.D_bf16) {
+                uint4 w;
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * g], v[8 * g + 1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * g + 2], v[8 * g + 3]);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * g + 4], v[8 * g + 5]);
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * g + 6], v[8 * g + 7]);
+                w.x = *reinterpret_cast<uint32_t*>(&h0);
+                w.y = *reinterpret_cast<uint32_t*>(&h1);
+                w.z = *reinterpret_cast<uint32_t*>(&h2);
+                w.w = *reinterpret_cast<uint32_t*>(&h3);
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D_bf16) + row * p.N + col) = w;
+            }
+        }
+    }
+    if (threadIdx.x == 0 && *(volatile int*)&timed_out) set_status(p.status, kStatusTimeout);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"((uint32_t)TL::kAlloc)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes], box = 128 bytes x box_rows, 128-byte swizzle.
+static bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                             int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)kBKBytes, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES>
+static cudaError_t launch_gemm_cfg(const GemmParams& p, cudaStream_t st) {
+    CUtensorMap ma, mb;
+    if (!make_operand_map(&ma, p.A, p.M, p.K / 2, kBM) || !make_operand_map(&mb, p.B, p.N, p.K / 2, BN))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel<BN, STAGES>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const dim3 grid((unsigned)((p.N + BN - 1) / BN), (unsigned)((p.M + kBM - 1) / kBM));
+    gemm_nvf4_kernel<BN, STAGES><<<grid, 128, smem, st>>>(ma, mb, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
+    (void)sm_count;
+    return launch_gemm_cfg<256, 4>(p, st);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,469 @@
+// quantize.cu -- memory-bound kernels of the NVFP4 training path on sm_100a:
+//   * amax prepass (tensor max |x|, and max |RHT(x)| of the column orientation)
+//   * fused quantize: one read of a bf16 tile, row and/or column orientation,
+//     1x16 or 16x16 blocks, RNE or Philox stochastic rounding, optional 16-point
+//     random Hadamard transform in front of the column orientation
+//   * standalone RHT, and the zero fill of the scale padding.
+//
+// Method: two-level NVFP4 scaling ("Nemotron NVFP4" explainer, "What NVFP4
+// actually is"); 16x16 weight blocks, RHT on the wgrad inputs, SR on gradients
+// ("NVIDIA's 4-bit floating point pushes AI training limits", artiverse.ca).
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+
+// ============================================================================
+// 16-point Hadamard butterfly in fp64.  The Sylvester H16 is symmetric, so
+// x . diag(s) . H16 == H16 . (s * x); four radix-2 stages compute it.  Inputs
+// are bf16 values (8 significant bits), so every partial sum is exact while the
+// chunk's exponents span at most 41 binades; the fp32 rounding of the result is
+// then the correctly rounded value of the exact sum.
+// ============================================================================
+__device__ __forceinline__ void fwht16(double (&y)[16]) {
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if ((i & h) == 0) {
+                const double a = y[i], b = y[i + h];
+                y[i] = a + b;
+                y[i + h] = a - b;
+            }
+        }
+    }
+}
+
+// bf16 bit pattern with its sign flipped where the rotation sign is -1.
+__device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t flip) {
+    return (double)__uint_as_float((bits16 ^ (flip << 15)) << 16);
+}
+
+// ============================================================================
+// amax prepass.  One warp handles a 16-row x 256-column unit, each lane 16 rows
+// x 8 columns (sixteen 16-byte loads).  Word 0 receives max |x| (fp32 bits of a
+// bf16 magnitude; NaN patterns sort above Inf), word 1 max |RHT16 down the
+// rows| (column orientation), as fp32 bits.  Both are combined with atomicMax.
+// ============================================================================
+template <bool kColRht>
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                   int64_t cols, uint32_t sign_mask,
+                                                   uint32_t* __restrict__ words) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t col_units = (cols + 255) >> 8;
+    const int64_t units = ((rows + 15) >> 4) * col_units;
+    uint32_t m_row = 0;   // two packed 16-bit magnitudes
+    double m_col = 0.0;
+    for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += (int64_t)gridDim.x * 8) {
+        const int64_t r0 = (u / col_units) * 16;
+        const int64_t c0 = (u % col_units) * 256 + lane * 8;
+        if (c0 >= cols) continue;
+        uint4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            v[i] = (r0 + i < rows) ? ld_stream_v4(x + (r0 + i) * cols + c0) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            m_row = __vmaxu2(m_row, v[i].x & 0x7FFF7FFFu);
+            m_row = __vmaxu2(m_row, v[i].y & 0x7FFF7FFFu);
+            m_row = __vmaxu2(m_row, v[i].z & 0x7FFF7FFFu);
+            m_row = __vmaxu2(m_row, v[i].w & 0x7FFF7FFFu);
+        }
+        if (kColRht) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                double y[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t w = (c >> 1) == 0 ? v[i].x : (c >> 1) == 1 ? v[i].y
+                                     : (c >> 1) == 2 ? v[i].z : v[i].w;
+                    const uint32_t b = (c & 1) ? (w >> 16) : (w & 0xFFFFu);
+                    y[i] = bf16_signed_to_f64(b, (sign_mask >> i) & 1u);
+                }
+                fwht16(y);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) m_col = fmax(m_col, fabs(y[i]));
+            }
+        }
+    }
+    uint32_t a_row = max(m_row & 0xFFFFu, m_row >> 16) << 16;
+    uint32_t a_col = kColRht ? __float_as_uint(__double2float_rn(m_col)) : 0u;
+    a_row = __reduce_max_sync(0xFFFFFFFFu, a_row);
+    a_col = __reduce_max_sync(0xFFFFFFFFu, a_col);
+    __shared__ uint32_t red[2][8];
+    if (lane == 0) {
+        red[0][warp] = a_row;
+        red[1][warp] = a_col;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t r = 0, c = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            r = max(r, red[0][w]);
+            c = max(c, red[1][w]);
+        }
+        if (r) atomicMax(words + 0, r);
+        if (kColRht && c) atomicMax(words + 1, c);
+    }
+}
+
+// ============================================================================
+// Shared helpers of the quantize kernels.
+// ============================================================================
+__device__ __forceinline__ bool finite_bits(uint32_t b) { return (b & 0x7FFFFFFFu) < 0x7F800000u; }
+
+// Eight values -> packed codes with RNE or SR (element index e0 .. e0+7 of the
+// quantized tensor, e0 % 8 == 0).
+__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float inv, bool sr,
+                                            uint64_t seed, uint32_t stream, uint64_t e0) {
+    float q[8];
+    if (!sr) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
+    } else {
+        const Philox4 p = sr_draws8(seed, stream, e0 >> 3);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = sr_e2m1_value(__fmul_rn(v[i], inv), draw16(p, i));
+    }
+    return e2m1x8_rn(q);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& w, float (&v)[8]) {
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x);
+    v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z);
+    v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+
+__device__ __forceinline__ float absmax8(const uint4& w) {
+    uint32_t m = __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                          __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+    return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+}
+
+// Reads the tensor amax words; false (and the error recorded) if non-finite.
+__device__ __forceinline__ bool load_tensor_scales(const QuantParams& p, TensorScale& tr,
+                                                   TensorScale& tc) {
+    const uint32_t wr = p.amax_words[0];
+    const uint32_t wc = p.col_rht ? p.amax_words[1] : wr;
+    const bool ok = finite_bits(wr) && finite_bits(wc);
+    const bool first = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
+    if (!ok) {
+        if (first) {
+            set_status(p.status, kStatusNonFinite);
+            if (p.row_g) *p.row_g = __uint_as_float(0x7FC00000u);
+            if (p.col_g) *p.col_g = __uint_as_float(0x7FC00000u);
+        }
+        return false;
+    }
+    tr = tensor_scale_from_amax(__uint_as_float(wr));
+    tc = tensor_scale_from_amax(__uint_as_float(wc));
+    if (first) {
+        if (p.row_g) *p.row_g = tr.g;
+        if (p.col_g) *p.col_g = tc.g;
+    }
+    return true;
+}
+
+// ============================================================================
+// Row orientation only, 1x16 blocks: every lane owns 8 consecutive elements
+// (one 16-byte load); a block is a lane pair.  Grid-stride over 8-chunks.
+// ============================================================================
+__global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
+    TensorScale tr, tc;
+    if (!load_tensor_scales(p, tr, tc)) return;
+    const int64_t cpr = p.cols >> 3;  // 8-chunks per row (even)
+    const int64_t nchunks = p.rows * cpr;
+    const int64_t katoms = (p.cols / 16 + 3) >> 2;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // warp-uniform trip count: every lane takes part in the pair shuffle
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < nchunks;
+         base += stride) {
+        const int64_t q = base + (threadIdx.x & 31);
+        const bool valid = q < nchunks;
+        const uint4 w = valid ? ld_stream_v4(p.x + q * 8) : make_uint4(0, 0, 0, 0);
+        float amax = absmax8(w);
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        uint32_t s;
+        float inv;
+        block_scale(amax, tr, s, inv);
+        float v[8];
+        unpack8(w, v);
+        const uint32_t codes = encode8(v, inv, p.row_sr, p.seed, 0u, (uint64_t)q * 8);
+        if (valid) {
+            reinterpret_cast<uint32_t*>(p.row_data)[q] = codes;
+            if ((q & 1) == 0) {
+                const int64_t r = q / cpr, kb = (q % cpr) >> 1;
+                p.row_sf[sf_offset(r, kb, katoms)] = (uint8_t)s;
+            }
+        }
+    }
+}
+
+// ============================================================================
+// Tile kernel: a CTA loads a 64 x 128 bf16 tile once (registers + shared
+// memory) and writes the row orientation (from registers, lane pairs) and/or
+// the column orientation (from shared memory, one lane per column, two
+// 16-row chunks per lane).  k2D: 16x16 blocks, the tile scale is found by the
+// column pass and shared by both orientations.  kRht: 16-point RHT in fp64
+// down each column chunk before the column orientation is quantized.
+// ============================================================================
+constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;
+
+template <bool k2D, bool kRht>
+__global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
+    __shared__ __align__(16) uint16_t tile[kTR][kPitch];
+    __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
+    __shared__ float tile_inv[kTR / 16][kTC / 16];
+
+    TensorScale tr, tc;
+    if (!load_tensor_scales(p, tr, tc)) return;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t r0 = (int64_t)blockIdx.y * kTR, c0 = (int64_t)blockIdx.x * kTC;
+    const bool want_row = p.row_data != nullptr;
+    const bool want_col = p.col_data != nullptr;
+    const bool use_smem = want_col || k2D;
+
+    // ---- load: chunk q = k*256 + tid covers row q/16, columns (q%16)*8 .. +7
+    uint4 reg[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int q = k * 256 + tid;
+        const int lr = q >> 4, lc = (q & 15) * 8;
+        const int64_t r = r0 + lr, c = c0 + lc;
+        reg[k] = (r < p.rows && c < p.cols) ? ld_stream_v4(p.x + r * p.cols + c)
+                                            : make_uint4(0, 0, 0, 0);
+        if (use_smem) *reinterpret_cast<uint4*>(&tile[lr][lc]) = reg[k];
+    }
+    if (use_smem) __syncthreads();
+
+    // ---- column pass: lane -> column lc, chunks j0, j0+1 (16 rows each)
+    if (use_smem) {
+        const int lc = 32 * (warp & 3) + lane;
+        const int j0 = 2 * (warp >> 2);
+        const int64_t c = c0 + lc;
+        const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
+        uint32_t out[4];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int j = j0 + jj;
+            float y[16];
+            if (kRht) {
+                double d[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    d[i] = bf16_signed_to_f64(tile[16 * j + i][lc], (p.sign_mask >> i) & 1u);
+                fwht16(d);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) y[i] = __double2float_rn(d[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) y[i] = __uint_as_float((uint32_t)tile[16 * j + i][lc] << 16);
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
+            uint32_t s;
+            float inv;
+            if (k2D) {
+                // 16x16 tile: 16 lanes hold its 16 columns
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+                block_scale(amax, tc, s, inv);
+                if ((lane & 15) == 0) {
+                    tile_s[j][lc >> 4] = s;
+                    tile_inv[j][lc >> 4] = inv;
+                }
+            } else {
+                block_scale(amax, tc, s, inv);
+            }
+            if (want_col) {
+                const uint64_t e0 = (uint64_t)c * (uint64_t)p.rows + (uint64_t)(r0 + 16 * j);
+                float lo8[8], hi8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    lo8[i] = y[i];
+                    hi8[i] = y[8 + i];
+                }
+                out[2 * jj] = encode8(lo8, inv, p.col_sr, p.seed, 1u, e0);
+                out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, p.seed, 1u, e0 + 8);
+                if (c < p.cols && r0 + 16 * j < p.rows)
+                    p.col_sf[sf_offset(c, (r0 >> 4) + j, katoms_c)] = (uint8_t)s;
+            }
+        }
+        if (want_col && c < p.cols) {
+            uint8_t* base = p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j0) >> 1);
+            if (r0 + 16 * j0 < p.rows)
+                *reinterpret_cast<uint2*>(base) = make_uint2(out[0], out[1]);
+            if (r0 + 16 * (j0 + 1) < p.rows)
+                *reinterpret_cast<uint2*>(base + 8) = make_uint2(out[2], out[3]);
+        }
+        if (k2D) __syncthreads();
+    }
+
+    // ---- row pass from registers: a 16-block is a lane pair
+    if (want_row) {
+        const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int q = k * 256 + tid;
+            const int lr = q >> 4, lc = (q & 15) * 8;
+            const int64_t r = r0 + lr, c = c0 + lc;
+            uint32_t s;
+            float inv;
+            if (k2D) {
+                s = tile_s[lr >> 4][lc >> 4];
+                inv = tile_inv[lr >> 4][lc >> 4];
+            } else {
+                float amax = absmax8(reg[k]);
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+                block_scale(amax, tr, s, inv);
+            }
+            float v[8];
+            unpack8(reg[k], v);
+            const uint32_t codes =
+                encode8(v, inv, p.row_sr, p.seed, 0u, (uint64_t)r * (uint64_t)p.cols + (uint64_t)c);
+            if (r < p.rows && c < p.cols) {
+                *reinterpret_cast<uint32_t*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
+                if ((lc & 15) == 0) p.row_sf[sf_offset(r, c >> 4, katoms_r)] = (uint8_t)s;
+            }
+        }
+    }
+}
+
+// ============================================================================
+// Zero fill of the scale padding: rows [rows, pad128(rows)) and 16-blocks
+// [nb, pad4(nb)) of an operand with `rows` rows and `nb` 16-blocks per row.
+// ============================================================================
+__global__ void sf_pad_kernel(uint8_t* __restrict__ sf, int64_t rows, int64_t nb) {
+    const int64_t prow = (rows + 127) / 128 * 128, pnb = (nb + 3) / 4 * 4;
+    const int64_t katoms = pnb / 4;
+    const int64_t total = prow * pnb;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / pnb, kb = i % pnb;
+        if (r >= rows || kb >= nb) sf[sf_offset(r, kb, katoms)] = 0;
+    }
+}
+
+// ============================================================================
+// Standalone RHT.  axis 1: a thread transforms 16 contiguous elements.
+// axis 0: a thread transforms 8 columns x 16 rows (like the amax unit).
+// ============================================================================
+__global__ void __launch_bounds__(256) rht_axis1_kernel(const uint16_t* __restrict__ x, float* __restrict__ y,
+                                                       int64_t nchunks, uint32_t sign_mask) {
+    for (int64_t ch = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ch < nchunks;
+         ch += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 a = ld_stream_v4(x + ch * 16), b = ld_stream_v4(x + ch * 16 + 8);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        double d[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            d[i] = bf16_signed_to_f64((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu),
+                                      (sign_mask >> i) & 1u);
+        fwht16(d);
+        float4* out = reinterpret_cast<float4*>(y + ch * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            out[i] = make_float4(__double2float_rn(d[4 * i]), __double2float_rn(d[4 * i + 1]),
+                                 __double2float_rn(d[4 * i + 2]), __double2float_rn(d[4 * i + 3]));
+    }
+}
+
+__global__ void __launch_bounds__(256) rht_axis0_kernel(const uint16_t* __restrict__ x, float* __restrict__ y,
+                                                       int64_t rows, int64_t cols, uint32_t sign_mask) {
+    const int64_t cunits = cols / 8;
+    const int64_t units = (rows / 16) * cunits;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r0 = (u / cunits) * 16, c0 = (u % cunits) * 8;
+        uint4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = ld_stream_v4(x + (r0 + i) * cols + c0);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {  // columns 4*half .. 4*half+3
+            float o[16][4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int c = 4 * half + cc;
+                double d[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t w = (c >> 1) == 0 ? v[i].x : (c >> 1) == 1 ? v[i].y
+                                     : (c >> 1) == 2 ? v[i].z : v[i].w;
+                    d[i] = bf16_signed_to_f64((c & 1) ? (w >> 16) : (w & 0xFFFFu), (sign_mask >> i) & 1u);
+                }
+                fwht16(d);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i][cc] = __double2float_rn(d[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<float4*>(y + (r0 + i) * cols + c0 + 4 * half) =
+                    make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
+        }
+    }
+}
+
+// ============================================================================
+// Launchers
+// ============================================================================
+static int grid_for(int64_t work_items, int per_block, int sm_count, int blocks_per_sm) {
+    int64_t g = (work_items + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)sm_count * blocks_per_sm;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return (int)g;
+}
+
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
+                        uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st) {
+    const int64_t units = ((rows + 15) / 16) * ((cols + 255) / 256);
+    const int grid = grid_for(units, 8, sm_count, 8);
+    if (col_rht)
+        amax_kernel<true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words);
+    else
+        amax_kernel<false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const QuantParams& p, int sm_count, cudaStream_t st) {
+    const int64_t nchunks = p.rows * (p.cols / 8);
+    const int grid = grid_for(nchunks, 256, sm_count, 8);
+    quant_rows_kernel<<<grid, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, cudaStream_t st) {
+    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
+    if (two_d)
+        quant_tile_kernel<true, false><<<grid, 256, 0, st>>>(p);
+    else if (p.col_rht && p.col_data)
+        quant_tile_kernel<false, true><<<grid, 256, 0, st>>>(p);
+    else
+        quant_tile_kernel<false, false><<<grid, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st) {
+    if (rows % 128 == 0 && nb % 4 == 0) return cudaSuccess;
+    const int64_t total = (rows + 127) / 128 * 128 * ((nb + 3) / 4 * 4);
+    sf_pad_kernel<<<grid_for(total, 256, sm_count, 4), 256, 0, st>>>(sf, rows, nb);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rht(const uint16_t* x, float* y, int64_t rows, int64_t cols, int axis,
+                       uint32_t sign_mask, int sm_count, cudaStream_t st) {
+    if (axis == 1) {
+        const int64_t n = rows * cols / 16;
+        rht_axis1_kernel<<<grid_for(n, 256, sm_count, 8), 256, 0, st>>>(x, y, n, sign_mask);
+    } else {
+        const int64_t n = (rows / 16) * (cols / 8);
+        rht_axis0_kernel<<<grid_for(n, 256, sm_count, 4), 256, 0, st>>>(x, y, rows, cols, sign_mask);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4
