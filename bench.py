@@ -1,0 +1,444 @@
+"""Benchmark of the NVFP4 linear-layer training step on B200.
+
+One step = one pass of the whole hot path over one batch: quantize X (rows RNE +
+RHT columns), W (16x16, both orientations), dY (rows SR + RHT columns SR), and the
+fprop / dgrad / wgrad block-scaled FP4 GEMMs, on the 12B-class MLP up-projection
+(tokens M=8192, hidden K=5120, FFN N=20480), synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is device-timed whole-job TFLOP/s of the
+three GEMMs per step time (inputs resident in HBM); `e2e` is the same metric with
+the inputs copied from pinned host memory and the outputs read back every step.
+N > 1 runs independent replicas (weak scaling): the step has no exchange.
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 linear fprop+dgrad+wgrad TFLOPS and quantize GB/s, % of B200 roofline"
+WORKLOAD = "12B-class MLP up-projection training step (fprop+dgrad+wgrad), M=8192 K=5120 N=20480"
+M, K, N = 8192, 5120, 20480
+FLOPS_PER_GEMM = 2.0 * M * K * N
+FLOPS_PER_STEP = 3 * FLOPS_PER_GEMM
+KERNELS_PER_STEP = 9  # 2 amax + 2 quantize (fprop), 1 + 1 (dgrad), 3 GEMMs
+FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
+
+
+def env_rank():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(
+        os.environ.get("LOCAL_RANK", "0"))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while timing."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from nvfp4_bit_quantized_amax_b200 import capi
+    from nvfp4_bit_quantized_amax_b200 import synthetic as syn
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    capi.load()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # synthetic inputs (seeded per rank: every replica its own batch)
+    Xb, Wb, dYb = syn.mlp_inputs(M, K, N, seed=1000 * rank)
+
+    def to_dev(b):
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    X, W, dY = to_dev(Xb), to_dev(Wb), to_dev(dYb)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(capi.linear_workspace_bytes(M, K, N), dtype=torch.uint8, device=dev)
+    signs = syn.rht_signs(rank)
+    seed = 20260 + rank
+
+    def step(x=X, w=W, dy=dY):
+        capi.nvfp4_linear_fprop(x, w, Y, signs, ws)
+        capi.nvfp4_linear_dgrad(dy, dX, seed, signs, ws)
+        capi.nvfp4_linear_wgrad(None, dW, M, seed, signs, ws)
+
+    def timed(fn, iters, warm):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(iters):
+            fn()
+        e.record(stream)
+        e.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+        return s.elapsed_time(e) / iters
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    # ---- the timed step (inputs resident in HBM; per-step working set ~1.6 GB >> L2)
+    with ClockSampler(local_rank) as clk:
+        ms = timed(step, args.steps, max(args.warmup, 3))
+    ms = max_over_ranks(ms)
+    assert capi.nvfp4_read_status(ws) == 0
+    value = world * FLOPS_PER_STEP / (ms * 1e-3) / 1e12
+
+    out = {}
+    if rank == 0 or True:
+        # ---- per-kernel timing on the same stream (each launch alone, back to back)
+        iters = max(10, min(50, args.steps))
+        ops = {w: capi.nvfp4_linear_operand(ws, M, K, N, w) for w in range(6)}
+        lib = capi.load()
+
+        def gemm(a, b, alpha, D, Mx, Nx, Kx):
+            va, vb = ops[a], ops[b]
+            return lambda: lib.nvfp4_gemm(va.data, va.scales, vb.data, vb.scales,
+                                          va.tensor_scale, vb.tensor_scale, alpha, Mx, Nx, Kx,
+                                          D.data_ptr(), None, None, stream.cuda_stream)
+
+        g_ms = {
+            "fprop": timed(gemm(capi.LIN_X_ROW, capi.LIN_W_ROW, 1.0, Y, M, N, K), iters, 3),
+            "dgrad": timed(gemm(capi.LIN_DY_ROW, capi.LIN_W_COL, 1.0, dX, M, K, N), iters, 3),
+            "wgrad": timed(gemm(capi.LIN_DY_COL, capi.LIN_X_COL, 1.0 / 16, dW, N, K, M), iters, 3),
+        }
+        qws = torch.empty(capi.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+        def tview(w):
+            v = ops[w]
+            return (v.data, v.scales, v.tensor_scale)
+
+        def quant(x, bm, rr, cr, rht, row_w, col_w):
+            r = capi.Tensor(*tview(row_w), 0, 0) if row_w is not None else None
+            c = capi.Tensor(*tview(col_w), 0, 0) if col_w is not None else None
+            sgn = np.ascontiguousarray(signs)
+            opts = capi.QuantizeOpts(bm, rr, cr, seed, int(rht), sgn.ctypes.data)
+            import ctypes
+            args_ = (ctypes.c_void_p(x.data_ptr()), x.shape[0], x.shape[1], ctypes.byref(opts),
+                     ctypes.byref(r) if r is not None else None,
+                     ctypes.byref(c) if c is not None else None,
+                     ctypes.c_void_p(qws.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+            return lambda: lib.nvfp4_quantize_2d(*args_)
+
+        q_ms = {
+            "X_row+col_rht": (timed(quant(X, 0, 0, 0, True, capi.LIN_X_ROW, capi.LIN_X_COL), iters, 3), M * K),
+            "W_16x16_both": (timed(quant(W, 1, 0, 0, False, capi.LIN_W_ROW, capi.LIN_W_COL), iters, 3), N * K),
+            "dY_row_sr+col_rht_sr": (timed(quant(dY, 0, 1, 1, True, capi.LIN_DY_ROW, capi.LIN_DY_COL), iters, 3), M * N),
+        }
+        peaks, peak_kind = load_peaks()
+        fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+        gemm_avg_ms = sum(g_ms.values()) / 3
+        achieved = FLOPS_PER_GEMM / (gemm_avg_ms * 1e-3) / 1e12
+        # dual-orientation quantize: amax read 2 B + quantize read 2 B + 2 x (0.5 + 1/16) B written
+        q_bytes_per_el = 2.0 + 2.0 + 2 * (0.5 + 1.0 / 16)
+        quant = {k: {"ms": round(v[0], 4),
+                     "GB/s": round(q_bytes_per_el * v[1] / (v[0] * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(q_bytes_per_el * v[1] / (v[0] * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+                 for k, v in q_ms.items()}
+        q_total_bytes = sum(q_bytes_per_el * v[1] for v in q_ms.values())
+        q_total_ms = sum(v[0] for v in q_ms.values())
+        out["roofline"] = {
+            "bound": "tensor", "kernel": "gemm_nvf4_kernel (fprop/dgrad/wgrad average)",
+            "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / fp4_peak, 4), "traffic": args.traffic,
+            "peak_source": f"{peak_kind}: FP4 = {FP4_OVER_BF16:g} x bf16 burst "
+                           f"{peaks['bf16_tflops']} TFLOP/s (nominal 9 / 2.25 PFLOP/s ratio)",
+        }
+        out["kernels"] = {
+            "gemm_ms": {k: round(v, 4) for k, v in g_ms.items()},
+            "gemm_tflops": {k: round(FLOPS_PER_GEMM / (v * 1e-3) / 1e12, 1) for k, v in g_ms.items()},
+            "quantize": quant,
+            "quantize_GB/s": round(q_total_bytes / (q_total_ms * 1e-3) / 1e9, 1),
+            "quantize_frac_hbm": round(q_total_bytes / (q_total_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+            "hbm_peak_GB/s": peaks["hbm_gbs"],
+        }
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        hX = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        hW = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        hdY = torch.from_numpy(dYb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        hY = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        hdX = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+        hdW = torch.empty((N, K), dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            X.copy_(hX, non_blocking=True)
+            W.copy_(hW, non_blocking=True)
+            dY.copy_(hdY, non_blocking=True)
+            step()
+            hY.copy_(Y, non_blocking=True)
+            hdX.copy_(dX, non_blocking=True)
+            hdW.copy_(dW, non_blocking=True)
+
+        e_iters = max(3, min(10, args.steps))
+        e_ms = max_over_ranks(timed(e2e_step, e_iters, 2))
+        h2d = 2 * (M * K + N * K + M * N)
+        e2e = {"value": round(world * FLOPS_PER_STEP / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+               "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic (seeded: X~N(0,1), W~N(0,0.02^2), dY~N(0,1e-3^2), bf16)",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N,
+                   "global_batch_tokens": M * world,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (629 MB bf16 inputs, ~1.6 GB touched per step)",
+                   "recipe": "X,dY 1x16; W 16x16; SR on dY; 16-pt RHT on wgrad operands"},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    line.update(out)
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- oracle
+def oracle_sample_step(Ms, Ks, Ns, nthreads=0):
+    """The same step (same recipe, same distributions) on a reduced shape, run by the
+    CPU oracle: six quantizations and three fp64 GEMMs.  Returns seconds."""
+    from nvfp4_bit_quantized_amax_b200 import synthetic as syn
+    from oracle import oracle as ora
+
+    X, W, dY = syn.mlp_inputs(Ms, Ks, Ns, seed=0)
+    s = syn.rht_signs(0)
+    t0 = time.perf_counter()
+    q = {}
+    for name, x, orient, rht, bm, rnd in (("xr", X, 0, 0, 0, 0), ("xc", X, 1, 1, 0, 0),
+                                          ("wr", W, 0, 0, 1, 0), ("wc", W, 1, 0, 1, 0),
+                                          ("dr", dY, 0, 0, 0, 1), ("dc", dY, 1, 1, 0, 1)):
+        p, sf, g, _ = ora.quantize(x, orient, rht, s, bm, rnd, 7, nthreads=nthreads)
+        q[name] = (p, sf, float(g))
+    for a, b, alpha in (("xr", "wr", 1.0), ("dr", "wc", 1.0), ("dc", "xc", 1.0 / 16)):
+        pa, sa, ga = q[a]
+        pb, sb, gb = q[b]
+        ora.gemm(pa, sa, pb, sb, alpha * ga * gb, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(budget_s=15.0):
+    cores = os.cpu_count() or 1
+    shape = (256, 256, 512)
+    t = oracle_sample_step(*shape)
+    reps = 1
+    # grow the sample until it is ~budget_s of CPU work (bounded)
+    while t * reps < budget_s / 4 and shape[0] < 1024:
+        shape = (shape[0] * 2, shape[1] * 2, shape[2] * 2)
+        t = oracle_sample_step(*shape)
+    flops = 3 * 2.0 * shape[0] * shape[1] * shape[2]
+    return {"value": round(flops / t / 1e12, 6), "unit": "TFLOPS", "cores": cores,
+            "kind": "oracle",
+            "sample": f"whole step (6 quantizations + 3 fp64 GEMMs) at M={shape[0]} K={shape[1]} "
+                      f"N={shape[2]} instead of 8192/5120/20480, same recipe and distributions; "
+                      f"{t:.1f} s on {cores} threads"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cores = os.cpu_count() or 1
+    shape = (256, 256, 512)
+    flops = 3 * 2.0 * shape[0] * shape[1] * shape[2]
+    for _ in range(max(args.warmup, 3)):
+        oracle_sample_step(*shape)
+    times = [oracle_sample_step(*shape) for _ in range(args.steps)]
+    per = sum(times) / len(times)
+    value = flops / per / 1e12
+    sample = (f"whole step at M={shape[0]} K={shape[1]} N={shape[2]} per timed step (same recipe "
+              f"and distributions as the 8192/5120/20480 workload)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "parallelism": "single"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_kernel(args):
+    """Single-kernel mode for profilers: quantize synthetic bf16 inputs of the given
+    shape, then launch one kernel `--steps` times.  --kernel gemm (M,N,K),
+    quant-x / quant-w / quant-dy (rows,cols): the three fused quantize passes."""
+    import torch
+
+    from nvfp4_bit_quantized_amax_b200 import capi
+    from nvfp4_bit_quantized_amax_b200 import synthetic as syn
+
+    dev = torch.device("cuda", 0)
+    dims = [int(v) for v in args.shape.split(",")]
+    signs = syn.rht_signs(0)
+
+    def to_dev(b):
+        return torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    def operand(rows, cols, seed):
+        x = to_dev(syn.normal_bf16((rows, cols), seed))
+        op = (torch.empty(capi.packed_bytes(rows, cols), dtype=torch.uint8, device=dev),
+              torch.empty(capi.scale_bytes(rows, cols), dtype=torch.uint8, device=dev),
+              torch.empty(1, dtype=torch.float32, device=dev))
+        ws = torch.empty(capi.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+        capi.nvfp4_quantize(x, 0, 0, 0, *op, ws)
+        return op
+
+    if args.kernel == "gemm":
+        Mk, Nk, Kk = dims
+        a, b = operand(Mk, Kk, 1), operand(Nk, Kk, 2)
+        D = torch.empty((Mk, Nk), dtype=torch.bfloat16, device=dev)
+        fn = lambda: capi.nvfp4_gemm(a[0], a[1], b[0], b[1], 1.0, Mk, Nk, Kk, D_bf16=D,
+                                     scale_a=a[2], scale_b=b[2])
+    else:
+        rows, cols = dims
+        x = to_dev(syn.normal_bf16((rows, cols), 3))
+        ws = torch.empty(capi.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+        def bufs(r, c):
+            return (torch.empty(capi.packed_bytes(r, c), dtype=torch.uint8, device=dev),
+                    torch.empty(capi.scale_bytes(r, c), dtype=torch.uint8, device=dev),
+                    torch.empty(1, dtype=torch.float32, device=dev))
+        ro, co = bufs(rows, cols), bufs(cols, rows)
+        bm, rr, cr, rht = {"quant-x": (0, 0, 0, 1), "quant-w": (1, 0, 0, 0),
+                           "quant-dy": (0, 1, 1, 1)}[args.kernel]
+        fn = lambda: capi.nvfp4_quantize_2d(x, bm, rr, cr, 5, rht, signs, ro, co, ws)
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel": args.kernel, "shape": dims, "launches": args.steps}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", default=None, choices=["gemm", "quant-x", "quant-w", "quant-dy"],
+                    help="profiler mode: launch one kernel kind only")
+    ap.add_argument("--shape", default="4096,8192,5120")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per GEMM launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+    rank, world, local_rank = env_rank()
+    if args.kernel:
+        run_kernel(args)
+    elif args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()
