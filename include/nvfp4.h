@@ -187,6 +187,28 @@ enum {
 int nvfp4_linear_operand(void* ws, int64_t M, int64_t K, int64_t N, int which,
                          nvfp4_tensor* out);
 
+/*
+ * nvfp4_quantize_noalloc -- nvfp4_quantize without the workspace argument, for
+ * callers that cannot allocate device memory (for example a plugin that is handed
+ * only its input and output buffers by a host framework owning every device
+ * allocation, or a real-time loop that must not allocate after start-up).
+ * The pages have no counterpart; this is a library convenience.
+ * Arguments, layouts, results and errors are those of nvfp4_quantize.  Its 64
+ * bytes of scratch (tensor amax words, status word) live in a static device array
+ * of NVFP4_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
+ * until exit; a call needing more than that would be refused with
+ * NVFP4_ERR_WORKSPACE.  The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  All calls share the array and each clears it on its stream
+ * before use: calls that overlap on the GPU (other streams, other threads) race.
+ * There is no status word to read back: an Inf/NaN input shows as a NaN
+ * tensor_scale.  It calls no allocator.
+ */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+int nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int block_mode,
+                           int rounding, uint64_t seed, uint8_t* packed, uint8_t* scales,
+                           float* tensor_scale, nvfp4_stream_t stream);
+
 /* Status word of a quantize or linear workspace (synchronizes `stream`, then
  * clears the word).  *status = NVFP4_OK or the first device error recorded.    */
 int nvfp4_read_status(void* workspace, int* status, nvfp4_stream_t stream);

@@ -26,7 +26,7 @@ EXPORTS = (
     "nvfp4_quantize", "nvfp4_quantize_2d", "nvfp4_rht", "nvfp4_gemm",
     "nvfp4_linear_workspace_bytes", "nvfp4_linear_fprop", "nvfp4_linear_dgrad",
     "nvfp4_linear_wgrad", "nvfp4_linear_operand", "nvfp4_read_status",
-    "nvfp4_status_string", "nvfp4_version",
+    "nvfp4_status_string", "nvfp4_version", "nvfp4_quantize_noalloc",
 )
 
 
@@ -77,6 +77,7 @@ def load(path: str = LIB_PATH):
         "nvfp4_read_status": (ci, [vp, C.POINTER(ci), vp]),
         "nvfp4_status_string": (C.c_char_p, [ci]),
         "nvfp4_version": (ci, []),
+        "nvfp4_quantize_noalloc": (ci, [vp, i64, i64, ci, ci, u64, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -137,6 +138,15 @@ def nvfp4_quantize(x, block_mode, rounding, seed, packed, scales, tensor_scale, 
     _check("nvfp4_quantize", load().nvfp4_quantize(
         _ptr(x), rows, cols, block_mode, rounding, seed, _ptr(packed), _ptr(scales),
         _ptr(tensor_scale), _ptr(workspace), _stream(stream)))
+
+
+def nvfp4_quantize_noalloc(x, block_mode, rounding, seed, packed, scales, tensor_scale,
+                           stream=None):
+    """nvfp4_quantize without a workspace (scratch in the library's static array)."""
+    rows, cols = x.shape
+    _check("nvfp4_quantize_noalloc", load().nvfp4_quantize_noalloc(
+        _ptr(x), rows, cols, block_mode, rounding, seed, _ptr(packed), _ptr(scales),
+        _ptr(tensor_scale), _stream(stream)))
 
 
 def make_tensor(data, scales, tensor_scale):
