@@ -5,17 +5,20 @@
 // fprop, dgrad and wgrad GEMMs of the NVFP4 linear layer all take this form
 // ("NVIDIA's 4-bit floating point pushes AI training limits", artiverse.ca).
 //
-// Design (one CTA = one 128 x BN output tile, 128 threads):
+// Design (one CTA = one 128 x BN output tile, 192 threads):
 //   warp 0 lane 0   TMA producer: A/B tiles (128-byte swizzled K-major boxes of
 //                   256 FP4 along K) and the matching 512-byte scale atoms
 //                   (bulk copies) into a STAGES-deep shared-memory ring.
-//   warp 1 lane 0   MMA issuer: copies the stage's scale atoms to TMEM with
-//                   tcgen05.cp (32x128b, replicated to the four lane quadrants),
-//                   then four tcgen05.mma kind::mxf4nvf4 block_scale (K = 64 each)
-//                   into the fp32 accumulator in TMEM; tcgen05.commit frees the
-//                   stage, and a final commit signals the epilogue.
-//   warps 0-3       epilogue: tcgen05.ld of their 32 accumulator lanes, scale by
-//                   alpha * gA * gB, store fp32 and/or bf16.
+//   warps 2-5       scale writers: copy each stage's scale atoms from shared memory
+//                   into a 4-deep ring of TMEM scale regions with tcgen05.st (each
+//                   warp its 32-lane quadrant, every quadrant a full copy), so the
+//                   tensor pipe spends no cycles on scale copies; after the last
+//                   k-tile the same warps run the epilogue: tcgen05.ld of their
+//                   quadrant, scale by alpha * gA * gB, store fp32 and/or bf16.
+//   warp 1 lane 0   MMA issuer: four tcgen05.mma kind::mxf4nvf4 block_scale
+//                   (K = 64 each) per stage into the fp32 accumulator in TMEM;
+//                   tcgen05.commit frees the stage and the scale region, and a
+//                   final commit signals the epilogue.
 // Every wait is bounded: after ~1 s the kernel records NVFP4_ERR_TIMEOUT in the
 // status word, stops issuing work, drains its own copies and frees TMEM.
 #include <cuda.h>
@@ -89,11 +92,21 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                      bar)
                  : "memory");
 }
-// Copy one 512-byte scale atom (32 lines of 16 bytes) into 4 TMEM columns, the
-// 32 lines replicated into each of the four 32-lane quadrants.
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
+// Write 16 / 32 consecutive TMEM columns of this warp's 32 lanes (lane i: row i of
+// the quadrant), then wait for the writes to land.
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
@@ -118,9 +131,6 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
 __device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
     return make_sdesc(saddr, 16, 1024, 2);
 }
-// Scale atom source of tcgen05.cp: unswizzled 8 x 16-byte core matrices, 128 B apart.
-__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) { return make_sdesc(saddr, 0, 128, 0); }
-
 // Instruction descriptor of kind::mxf4nvf4 block-scaled MMA: E2M1 A and B
 // (format 1), K-major both, UE4M3 scales (scale format 0), M = 128, N = BN,
 // K = 64 per instruction, dense.
@@ -139,6 +149,8 @@ struct __align__(1024) GemmSmem {
     uint8_t sfb[STAGES][(BN / 128) * 4 * 512];  // per 128-row group, 4 atoms
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
+    uint64_t sf_full[4];   // scale region r written (4 scale-writer warps arrive)
+    uint64_t sf_empty[4];  // scale region r free again (MMA commit)
     uint64_t acc_full;
     uint32_t tmem_base;
 };
@@ -148,17 +160,19 @@ struct TmemLayout {
     static constexpr int kSfaCols = 16;                   // 4 k-steps x 4 columns
     static constexpr int kSfbCols = 4 * 4 * (BN / 128);   // 4 k-steps x 4 columns per group
     static constexpr int kRegion = kSfaCols + kSfbCols;   // scales of one stage
-    static constexpr int kUsed = BN + 2 * kRegion;        // accumulator + two scale regions
+    static constexpr int kRegions = 4;                    // ring of scale regions
+    static constexpr int kUsed = BN + kRegions * kRegion; // accumulator + scale ring
     static constexpr int kAlloc = kUsed <= 32 ? 32 : kUsed <= 64 ? 64 : kUsed <= 128 ? 128
                                 : kUsed <= 256 ? 256 : 512;
 };
 
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(192, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p) {
     using Smem = GemmSmem<BN, STAGES>;
     using TL = TmemLayout<BN>;
+    constexpr int R = TL::kRegions;
     extern __shared__ uint8_t smem_raw[];
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -174,6 +188,10 @@ __global__ void __launch_bounds__(128, 1)
             mbar_init(smem_addr(&S.full[s]), 1);
             mbar_init(smem_addr(&S.empty[s]), 1);
         }
+        for (int r = 0; r < R; ++r) {
+            mbar_init(smem_addr(&S.sf_full[r]), 4);
+            mbar_init(smem_addr(&S.sf_empty[r]), 1);
+        }
         mbar_init(smem_addr(&S.acc_full), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -184,13 +202,12 @@ __global__ void __launch_bounds__(128, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    __shared__ int timed_out;
+    if (threadIdx.x == 0) timed_out = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-    __shared__ int timed_out;
-    if (threadIdx.x == 0) timed_out = 0;
-    __syncthreads();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -235,93 +252,132 @@ __global__ void __launch_bounds__(128, 1)
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = nvf4_idesc<BN>();
             for (int kt = 0; kt < KT; ++kt) {
-                const int s = kt % STAGES;
-                if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(kt / STAGES) & 1u)) {
+                const int s = kt % STAGES, r = kt % R;
+                if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(kt / STAGES) & 1u) ||
+                    !mbar_wait(smem_addr(&S.sf_full[r]), (uint32_t)(kt / R) & 1u)) {
                     timed_out = 1;
                     break;
                 }
                 tc_fence_after();
                 const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
                 const int nks = rem < 4 ? (int)rem : 4;
-                const uint32_t region = (uint32_t)(BN + (kt & 1) * TL::kRegion);
-                const uint32_t t_sfa = tmem + region;
-                const uint32_t t_sfb = tmem + region + TL::kSfaCols;
+                const uint32_t t_sfa = tmem + (uint32_t)(BN + r * TL::kRegion);
+                const uint32_t t_sfb = t_sfa + TL::kSfaCols;
                 const uint32_t a_base = smem_addr(S.a[s]), b_base = smem_addr(S.b[s]);
-                for (int j = 0; j < nks; ++j) {
-                    tc_cp_sf(t_sfa + 4 * j, sf_desc(smem_addr(S.sfa[s] + j * 512)));
-                    for (int g = 0; g < BN / 128; ++g)
-                        tc_cp_sf(t_sfb + 4 * (BN / 128) * j + 4 * g,
-                                 sf_desc(smem_addr(S.sfb[s] + g * 2048 + j * 512)));
-                }
                 for (int j = 0; j < nks; ++j) {
                     tc_mma_nvf4(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
                                 idesc, t_sfa + 4 * j, t_sfb + 4 * (BN / 128) * j,
                                 (kt > 0 || j > 0) ? 1u : 0u);
                 }
                 tc_commit(smem_addr(&S.empty[s]));
+                tc_commit(smem_addr(&S.sf_empty[r]));
             }
             tc_commit(smem_addr(&S.acc_full));
         }
         __syncwarp();
-    }
-
-    // ---------------------------------------------------- epilogue (all warps)
-    const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), 0);
-    tc_fence_after();
-    __syncwarp();
-    if (!acc_ok) timed_out = 1;
-    const bool bad = *(volatile int*)&timed_out != 0;
-    float alpha = p.alpha;
-    if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
-    if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
-    const int64_t row = m0 + warp * 32 + lane;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-            "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-              "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-              "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-              "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-              "=r"(r[31])
-            : "r"(taddr));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (bad || row >= p.M) continue;
-        const int64_t col0 = n0 + c * 32;
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const int64_t col = col0 + 8 * g;
-            if (col >= p.N) break;
-            if (p.D_f32) {
-                float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
-                d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
-                d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+    } else {
+        // ---------------------------------------------------- scale writers
+        // TMEM quadrant q = warp % 4 (lanes 32q .. 32q+31).  Scale atom j of a
+        // stage holds, in 16-byte line l, the 4-block scales of rows l, l+32, l+64,
+        // l+96; lane l of every quadrant gets line l in 4 consecutive columns, the
+        // layout the block-scaled MMA reads (row l + 32i in column i).
+        const int q = warp & 3;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        for (int kt = 0; kt < KT; ++kt) {
+            const int s = kt % STAGES, r = kt % R;
+            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(kt / STAGES) & 1u) ||
+                (kt >= R && !mbar_wait(smem_addr(&S.sf_empty[r]), ((uint32_t)(kt / R) & 1u) ^ 1u))) {
+                timed_out = 1;
+                break;
             }
-            if (p.D_bf16) {
-                uint4 w;
-                __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * g], v[8 * g + 1]);
-                __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * g + 2], v[8 * g + 3]);
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * g + 4], v[8 * g + 5]);
-                __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * g + 6], v[8 * g + 7]);
-                w.x = *reinterpret_cast<uint32_t*>(&h0);
-                w.y = *reinterpret_cast<uint32_t*>(&h1);
-                w.z = *reinterpret_cast<uint32_t*>(&h2);
-                w.w = *reinterpret_cast<uint32_t*>(&h3);
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D_bf16) + row * p.N + col) = w;
+            tc_fence_after();  // the MMAs that read this region before are complete
+            const uint32_t col = (uint32_t)(BN + r * TL::kRegion);
+            uint32_t v[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 w = *reinterpret_cast<const uint4*>(S.sfa[s] + j * 512 + lane * 16);
+                v[4 * j] = w.x; v[4 * j + 1] = w.y; v[4 * j + 2] = w.z; v[4 * j + 3] = w.w;
+            }
+            tc_st16(lane_base + col, v);
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h) {  // 16 columns per group pair of k-steps
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    // column order of the B scales: k-step j, group g -> 4*(BN/128)*j + 4*g
+                    const int idx = h * 4 + jj;            // 0 .. 4*(BN/128)-1
+                    const int j = idx / (BN / 128), g = idx % (BN / 128);
+                    const uint4 w = *reinterpret_cast<const uint4*>(S.sfb[s] + g * 2048 + j * 512 + lane * 16);
+                    v[4 * jj] = w.x; v[4 * jj + 1] = w.y; v[4 * jj + 2] = w.z; v[4 * jj + 3] = w.w;
+                }
+                tc_st16(lane_base + col + TL::kSfaCols + 16 * h, v);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&S.sf_full[r]));
+        }
+        __syncwarp();
+
+        // ---------------------------------------------------- epilogue
+        const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), 0);
+        tc_fence_after();
+        __syncwarp();
+        if (!acc_ok) timed_out = 1;
+        const bool bad = *(volatile int*)&timed_out != 0;
+        float alpha = p.alpha;
+        if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
+        if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
+        const int64_t row = m0 + q * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            const uint32_t taddr = lane_base + (uint32_t)(c * 32);
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+                "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                  "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                  "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+                  "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+                  "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+                  "=r"(r[31])
+                : "r"(taddr));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            if (bad || row >= p.M) continue;
+            const int64_t col0 = n0 + c * 32;
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int64_t col = col0 + 8 * g;
+                if (col >= p.N) break;
+                if (p.D_f32) {
+                    float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
+                    d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
+                    d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+                }
+                if (p.D_bf16) {
+                    uint4 w;
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * g], v[8 * g + 1]);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * g + 2], v[8 * g + 3]);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * g + 4], v[8 * g + 5]);
+                    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * g + 6], v[8 * g + 7]);
+                    w.x = *reinterpret_cast<uint32_t*>(&h0);
+                    w.y = *reinterpret_cast<uint32_t*>(&h1);
+                    w.z = *reinterpret_cast<uint32_t*>(&h2);
+                    w.w = *reinterpret_cast<uint32_t*>(&h3);
+                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D_bf16) + row * p.N + col) = w;
+                }
             }
         }
     }
+    __syncthreads();
     if (threadIdx.x == 0 && *(volatile int*)&timed_out) set_status(p.status, kStatusTimeout);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"((uint32_t)TL::kAlloc)
                      : "memory");
@@ -371,7 +427,7 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, cudaStream_t st) {
         configured = true;
     }
     const dim3 grid((unsigned)((p.N + BN - 1) / BN), (unsigned)((p.M + kBM - 1) / kBM));
-    gemm_nvf4_kernel<BN, STAGES><<<grid, 128, smem, st>>>(ma, mb, p);
+    gemm_nvf4_kernel<BN, STAGES><<<grid, 192, smem, st>>>(ma, mb, p);
     return cudaGetLastError();
 }
 
