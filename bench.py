@@ -246,6 +246,11 @@ def run_ours(args, rank, world, local_rank):
             "hbm_peak_GB/s": peaks["hbm_gbs"],
         }
 
+    # ---- mixture-of-experts expert layer (64 experts, Zipf(1.1) top-4 routing)
+    if not args.no_moe:
+        out["moe"] = moe_step_bench(capi, syn, dev, stream, timed, max_over_ranks, world,
+                                    iters=max(3, min(20, args.steps // 5)))
+
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
@@ -297,6 +302,51 @@ def run_ours(args, rank, world, local_rank):
     }
     line.update(out)
     print(json.dumps(line), flush=True)
+
+
+def moe_step_bench(capi, syn, dev, stream, timed, max_over_ranks, world, iters):
+    """Expert layer of the MoE config: gather routed token rows, per-expert NVFP4
+    fprop / dgrad / wgrad, combine the routed input gradients.  Useful FLOPs count
+    the routed tokens only (padding rows excluded)."""
+    import torch
+    s = syn.MOE
+    E, K, N, T, k = s["experts"], s["hidden"], s["ffn"], s["tokens"], s["topk"]
+    d = syn.moe_inputs(T, E, K, N, k, s["zipf_s"], seed=0)
+    rows = int(d["group_rows"].sum())
+
+    def to_dev(b):
+        return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x_tok = to_dev(d["X"])
+    W = to_dev(d["W"].reshape(E * N, K)).view(E, N, K)
+    dY = to_dev(d["dY"])
+    row_src = torch.from_numpy(d["row_src"]).to(dev)
+    slots = torch.from_numpy(d["slots"]).to(dev)
+    X_perm = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
+    Y = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
+    dX_tok = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((E, N, K), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(capi.moe_workspace_bytes(d["group_rows"], K, N), dtype=torch.uint8, device=dev)
+    signs = syn.rht_signs(0)
+
+    def step():
+        capi.nvfp4_moe_gather(x_tok, row_src, X_perm)
+        capi.nvfp4_moe_linear_fprop(X_perm, W, Y, d["group_rows"], signs, ws)
+        capi.nvfp4_moe_linear_dgrad(dY, dX, d["group_rows"], 7, signs, ws)
+        capi.nvfp4_moe_combine(dX, slots, dX_tok)
+        capi.nvfp4_moe_linear_wgrad(dW, d["group_rows"], 7, signs, ws)
+
+    ms = max_over_ranks(timed(step, iters, 3))
+    useful = 3 * 2.0 * T * k * K * N
+    padded = 3 * 2.0 * rows * K * N
+    return {"workload": "MoE expert layer: 64 experts, hidden 2048, FFN 1024, 16384 tokens, "
+                        "top-4 of Zipf(1.1)",
+            "ms_per_step": round(ms, 4),
+            "useful_tflops": round(world * useful / (ms * 1e-3) / 1e12, 1),
+            "executed_tflops_incl_padding": round(world * padded / (ms * 1e-3) / 1e12, 1),
+            "routed_rows": T * k, "padded_rows": rows,
+            "group_rows_max_min": [int(d["group_rows"].max()), int(d["group_rows"].min())]}
 
 
 # --------------------------------------------------------------------------- oracle
@@ -427,6 +477,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-moe", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per GEMM launch from an ncu capture of this kernel")

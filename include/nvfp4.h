@@ -175,6 +175,45 @@ int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N
 int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N, uint64_t seed,
                        const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
+/*
+ * Mixture-of-experts expert layer in NVFP4.  Only the expert weight-GEMMs run in FP4
+ * in the models the pages describe ("Nemotron NVFP4" explainer, "The model underneath"
+ * and "The honest part"); each expert is a linear layer with its own tensor scales and
+ * the same recipe as above.
+ *   Token rows are permuted into expert-contiguous segments: expert e owns rows
+ *   [off_e, off_e + group_rows[e]) of the permuted buffers (off_e = prefix sum), with
+ *   group_rows[e] a multiple of 64 (the routed tokens followed by zero rows).
+ *   group_rows: HOST array of E entries (0 allowed: the expert is skipped).
+ *   W [E][N][K] and dW [E][N][K] bf16; X_perm [sum][K], Y_perm / dY_perm [sum][N],
+ *   dX_perm [sum][K].  Expert e draws stochastic rounding with seed + e.
+ *   ws: nvfp4_moe_workspace_bytes() bytes; it holds one linear workspace per expert
+ *   (nvfp4_moe_expert_workspace gives expert e's, for nvfp4_linear_operand and
+ *   nvfp4_read_status).
+ */
+size_t nvfp4_moe_workspace_bytes(const int64_t* group_rows, int E, int64_t K, int64_t N);
+int nvfp4_moe_expert_workspace(void* ws, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                               int expert, void** expert_ws, size_t* expert_ws_bytes);
+int nvfp4_moe_linear_fprop(const void* X_perm, const void* W, void* Y_perm,
+                           const int64_t* group_rows, int E, int64_t K, int64_t N,
+                           const int8_t* rht_signs, void* ws, size_t ws_bytes,
+                           nvfp4_stream_t stream);
+int nvfp4_moe_linear_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
+                           int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
+                           size_t ws_bytes, nvfp4_stream_t stream);
+int nvfp4_moe_linear_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                           uint64_t seed, const int8_t* rht_signs, void* ws, size_t ws_bytes,
+                           nvfp4_stream_t stream);
+/*
+ * nvfp4_moe_gather: dst[i] = src[row_src[i]] for rows of `cols` bf16 (row_src device
+ * int32 [rows]; -1 writes a zero row).  cols % 8 == 0.
+ * nvfp4_moe_combine: dst[t] = bf16(sum over j < topk of src[slots[t*topk + j]]) with an
+ * fp32 sum in j order (slots device int32 [tokens][topk]; -1 entries are skipped).
+ */
+int nvfp4_moe_gather(const void* src, const int32_t* row_src, int64_t rows, int64_t cols,
+                     void* dst, nvfp4_stream_t stream);
+int nvfp4_moe_combine(const void* src, const int32_t* slots, int64_t tokens, int topk,
+                      int64_t cols, void* dst, nvfp4_stream_t stream);
+
 /* Views of the quantized operands a linear workspace holds (no device access). */
 enum {
     NVFP4_LIN_X_ROW = 0,  /* X,   M x K, 1x16 RNE                 */

@@ -27,6 +27,8 @@ EXPORTS = (
     "nvfp4_linear_workspace_bytes", "nvfp4_linear_fprop", "nvfp4_linear_dgrad",
     "nvfp4_linear_wgrad", "nvfp4_linear_operand", "nvfp4_read_status",
     "nvfp4_status_string", "nvfp4_version", "nvfp4_quantize_noalloc",
+    "nvfp4_moe_workspace_bytes", "nvfp4_moe_expert_workspace", "nvfp4_moe_linear_fprop",
+    "nvfp4_moe_linear_dgrad", "nvfp4_moe_linear_wgrad", "nvfp4_moe_gather", "nvfp4_moe_combine",
 )
 
 
@@ -78,6 +80,14 @@ def load(path: str = LIB_PATH):
         "nvfp4_status_string": (C.c_char_p, [ci]),
         "nvfp4_version": (ci, []),
         "nvfp4_quantize_noalloc": (ci, [vp, i64, i64, ci, ci, u64, vp, vp, vp, vp]),
+        "nvfp4_moe_workspace_bytes": (sz, [vp, ci, i64, i64]),
+        "nvfp4_moe_expert_workspace": (ci, [vp, vp, ci, i64, i64, ci, C.POINTER(vp),
+                                            C.POINTER(sz)]),
+        "nvfp4_moe_linear_fprop": (ci, [vp, vp, vp, vp, ci, i64, i64, vp, vp, sz, vp]),
+        "nvfp4_moe_linear_dgrad": (ci, [vp, vp, vp, ci, i64, i64, u64, vp, vp, sz, vp]),
+        "nvfp4_moe_linear_wgrad": (ci, [vp, vp, ci, i64, i64, u64, vp, vp, sz, vp]),
+        "nvfp4_moe_gather": (ci, [vp, vp, i64, i64, vp, vp]),
+        "nvfp4_moe_combine": (ci, [vp, vp, i64, ci, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -219,6 +229,70 @@ def nvfp4_linear_operand(ws, M, K, N, which):
     _check("nvfp4_linear_operand", load().nvfp4_linear_operand(
         C.c_void_p(ws.data_ptr()), M, K, N, which, C.byref(t)))
     return t
+
+
+# ---- mixture of experts -----------------------------------------------------------
+def _rows(group_rows):
+    import numpy as np
+    g = np.ascontiguousarray(np.asarray(group_rows, dtype=np.int64))
+    return g, g.ctypes.data_as(C.c_void_p)
+
+
+def moe_workspace_bytes(group_rows, K, N):
+    g, gp = _rows(group_rows)
+    return load().nvfp4_moe_workspace_bytes(gp, len(g), K, N)
+
+
+def nvfp4_moe_expert_workspace(ws, group_rows, K, N, expert):
+    g, gp = _rows(group_rows)
+    p, n = C.c_void_p(), C.c_size_t()
+    _check("nvfp4_moe_expert_workspace", load().nvfp4_moe_expert_workspace(
+        C.c_void_p(ws.data_ptr()), gp, len(g), K, N, expert, C.byref(p), C.byref(n)))
+    return p.value, n.value
+
+
+def nvfp4_moe_linear_fprop(X_perm, W, Y_perm, group_rows, rht_signs, ws, stream=None):
+    g, gp = _rows(group_rows)
+    E, N, K = W.shape
+    keep, sp = _signs(rht_signs)
+    _check("nvfp4_moe_linear_fprop", load().nvfp4_moe_linear_fprop(
+        _ptr(X_perm), _ptr(W), _ptr(Y_perm), gp, E, K, N, sp, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep, g
+
+
+def nvfp4_moe_linear_dgrad(dY_perm, dX_perm, group_rows, seed, rht_signs, ws, stream=None):
+    g, gp = _rows(group_rows)
+    K = dX_perm.shape[1]
+    N = dY_perm.shape[1]
+    keep, sp = _signs(rht_signs)
+    _check("nvfp4_moe_linear_dgrad", load().nvfp4_moe_linear_dgrad(
+        _ptr(dY_perm), _ptr(dX_perm), gp, len(g), K, N, seed, sp, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep, g
+
+
+def nvfp4_moe_linear_wgrad(dW, group_rows, seed, rht_signs, ws, stream=None):
+    g, gp = _rows(group_rows)
+    E, N, K = dW.shape
+    keep, sp = _signs(rht_signs)
+    _check("nvfp4_moe_linear_wgrad", load().nvfp4_moe_linear_wgrad(
+        _ptr(dW), gp, E, K, N, seed, sp, _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    del keep, g
+
+
+def nvfp4_moe_gather(src, row_src, dst, stream=None):
+    rows, cols = dst.shape
+    _check("nvfp4_moe_gather", load().nvfp4_moe_gather(_ptr(src), _ptr(row_src), rows, cols,
+                                                       _ptr(dst), _stream(stream)))
+
+
+def nvfp4_moe_combine(src, slots, dst, stream=None):
+    tokens, topk = slots.shape
+    cols = dst.shape[1]
+    _check("nvfp4_moe_combine", load().nvfp4_moe_combine(_ptr(src), _ptr(slots), tokens, topk,
+                                                         cols, _ptr(dst), _stream(stream)))
 
 
 def nvfp4_read_status(workspace, stream=None):

@@ -143,6 +143,42 @@ int gemm_call(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint
     return cuda_status(launch_gemm(g, sms, st));
 }
 
+// ---------------------------------------------------------------- mixture of experts
+int moe_check(const int64_t* group_rows, int E, int64_t K, int64_t N) {
+    if (!group_rows || E < 1) return NVFP4_ERR_ARG;
+    if (K < 64 || N < 64 || K % 64 || N % 64) return NVFP4_ERR_SHAPE;
+    for (int e = 0; e < E; ++e)
+        if (group_rows[e] < 0 || group_rows[e] % 64) return NVFP4_ERR_SHAPE;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" size_t nvfp4_moe_workspace_bytes(const int64_t* group_rows, int E, int64_t K, int64_t N);
+
+namespace {
+// Calls fn(e, row offset, expert workspace, bytes) for every non-empty expert.
+template <class F>
+int moe_for_each(const int64_t* group_rows, int E, int64_t K, int64_t N, void* ws,
+                        size_t ws_bytes, F&& fn) {
+    int rc = moe_check(group_rows, E, K, N);
+    if (rc) return rc;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (ws_bytes < nvfp4_moe_workspace_bytes(group_rows, E, K, N)) return NVFP4_ERR_WORKSPACE;
+    int64_t row = 0;
+    size_t off = 0;
+    for (int e = 0; e < E; ++e) {
+        const int64_t m = group_rows[e];
+        if (m == 0) continue;
+        const size_t bytes = nvfp4_linear_workspace_bytes(m, K, N);
+        rc = fn(e, row, static_cast<uint8_t*>(ws) + off, bytes);
+        if (rc) return rc;
+        row += m;
+        off += (size_t)pad((int64_t)bytes, 256);
+    }
+    return NVFP4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -389,6 +425,88 @@ int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N
     // dW = (dY^T D H)(X^T D H)^T / 16: the rotation cancels, H H^T = 16 I
     return gemm_call(dc.data, dc.scales, xc.data, xc.scales, dc.tensor_scale, xc.tensor_scale,
                      1.0f / 16.0f, N, K, M, dW, nullptr, status, sms, st);
+}
+
+size_t nvfp4_moe_workspace_bytes(const int64_t* group_rows, int E, int64_t K, int64_t N) {
+    if (moe_check(group_rows, E, K, N)) return 0;
+    size_t total = 0;
+    for (int e = 0; e < E; ++e)
+        if (group_rows[e] > 0) total += (size_t)pad((int64_t)nvfp4_linear_workspace_bytes(group_rows[e], K, N), 256);
+    return total;
+}
+
+int nvfp4_moe_expert_workspace(void* ws, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                               int expert, void** expert_ws, size_t* expert_ws_bytes) {
+    int rc = moe_check(group_rows, E, K, N);
+    if (rc) return rc;
+    if (!ws || !expert_ws || !expert_ws_bytes || expert < 0 || expert >= E) return NVFP4_ERR_ARG;
+    size_t off = 0;
+    for (int e = 0; e < expert; ++e)
+        if (group_rows[e] > 0) off += (size_t)pad((int64_t)nvfp4_linear_workspace_bytes(group_rows[e], K, N), 256);
+    *expert_ws = static_cast<uint8_t*>(ws) + off;
+    *expert_ws_bytes = group_rows[expert] > 0 ? nvfp4_linear_workspace_bytes(group_rows[expert], K, N) : 0;
+    return NVFP4_OK;
+}
+
+int nvfp4_moe_linear_fprop(const void* X_perm, const void* W, void* Y_perm,
+                           const int64_t* group_rows, int E, int64_t K, int64_t N,
+                           const int8_t* rht_signs, void* ws, size_t ws_bytes,
+                           nvfp4_stream_t stream) {
+    if (!X_perm || !W || !Y_perm) return NVFP4_ERR_ARG;
+    return moe_for_each(group_rows, E, K, N, ws, ws_bytes, [&](int e, int64_t row, void* w, size_t b) {
+        return nvfp4_linear_fprop(static_cast<const uint16_t*>(X_perm) + row * K,
+                                  static_cast<const uint16_t*>(W) + (int64_t)e * N * K,
+                                  static_cast<uint16_t*>(Y_perm) + row * N, group_rows[e], K, N,
+                                  rht_signs, w, b, stream);
+    });
+}
+
+int nvfp4_moe_linear_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
+                           int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
+                           size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!dY_perm || !dX_perm) return NVFP4_ERR_ARG;
+    return moe_for_each(group_rows, E, K, N, ws, ws_bytes, [&](int e, int64_t row, void* w, size_t b) {
+        return nvfp4_linear_dgrad(static_cast<const uint16_t*>(dY_perm) + row * N,
+                                  static_cast<uint16_t*>(dX_perm) + row * K, group_rows[e], K, N,
+                                  seed + (uint64_t)e, rht_signs, w, b, stream);
+    });
+}
+
+int nvfp4_moe_linear_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                           uint64_t seed, const int8_t* rht_signs, void* ws, size_t ws_bytes,
+                           nvfp4_stream_t stream) {
+    if (!dW) return NVFP4_ERR_ARG;
+    return moe_for_each(group_rows, E, K, N, ws, ws_bytes, [&](int e, int64_t row, void* w, size_t b) {
+        (void)row;
+        return nvfp4_linear_wgrad(nullptr, static_cast<uint16_t*>(dW) + (int64_t)e * N * K,
+                                  group_rows[e], K, N, seed + (uint64_t)e, rht_signs, w, b, stream);
+    });
+}
+
+int nvfp4_moe_gather(const void* src, const int32_t* row_src, int64_t rows, int64_t cols,
+                     void* dst, nvfp4_stream_t stream) {
+    if (!src || !row_src || !dst) return NVFP4_ERR_ARG;
+    if (rows < 1 || cols < 8 || cols % 8) return NVFP4_ERR_SHAPE;
+    if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(row_src, 4)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    return cuda_status(launch_moe_gather(static_cast<const uint16_t*>(src), row_src,
+                                         static_cast<uint16_t*>(dst), rows, cols, sms,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_moe_combine(const void* src, const int32_t* slots, int64_t tokens, int topk,
+                      int64_t cols, void* dst, nvfp4_stream_t stream) {
+    if (!src || !slots || !dst || topk < 1) return NVFP4_ERR_ARG;
+    if (tokens < 1 || cols < 8 || cols % 8) return NVFP4_ERR_SHAPE;
+    if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(slots, 4)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    return cuda_status(launch_moe_combine(static_cast<const uint16_t*>(src), slots,
+                                          static_cast<uint16_t*>(dst), tokens, cols, topk, sms,
+                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int nvfp4_read_status(void* workspace, int* status, nvfp4_stream_t stream) {

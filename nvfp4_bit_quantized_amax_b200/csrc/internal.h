@@ -31,6 +31,11 @@ cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, c
 cudaError_t launch_rht(const uint16_t* x, float* y, int64_t rows, int64_t cols, int axis,
                        uint32_t sign_mask, int sm_count, cudaStream_t st);
 
+cudaError_t launch_moe_gather(const uint16_t* src, const int32_t* idx, uint16_t* dst, int64_t rows,
+                              int64_t cols, int sm_count, cudaStream_t st);
+cudaError_t launch_moe_combine(const uint16_t* src, const int32_t* slot, uint16_t* dst,
+                               int64_t tokens, int64_t cols, int topk, int sm_count, cudaStream_t st);
+
 struct GemmParams {
     const uint8_t* A;    // [M][K/2]
     const uint8_t* sfA;  // swizzled

@@ -8,6 +8,8 @@
 // Method: two-level NVFP4 scaling ("Nemotron NVFP4" explainer, "What NVFP4
 // actually is"); 16x16 weight blocks, RHT on the wgrad inputs, SR on gradients
 // ("NVIDIA's 4-bit floating point pushes AI training limits", artiverse.ca).
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -463,6 +465,76 @@ cudaError_t launch_rht(const uint16_t* x, float* y, int64_t rows, int64_t cols, 
         const int64_t n = (rows / 16) * (cols / 8);
         rht_axis0_kernel<<<grid_for(n, 256, sm_count, 4), 256, 0, st>>>(x, y, rows, cols, sign_mask);
     }
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4
+
+// ============================================================================
+// Mixture-of-experts routing (data movement around the expert GEMMs).
+// gather: dst[i] = src[idx[i]] (a row of bf16), or zeros where idx[i] < 0 (the
+//         padding rows that round each expert's segment up).
+// combine: out[t] = bf16( sum_j src[slot[t][j]] ) in fp32, j = 0 .. topk-1 in order.
+// ============================================================================
+namespace nvfp4 {
+
+__global__ void __launch_bounds__(256) moe_gather_kernel(const uint16_t* __restrict__ src,
+                                                         const int32_t* __restrict__ idx,
+                                                         uint16_t* __restrict__ dst, int64_t rows,
+                                                         int64_t cols) {
+    const int64_t vpr = cols / 8;  // 16-byte vectors per row
+    const int64_t total = rows * vpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / vpr, c = i % vpr;
+        const int32_t s = idx[r];
+        const uint4 v = s >= 0 ? ld_stream_v4(src + (int64_t)s * cols + c * 8) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(dst + r * cols + c * 8) = v;
+    }
+}
+
+__global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __restrict__ src,
+                                                          const int32_t* __restrict__ slot,
+                                                          uint16_t* __restrict__ dst, int64_t tokens,
+                                                          int64_t cols, int topk) {
+    const int64_t vpr = cols / 8;
+    const int64_t total = tokens * vpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / vpr, c = i % vpr;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < topk; ++j) {
+            const int32_t s = slot[t * topk + j];
+            if (s < 0) continue;
+            const uint4 v = ld_stream_v4(src + (int64_t)s * cols + c * 8);
+            float f[8];
+            f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+            f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = __fadd_rn(acc[k], f[k]);
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
+            w[k] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(dst + t * cols + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+cudaError_t launch_moe_gather(const uint16_t* src, const int32_t* idx, uint16_t* dst, int64_t rows,
+                              int64_t cols, int sm_count, cudaStream_t st) {
+    const int64_t total = rows * (cols / 8);
+    moe_gather_kernel<<<grid_for(total, 256, sm_count, 8), 256, 0, st>>>(src, idx, dst, rows, cols);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_combine(const uint16_t* src, const int32_t* slot, uint16_t* dst,
+                               int64_t tokens, int64_t cols, int topk, int sm_count, cudaStream_t st) {
+    const int64_t total = tokens * (cols / 8);
+    moe_combine_kernel<<<grid_for(total, 256, sm_count, 8), 256, 0, st>>>(src, slot, dst, tokens, cols,
+                                                                         topk);
     return cudaGetLastError();
 }
 

@@ -59,15 +59,45 @@ def rht_signs(seed) -> np.ndarray:
     return (_rng(seed).integers(0, 2, size=16) * 2 - 1).astype(np.int8)
 
 
-def moe_group_sizes(n_tokens=16384, n_experts=64, topk=4, zipf_s=1.1, seed=0) -> np.ndarray:
-    """Tokens routed to each expert: every token picks `topk` distinct experts
-    without replacement, expert e drawn with probability proportional to
-    (rank_e)^-zipf_s (Gumbel top-k sampling)."""
+def moe_topk_ids(n_tokens=16384, n_experts=64, topk=4, zipf_s=1.1, seed=0) -> np.ndarray:
+    """Experts of every token, [n_tokens, topk] int32: `topk` distinct experts drawn
+    without replacement, expert e with probability proportional to (e+1)^-zipf_s
+    (Gumbel top-k sampling)."""
     rng = _rng(seed)
     logp = -zipf_s * np.log(np.arange(1, n_experts + 1, dtype=np.float64))
     gumbel = rng.gumbel(size=(n_tokens, n_experts))
-    picks = np.argsort(-(logp[None, :] + gumbel), axis=1)[:, :topk]
-    return np.bincount(picks.ravel(), minlength=n_experts).astype(np.int64)
+    return np.argsort(-(logp[None, :] + gumbel), axis=1)[:, :topk].astype(np.int32)
+
+
+def moe_group_sizes(n_tokens=16384, n_experts=64, topk=4, zipf_s=1.1, seed=0) -> np.ndarray:
+    """Tokens routed to each expert (no padding)."""
+    ids = moe_topk_ids(n_tokens, n_experts, topk, zipf_s, seed)
+    return np.bincount(ids.ravel(), minlength=n_experts).astype(np.int64)
+
+
+def moe_layout(topk_ids: np.ndarray, n_experts: int, pad: int = 64):
+    """Expert-contiguous row layout of the routed copies of every token.
+
+    Returns (group_rows [E] int64, row_src [rows] int32, slots [T, topk] int32):
+    expert e owns rows [off_e, off_e + group_rows[e]) (its tokens in token order,
+    then zero rows up to a multiple of `pad`); row_src[i] is the token whose row
+    lands at permuted row i (-1 for padding); slots[t, j] is the permuted row of
+    the j-th routed copy of token t."""
+    T, k = topk_ids.shape
+    flat = topk_ids.ravel().astype(np.int64)
+    counts = np.bincount(flat, minlength=n_experts).astype(np.int64)
+    group_rows = (counts + pad - 1) // pad * pad
+    offsets = np.concatenate([[0], np.cumsum(group_rows)[:-1]])
+    order = np.argsort(flat, kind="stable")            # copies grouped by expert, token order
+    expert_of = flat[order]
+    first = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    rank_in_group = np.arange(flat.size) - first[expert_of]
+    dest = offsets[expert_of] + rank_in_group
+    row_src = np.full(int(group_rows.sum()), -1, dtype=np.int32)
+    row_src[dest] = (order // k).astype(np.int32)
+    slots = np.empty(flat.size, dtype=np.int32)
+    slots[order] = dest.astype(np.int32)
+    return group_rows, row_src, slots.reshape(T, k)
 
 
 # Workload table: the shapes the parity tests and the bench use.
@@ -75,6 +105,21 @@ LINEAR_SMALL = dict(M=256, K=256, N=256)            # outlier case
 MLP_12B = dict(M=8192, K=5120, N=20480)             # dense up-projection step
 QUANT_SWEEP = dict(rows=8192, cols=8192)
 MOE = dict(experts=64, hidden=2048, ffn=1024, tokens=16384, topk=4, zipf_s=1.1)
+
+
+def moe_inputs(tokens, experts, hidden, ffn, topk, zipf_s, seed=0, pad=64):
+    """Token activations X [T, hidden] ~ N(0,1), expert weights W [E, ffn, hidden] ~
+    N(0, 0.02^2), routing, and the permuted output gradient dY [rows, ffn] ~ N(0,1)
+    with zero padding rows."""
+    ids = moe_topk_ids(tokens, experts, topk, zipf_s, seed)
+    group_rows, row_src, slots = moe_layout(ids, experts, pad)
+    X = normal_bf16((tokens, hidden), seed + 1)
+    W = normal_bf16((experts, ffn, hidden), seed + 2, std=0.02)
+    dY = normal_bf16((int(group_rows.sum()), ffn), seed + 3)
+    dY[row_src < 0] = 0
+    return dict(X=X, W=W, dY=dY, group_rows=group_rows, row_src=row_src, slots=slots, ids=ids)
+
+
 GEMM_SQUARE = (1024, 2048, 4096, 8192, 16384)
 GEMM_SKINNY_WGRAD = [(4096, 4096), (4096, 8192), (8192, 4096), (8192, 8192)]  # (N, K), red=32768
 
