@@ -5,20 +5,24 @@
 // fprop, dgrad and wgrad GEMMs of the NVFP4 linear layer all take this form
 // ("NVIDIA's 4-bit floating point pushes AI training limits", artiverse.ca).
 //
-// Design (one CTA = one 128 x BN output tile, 192 threads):
+// Design: a persistent kernel, one CTA per SM, 448 threads; CTA c computes the
+// 128 x BN output tiles c, c + gridDim.x, ... in turn.
 //   warp 0 lane 0   TMA producer: A/B tiles (128-byte swizzled K-major boxes of
 //                   256 FP4 along K) and the matching 512-byte scale atoms
-//                   (bulk copies) into a STAGES-deep shared-memory ring.
+//                   (bulk copies) into a STAGES-deep shared-memory ring, running
+//                   ahead across tile boundaries.
 //   warps 2-5       scale writers: copy each stage's scale atoms from shared memory
 //                   into a 4-deep ring of TMEM scale regions with tcgen05.st (each
 //                   warp its 32-lane quadrant, every quadrant a full copy), so the
-//                   tensor pipe spends no cycles on scale copies; after the last
-//                   k-tile the same warps run the epilogue: tcgen05.ld of their
-//                   quadrant, scale by alpha * gA * gB, store fp32 and/or bf16.
+//                   tensor pipe spends no cycles on scale copies.
 //   warp 1 lane 0   MMA issuer: four tcgen05.mma kind::mxf4nvf4 block_scale
 //                   (K = 64 each) per stage into the fp32 accumulator in TMEM;
 //                   tcgen05.commit frees the stage and the scale region, and a
-//                   final commit signals the epilogue.
+//                   commit per tile hands the accumulator to the epilogue.
+//   warps 6-13      epilogue: two warps per TMEM quadrant, 128 columns each; they
+//                   drain the accumulator into registers (scaled by alpha*gA*gB and
+//                   rounded to bf16), release TMEM so the next tile's MMAs start,
+//                   then store while the next tile's mainloop runs.
 // Every wait is bounded: after ~1 s the kernel records NVFP4_ERR_TIMEOUT in the
 // status word, stops issuing work, drains its own copies and frees TMEM.
 #include <cuda.h>
@@ -151,7 +155,8 @@ struct __align__(1024) GemmSmem {
     uint64_t empty[STAGES];
     uint64_t sf_full[4];   // scale region r written (4 scale-writer warps arrive)
     uint64_t sf_empty[4];  // scale region r free again (MMA commit)
-    uint64_t acc_full;
+    uint64_t acc_full;   // accumulator of the current tile complete (MMA commit)
+    uint64_t acc_empty;  // accumulator drained by the 8 epilogue warps
     uint32_t tmem_base;
 };
 
@@ -166,22 +171,25 @@ struct TmemLayout {
                                 : kUsed <= 256 ? 256 : 512;
 };
 
+constexpr int kGemmThreads = 448;
+
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p) {
     using Smem = GemmSmem<BN, STAGES>;
     using TL = TmemLayout<BN>;
     constexpr int R = TL::kRegions;
+    constexpr int G = BN / 128;  // 128-row groups of B per tile
     extern __shared__ uint8_t smem_raw[];
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = (int64_t)blockIdx.y * kBM;
-    const int64_t n0 = (int64_t)blockIdx.x * BN;
     const int64_t katoms = p.K / 64;                 // scale atoms per 128-row group
     const int KT = (int)((p.K + 255) / 256);         // k-tiles of 256
     const int64_t nb_groups = (p.N + 127) / 128;     // 128-row groups of B
+    const int64_t tiles_n = (p.N + BN - 1) / BN;
+    const int64_t tiles = ((p.M + kBM - 1) / kBM) * tiles_n;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -193,6 +201,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(smem_addr(&S.sf_empty[r]), 1);
         }
         mbar_init(smem_addr(&S.acc_full), 1);
+        mbar_init(smem_addr(&S.acc_empty), 8);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -212,38 +221,39 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
-            int armed = 0;  // k-tiles whose full barrier was armed
-            for (int kt = 0; kt < KT; ++kt) {
-                const int s = kt % STAGES;
-                const uint32_t use = (uint32_t)(kt / STAGES);
-                if (kt >= STAGES && !mbar_wait(smem_addr(&S.empty[s]), (use & 1u) ^ 1u)) {
-                    timed_out = 1;
-                    break;
+            int64_t it = 0;  // k-tiles issued by this CTA so far (all tiles)
+            for (int64_t tile = blockIdx.x; tile < tiles && !*(volatile int*)&timed_out; tile += gridDim.x) {
+                const int64_t m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * BN;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % STAGES);
+                    const uint32_t use = (uint32_t)(it / STAGES);
+                    if (it >= STAGES && !mbar_wait(smem_addr(&S.empty[s]), (use & 1u) ^ 1u)) {
+                        timed_out = 1;
+                        break;
+                    }
+                    const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
+                    const int nks = rem < 4 ? (int)rem : 4;
+                    const uint32_t sf_bytes = (uint32_t)nks * 512u;
+                    uint32_t bytes = kBM * kBKBytes + BN * kBKBytes + sf_bytes;
+                    for (int g = 0; g < G; ++g)
+                        if (n0 / 128 + g < nb_groups) bytes += sf_bytes;
+                    const uint32_t fb = smem_addr(&S.full[s]);
+                    mbar_expect_tx(fb, bytes);
+                    tma_load_2d(smem_addr(S.a[s]), &tmA, kt * kBKBytes, (int)m0, fb);
+                    tma_load_2d(smem_addr(S.b[s]), &tmB, kt * kBKBytes, (int)n0, fb);
+                    bulk_load(smem_addr(S.sfa[s]), p.sfA + ((m0 / 128) * katoms + (int64_t)kt * 4) * 512,
+                              sf_bytes, fb);
+                    for (int g = 0; g < G; ++g)
+                        if (n0 / 128 + g < nb_groups)
+                            bulk_load(smem_addr(S.sfb[s] + g * 2048),
+                                      p.sfB + ((n0 / 128 + g) * katoms + (int64_t)kt * 4) * 512,
+                                      sf_bytes, fb);
                 }
-                if (*(volatile int*)&timed_out) break;
-                const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
-                const int nks = rem < 4 ? (int)rem : 4;
-                uint32_t sf_bytes = (uint32_t)nks * 512u;
-                uint32_t bytes = kBM * kBKBytes + BN * kBKBytes + sf_bytes;
-                for (int g = 0; g < BN / 128; ++g)
-                    if (n0 / 128 + g < nb_groups) bytes += sf_bytes;
-                const uint32_t fb = smem_addr(&S.full[s]);
-                mbar_expect_tx(fb, bytes);
-                tma_load_2d(smem_addr(S.a[s]), &tmA, kt * kBKBytes, (int)m0, fb);
-                tma_load_2d(smem_addr(S.b[s]), &tmB, kt * kBKBytes, (int)n0, fb);
-                bulk_load(smem_addr(S.sfa[s]), p.sfA + ((m0 / 128) * katoms + (int64_t)kt * 4) * 512,
-                          sf_bytes, fb);
-                for (int g = 0; g < BN / 128; ++g)
-                    if (n0 / 128 + g < nb_groups)
-                        bulk_load(smem_addr(S.sfb[s] + g * 2048),
-                                  p.sfB + ((n0 / 128 + g) * katoms + (int64_t)kt * 4) * 512, sf_bytes,
-                                  fb);
-                armed = kt + 1;
             }
             if (*(volatile int*)&timed_out) {
                 // let copies already issued land before the CTA can exit
-                for (int kt = max(0, armed - STAGES); kt < armed; ++kt)
-                    mbar_wait(smem_addr(&S.full[kt % STAGES]), (uint32_t)(kt / STAGES) & 1u);
+                for (int64_t k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
+                    mbar_wait(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
             }
         }
         __syncwarp();
@@ -251,42 +261,57 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = nvf4_idesc<BN>();
-            for (int kt = 0; kt < KT; ++kt) {
-                const int s = kt % STAGES, r = kt % R;
-                if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(kt / STAGES) & 1u) ||
-                    !mbar_wait(smem_addr(&S.sf_full[r]), (uint32_t)(kt / R) & 1u)) {
+            int64_t it = 0;
+            uint32_t local = 0;  // tiles of this CTA so far
+            for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+                // the epilogue has drained the accumulator of the previous tile
+                if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u)) {
                     timed_out = 1;
                     break;
                 }
                 tc_fence_after();
-                const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
-                const int nks = rem < 4 ? (int)rem : 4;
-                const uint32_t t_sfa = tmem + (uint32_t)(BN + r * TL::kRegion);
-                const uint32_t t_sfb = t_sfa + TL::kSfaCols;
-                const uint32_t a_base = smem_addr(S.a[s]), b_base = smem_addr(S.b[s]);
-                for (int j = 0; j < nks; ++j) {
-                    tc_mma_nvf4(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
-                                idesc, t_sfa + 4 * j, t_sfb + 4 * (BN / 128) * j,
-                                (kt > 0 || j > 0) ? 1u : 0u);
+                bool bad = false;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % STAGES), r = (int)(it % R);
+                    if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u) ||
+                        !mbar_wait(smem_addr(&S.sf_full[r]), (uint32_t)(it / R) & 1u)) {
+                        bad = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
+                    const int nks = rem < 4 ? (int)rem : 4;
+                    const uint32_t t_sfa = tmem + (uint32_t)(BN + r * TL::kRegion);
+                    const uint32_t t_sfb = t_sfa + TL::kSfaCols;
+                    const uint32_t a_base = smem_addr(S.a[s]), b_base = smem_addr(S.b[s]);
+                    for (int j = 0; j < nks; ++j) {
+                        tc_mma_nvf4(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                                    idesc, t_sfa + 4 * j, t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit(smem_addr(&S.empty[s]));
+                    tc_commit(smem_addr(&S.sf_empty[r]));
                 }
-                tc_commit(smem_addr(&S.empty[s]));
-                tc_commit(smem_addr(&S.sf_empty[r]));
+                tc_commit(smem_addr(&S.acc_full));
+                if (bad) {
+                    timed_out = 1;
+                    break;
+                }
             }
-            tc_commit(smem_addr(&S.acc_full));
         }
         __syncwarp();
-    } else {
-        // ---------------------------------------------------- scale writers
+    } else if (warp < 6) {
+        // ---------------------------------------------------- scale writers (warps 2-5)
         // TMEM quadrant q = warp % 4 (lanes 32q .. 32q+31).  Scale atom j of a
         // stage holds, in 16-byte line l, the 4-block scales of rows l, l+32, l+64,
         // l+96; lane l of every quadrant gets line l in 4 consecutive columns, the
         // layout the block-scaled MMA reads (row l + 32i in column i).
         const int q = warp & 3;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        for (int kt = 0; kt < KT; ++kt) {
-            const int s = kt % STAGES, r = kt % R;
-            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(kt / STAGES) & 1u) ||
-                (kt >= R && !mbar_wait(smem_addr(&S.sf_empty[r]), ((uint32_t)(kt / R) & 1u) ^ 1u))) {
+        const int64_t total = ((tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) * KT;
+        for (int64_t it = 0; it < total; ++it) {
+            const int s = (int)(it % STAGES), r = (int)(it % R);
+            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u) ||
+                (it >= R && !mbar_wait(smem_addr(&S.sf_empty[r]), ((uint32_t)(it / R) & 1u) ^ 1u))) {
                 timed_out = 1;
                 break;
             }
@@ -300,12 +325,11 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_st16(lane_base + col, v);
 #pragma unroll
-            for (int h = 0; h < BN / 128; ++h) {  // 16 columns per group pair of k-steps
+            for (int h = 0; h < G; ++h) {  // 16 columns: k-steps and groups, order 4*G*j + 4*g
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    // column order of the B scales: k-step j, group g -> 4*(BN/128)*j + 4*g
-                    const int idx = h * 4 + jj;            // 0 .. 4*(BN/128)-1
-                    const int j = idx / (BN / 128), g = idx % (BN / 128);
+                    const int idx = h * 4 + jj;
+                    const int j = idx / G, g = idx % G;
                     const uint4 w = *reinterpret_cast<const uint4*>(S.sfb[s] + g * 2048 + j * 512 + lane * 16);
                     v[4 * jj] = w.x; v[4 * jj + 1] = w.y; v[4 * jj + 2] = w.z; v[4 * jj + 3] = w.w;
                 }
@@ -317,57 +341,73 @@ __global__ void __launch_bounds__(192, 1)
             if (lane == 0) mbar_arrive(smem_addr(&S.sf_full[r]));
         }
         __syncwarp();
-
-        // ---------------------------------------------------- epilogue
-        const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), 0);
-        tc_fence_after();
-        __syncwarp();
-        if (!acc_ok) timed_out = 1;
-        const bool bad = *(volatile int*)&timed_out != 0;
+    } else {
+        // ---------------------------------------------------- epilogue (warps 6-13)
+        const int q = warp & 3;                  // TMEM quadrant of this warp
+        const int half = (warp - 6) >> 2;        // columns [half * BN/2, +BN/2)
+        constexpr int HC = BN / 2;               // columns per epilogue warp
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
         float alpha = p.alpha;
         if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
         if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
-        const int64_t row = m0 + q * 32 + lane;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            const uint32_t taddr = lane_base + (uint32_t)(c * 32);
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-                "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                  "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-                  "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-                  "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-                  "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-                  "=r"(r[31])
-                : "r"(taddr));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            if (bad || row >= p.M) continue;
-            const int64_t col0 = n0 + c * 32;
-            float v[32];
+        uint32_t local = 0;
+        for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+            if (*(volatile int*)&timed_out) break;  // a stage failed: no further tiles arrive
+            const int64_t m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * BN;
+            const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u);
+            tc_fence_after();
+            __syncwarp();
+            if (!acc_ok) timed_out = 1;
+            const bool bad = *(volatile int*)&timed_out != 0;
+            const int64_t row = m0 + 32 * q + lane;
+            const int64_t col0 = n0 + half * HC;
+            uint32_t packed[HC / 2];  // bf16 pairs of this thread's row
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+            for (int c = 0; c < HC / 32; ++c) {
+                uint32_t r[32];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+                    "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                    : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                      "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                      "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+                      "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+                      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+                      "=r"(r[31])
+                    : "r"(lane_base + (uint32_t)(c * 32)));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                float v[32];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const int64_t col = col0 + 8 * g;
-                if (col >= p.N) break;
-                if (p.D_f32) {
-                    float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
-                    d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
-                    d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                if (p.D_f32 && !bad && row < p.M) {
+                    // fp32 output (checking path): stored before TMEM is released
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int64_t col = col0 + c * 32 + 8 * g;
+                        if (col >= p.N) break;
+                        float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
+                        d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
+                        d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+                    }
                 }
-                if (p.D_bf16) {
-                    uint4 w;
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * g], v[8 * g + 1]);
-                    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * g + 2], v[8 * g + 3]);
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * g + 4], v[8 * g + 5]);
-                    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * g + 6], v[8 * g + 7]);
-                    w.x = *reinterpret_cast<uint32_t*>(&h0);
-                    w.y = *reinterpret_cast<uint32_t*>(&h1);
-                    w.z = *reinterpret_cast<uint32_t*>(&h2);
-                    w.w = *reinterpret_cast<uint32_t*>(&h3);
-                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.D_bf16) + row * p.N + col) = w;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                    packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+            }
+            // accumulator drained: the next tile's MMAs may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&S.acc_empty));
+            if (p.D_bf16 && !bad && row < p.M) {
+                __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.D_bf16) + row * p.N;
+#pragma unroll
+                for (int g = 0; g < HC / 8; ++g) {
+                    const int64_t col = col0 + 8 * g;
+                    if (col >= p.N) break;
+                    *reinterpret_cast<uint4*>(drow + col) =
+                        make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
                 }
             }
         }
@@ -414,7 +454,7 @@ static bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, i
 }
 
 template <int BN, int STAGES>
-static cudaError_t launch_gemm_cfg(const GemmParams& p, cudaStream_t st) {
+static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream_t st) {
     CUtensorMap ma, mb;
     if (!make_operand_map(&ma, p.A, p.M, p.K / 2, kBM) || !make_operand_map(&mb, p.B, p.N, p.K / 2, BN))
         return cudaErrorInvalidValue;
@@ -426,14 +466,14 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const dim3 grid((unsigned)((p.N + BN - 1) / BN), (unsigned)((p.M + kBM - 1) / kBM));
-    gemm_nvf4_kernel<BN, STAGES><<<grid, 192, smem, st>>>(ma, mb, p);
+    const int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
+    const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
+    gemm_nvf4_kernel<BN, STAGES><<<grid, kGemmThreads, smem, st>>>(ma, mb, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
-    (void)sm_count;
-    return launch_gemm_cfg<256, 4>(p, st);
+    return launch_gemm_cfg<256, 4>(p, sm_count, st);
 }
 
 }  // namespace nvfp4
