@@ -108,48 +108,57 @@ __device__ __forceinline__ void block_scale(float amax_b, const TensorScale& ts,
 struct Philox4 {
     uint32_t x, y, z, w;
 };
-__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
-                                                 uint32_t c3, uint32_t k0, uint32_t k1) {
+
+// Philox4x32-10 with the key schedule taken from rk: round r uses
+// (rk[2r], rk[2r+1]) = (k0 + r * 0x9E3779B9, k1 + r * 0xBB67AE85).  The
+// schedule depends on the seed alone, so the host computes it once per launch
+// and the kernels read it from their parameters.
+__device__ __forceinline__ Philox4 philox4x32_10_rk(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                    uint32_t c3, const uint32_t (&rk)[20]) {
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
         const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
         const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-        const uint32_t n0 = hi1 ^ c1 ^ k0;
-        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        const uint32_t n0 = hi1 ^ c1 ^ rk[2 * r];
+        const uint32_t n2 = hi0 ^ c3 ^ rk[2 * r + 1];
         c0 = n0;
         c1 = lo1;
         c2 = n2;
         c3 = lo0;
-        k0 += 0x9E3779B9u;
-        k1 += 0xBB67AE85u;
     }
     return Philox4{c0, c1, c2, c3};
 }
 
 // Sixteen-bit draws of the 8 consecutive elements 8*group .. 8*group+7 of random
-// stream `stream`: element j takes half (j & 1) of word (j >> 1).
-__device__ __forceinline__ Philox4 sr_draws8(uint64_t seed, uint32_t stream, uint64_t group) {
-    return philox4x32_10((uint32_t)group, (uint32_t)(group >> 32), stream, 0u, (uint32_t)seed,
-                         (uint32_t)(seed >> 32));
+// stream `stream`: counter (group lo, group hi, stream, 0); element j takes half
+// (j & 1) of word (j >> 1).
+__device__ __forceinline__ Philox4 sr_draws8(const uint32_t (&rk)[20], uint32_t stream,
+                                             uint64_t group) {
+    return philox4x32_10_rk((uint32_t)group, (uint32_t)(group >> 32), stream, 0u, rk);
 }
 __device__ __forceinline__ uint32_t draw16(const Philox4& p, int j) {
     const uint32_t w = (j >> 1) == 0 ? p.x : (j >> 1) == 1 ? p.y : (j >> 1) == 2 ? p.z : p.w;
     return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
 }
 
-// Stochastic rounding of v onto the E2M1 grid (returns the rounded value, whose
-// E2M1 conversion is then exact): lo <= |v| < hi adjacent grid points,
-// p = (|v| - lo) / (hi - lo), round up iff r < p * 2^16.  The grid spacing is
-// 0.5 below 2, 1 below 4 and 2 below 6, so every step here is exact in fp32.
-__device__ __forceinline__ float sr_e2m1_value(float v, uint32_t r16) {
+// Stochastic rounding of v straight to its E2M1 code.  Let a = min(|v|, 6) and
+// lo <= a <= hi the adjacent grid points; the rule rounds up iff r < p * 2^16
+// with p = (a - lo) / (hi - lo) and r the 16-bit draw.  The map c(a) = 2a on
+// [0, 2], a + 2 on [2, 4], a / 2 + 4 on [4, 6] is affine between grid points and
+// sends the grid {0, .5, 1, 1.5, 2, 3, 4, 6} to the codes 0..7, so floor(c(a))
+// is the code of lo and frac(c(a)) is p.  With C = ceil(c(a) * 2^16), one fp32
+// FMA rounded upward (a times a power of two plus an integer, below 2^24, so the
+// only rounding is the ceiling), the code is floor(c) + [r < p * 2^16] =
+// (C + 65535 - r) >> 16; grid points (p = 0) never move.  The sign bit of v is
+// kept, zero included.
+__device__ __forceinline__ uint32_t sr_e2m1_code(float v, uint32_t r16) {
     const float a = fminf(fabsf(v), 6.0f);
-    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-    const float rstep = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-    const float lo = __fmul_rn(floorf(__fmul_rn(a, rstep)), step);
-    const float p = __fmul_rn(__fsub_rn(a, lo), rstep);
-    const bool up = __uint2float_rn(r16) < __fmul_rn(p, 65536.0f);
-    const float q = up ? __fadd_rn(lo, step) : lo;
-    return copysignf(q, v);
+    const bool lo2 = a < 2.0f, lo4 = a < 4.0f;
+    const float rs = lo2 ? 131072.0f : (lo4 ? 65536.0f : 32768.0f);      // slope * 2^16
+    const float b = lo2 ? 8388608.0f : (lo4 ? 8519680.0f : 8650752.0f);  // 2^23 + offset * 2^16
+    const uint32_t c = __float_as_uint(__fmaf_ru(a, rs, b));             // bits of 2^23 + C
+    const uint32_t code = (c - (0x4B000000u - 65535u) - r16) >> 16;
+    return code | ((__float_as_uint(v) >> 28) & 8u);
 }
 
 // ---------------------------------------------------------------- scale layout

@@ -21,7 +21,20 @@ struct QuantParams {
     uint64_t seed;
     int row_sr, col_sr, col_rht;
     uint32_t sign_mask;  // bit i set: rotation sign i is -1
+    uint32_t rk[20];     // Philox4x32-10 round keys of `seed` (filled by the launchers)
 };
+
+// Philox4x32-10 key schedule of a 64-bit seed: round r uses
+// (lo(seed) + r * 0x9E3779B9, hi(seed) + r * 0xBB67AE85), mod 2^32.
+inline void philox_round_keys(uint64_t seed, uint32_t (&rk)[20]) {
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        rk[2 * r] = k0;
+        rk[2 * r + 1] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+}
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
                         uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st);

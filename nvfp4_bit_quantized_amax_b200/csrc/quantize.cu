@@ -116,19 +116,21 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
 __device__ __forceinline__ bool finite_bits(uint32_t b) { return (b & 0x7FFFFFFFu) < 0x7F800000u; }
 
 // Eight values -> packed codes with RNE or SR (element index e0 .. e0+7 of the
-// quantized tensor, e0 % 8 == 0).
+// quantized tensor, e0 % 8 == 0); element i lands in bits [4i, 4i+4).
 __device__ __forceinline__ uint32_t encode8(const float (&v)[8], float inv, bool sr,
-                                            uint64_t seed, uint32_t stream, uint64_t e0) {
-    float q[8];
+                                            const uint32_t (&rk)[20], uint32_t stream,
+                                            uint64_t e0) {
     if (!sr) {
+        float q[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
-    } else {
-        const Philox4 p = sr_draws8(seed, stream, e0 >> 3);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = sr_e2m1_value(__fmul_rn(v[i], inv), draw16(p, i));
+        return e2m1x8_rn(q);
     }
-    return e2m1x8_rn(q);
+    const Philox4 r = sr_draws8(rk, stream, e0 >> 3);
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out |= sr_e2m1_code(__fmul_rn(v[i], inv), draw16(r, i)) << (4 * i);
+    return out;
 }
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&v)[8]) {
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
         block_scale(amax, tr, s, inv);
         float v[8];
         unpack8(w, v);
-        const uint32_t codes = encode8(v, inv, p.row_sr, p.seed, 0u, (uint64_t)q * 8);
+        const uint32_t codes = encode8(v, inv, p.row_sr, p.rk, 0u, (uint64_t)q * 8);
         if (valid) {
             reinterpret_cast<uint32_t*>(p.row_data)[q] = codes;
             if ((q & 1) == 0) {
@@ -289,8 +291,8 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
                     lo8[i] = y[i];
                     hi8[i] = y[8 + i];
                 }
-                out[2 * jj] = encode8(lo8, inv, p.col_sr, p.seed, 1u, e0);
-                out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, p.seed, 1u, e0 + 8);
+                out[2 * jj] = encode8(lo8, inv, p.col_sr, p.rk, 1u, e0);
+                out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, p.rk, 1u, e0 + 8);
                 if (c < p.cols && r0 + 16 * j < p.rows)
                     p.col_sf[sf_offset(c, (r0 >> 4) + j, katoms_c)] = (uint8_t)s;
             }
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
             float v[8];
             unpack8(reg[k], v);
             const uint32_t codes =
-                encode8(v, inv, p.row_sr, p.seed, 0u, (uint64_t)r * (uint64_t)p.cols + (uint64_t)c);
+                encode8(v, inv, p.row_sr, p.rk, 0u, (uint64_t)r * (uint64_t)p.cols + (uint64_t)c);
             if (r < p.rows && c < p.cols) {
                 *reinterpret_cast<uint32_t*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
                 if ((lc & 15) == 0) p.row_sf[sf_offset(r, c >> 4, katoms_r)] = (uint8_t)s;
@@ -431,14 +433,18 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant_rows(const QuantParams& p, int sm_count, cudaStream_t st) {
+cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStream_t st) {
+    QuantParams p = params;
+    philox_round_keys(p.seed, p.rk);
     const int64_t nchunks = p.rows * (p.cols / 8);
     const int grid = grid_for(nchunks, 256, sm_count, 8);
     quant_rows_kernel<<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, cudaStream_t st) {
+cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, cudaStream_t st) {
+    QuantParams p = params;
+    philox_round_keys(p.seed, p.rk);
     const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
     if (two_d)
         quant_tile_kernel<true, false><<<grid, 256, 0, st>>>(p);
