@@ -29,6 +29,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -124,6 +126,28 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// Bulk tensor store of a shared-memory box to global memory (async proxy), and
+// its completion groups: .read waits until the source buffer may be reused.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Generic-proxy shared-memory writes made visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z,
+                                             uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading and
 // stride byte offsets (all >> 4), descriptor version 1, layout type.
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
@@ -149,6 +173,7 @@ template <int BN, int STAGES>
 struct __align__(1024) GemmSmem {
     uint8_t a[STAGES][kBM * kBKBytes];          // 16 KB / stage
     uint8_t b[STAGES][BN * kBKBytes];           // BN * 128 B / stage
+    uint8_t dstage[8][32 * 32];                 // per epilogue warp: 32 rows x 16 bf16, 32B-swizzled
     uint8_t sfa[STAGES][4 * 512];               // 4 atoms: 128 rows x 16 blocks
     uint8_t sfb[STAGES][(BN / 128) * 4 * 512];  // per 128-row group, 4 atoms
     uint64_t full[STAGES];
@@ -176,7 +201,7 @@ constexpr int kGemmThreads = 448;
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
     using Smem = GemmSmem<BN, STAGES>;
     using TL = TmemLayout<BN>;
     constexpr int R = TL::kRegions;
@@ -400,17 +425,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&S.acc_empty));
-            if (p.D_bf16 && !bad && row < p.M) {
-                __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.D_bf16) + row * p.N;
+            if (p.D_bf16 && !bad && m0 + 32 * q < p.M) {
+                // stage 32 rows x 16 columns at a time in this warp's buffer (row = lane,
+                // 16-byte half j of a row at half j ^ ((row / 4) % 2): the 32-byte swizzle
+                // the store's tensor map undoes; conflict-free), then one bulk tensor
+                // store; rows and columns past M and N are clipped by the tensor map.
+                const uint32_t buf = smem_addr(S.dstage[warp - 6]);
+                const uint32_t sw = (uint32_t)((lane >> 2) & 1);
 #pragma unroll
-                for (int g = 0; g < HC / 8; ++g) {
-                    const int64_t col = col0 + 8 * g;
-                    if (col >= p.N) break;
-                    *reinterpret_cast<uint4*>(drow + col) =
-                        make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+                for (int h = 0; h < HC / 16; ++h) {
+                    if (col0 + 16 * h >= p.N) break;
+                    if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        st_shared_v4(buf + (uint32_t)lane * 32u + (((uint32_t)j ^ sw) << 4),
+                                     packed[8 * h + 4 * j], packed[8 * h + 4 * j + 1],
+                                     packed[8 * h + 4 * j + 2], packed[8 * h + 4 * j + 3]);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmD, buf, (int)(col0 + 16 * h), (int)(m0 + 32 * q));
+                        bulk_commit();
+                    }
                 }
             }
         }
+        if (lane == 0) bulk_wait_all();  // every store of this warp has landed
+        __syncwarp();
     }
     __syncthreads();
     if (threadIdx.x == 0 && *(volatile int*)&timed_out) set_status(p.status, kStatusTimeout);
@@ -453,11 +495,27 @@ static bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, i
     return r == CUDA_SUCCESS;
 }
 
+// bf16 output [M][N] (N % 8 == 0), box = 16 columns x 32 rows, 32-byte swizzle.
+static bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    cuuint32_t box[2] = {16, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int BN, int STAGES>
 static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream_t st) {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, md;
     if (!make_operand_map(&ma, p.A, p.M, p.K / 2, kBM) || !make_operand_map(&mb, p.B, p.N, p.K / 2, BN))
         return cudaErrorInvalidValue;
+    memset(&md, 0, sizeof(md));
+    if (p.D_bf16 && !make_output_map(&md, p.D_bf16, p.M, p.N)) return cudaErrorInvalidValue;
     const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
     static bool configured = false;
     if (!configured) {
@@ -468,7 +526,7 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream
     }
     const int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
-    gemm_nvf4_kernel<BN, STAGES><<<grid, kGemmThreads, smem, st>>>(ma, mb, p);
+    gemm_nvf4_kernel<BN, STAGES><<<grid, kGemmThreads, smem, st>>>(ma, mb, md, p);
     return cudaGetLastError();
 }
 
