@@ -109,25 +109,78 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# --------------------------------------------------------------------------- ranks
+def init_ranks(world, dev, backend="nccl", timeout_s=120):
+    """Process group of the `world` ranks (none at world 1) and the two collective
+    steps the bench takes: a barrier and the maximum of a float over ranks.  Every
+    rank calls both in the same order; the short timeout turns a lost rank into an
+    error instead of a hang."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        kw = {"device_id": dev} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return float(v)
+        t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    def finish():
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+    return barrier, max_over_ranks, finish
+
+
+def whole_job_tflops(world, flops_per_rank_step, ms_max):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_max * 1e-3) / 1e12
+
+
+def bench_line(world, steps, warmup, ms, value, clocks, e2e, cpu, extra):
+    """The JSON line rank 0 prints (weak scaling: every rank a full replica)."""
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+        "steps": steps, "warmup": max(warmup, 3), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic (seeded: X~N(0,1), W~N(0,0.02^2), dY~N(0,1e-3^2), bf16)",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N,
+                   "global_batch_tokens": M * world,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (629 MB bf16 inputs, ~1.6 GB touched per step)",
+                   "recipe": "X,dY 1x16; W 16x16; SR on dY; 16-pt RHT on wgrad operands"},
+        "gpu_launches": KERNELS_PER_STEP * steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    line.update(extra)
+    return line
+
+
 # --------------------------------------------------------------------------- ours
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     from nvfp4_bit_quantized_amax_b200 import capi
     from nvfp4_bit_quantized_amax_b200 import synthetic as syn
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=dev,
-                                timeout=__import__("datetime").timedelta(seconds=120))
+    barrier, max_over_ranks, finish = init_ranks(world, dev, "nccl")
     capi.load()
     stream = torch.cuda.current_stream()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
 
     # synthetic inputs (seeded per rank: every replica its own batch)
     Xb, Wb, dYb = syn.mlp_inputs(M, K, N, seed=1000 * rank)
@@ -163,19 +216,12 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         return s.elapsed_time(e) / iters
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.item()
-
     # ---- the timed step (inputs resident in HBM; per-step working set ~1.6 GB >> L2)
     with ClockSampler(local_rank) as clk:
         ms = timed(step, args.steps, max(args.warmup, 3))
     ms = max_over_ranks(ms)
     assert capi.nvfp4_read_status(ws) == 0
-    value = world * FLOPS_PER_STEP / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, FLOPS_PER_STEP, ms)
 
     out = {}
     if rank == 0 or True:
@@ -273,34 +319,17 @@ def run_ours(args, rank, world, local_rank):
         e_iters = max(3, min(10, args.steps))
         e_ms = max_over_ranks(timed(e2e_step, e_iters, 2))
         h2d = 2 * (M * K + N * K + M * N)
-        e2e = {"value": round(world * FLOPS_PER_STEP / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+        e2e = {"value": round(whole_job_tflops(world, FLOPS_PER_STEP, e_ms), 2), "unit": "TFLOPS",
                "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    finish()
     if rank != 0:
         return
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
-        "data": "synthetic (seeded: X~N(0,1), W~N(0,0.02^2), dY~N(0,1e-3^2), bf16)",
-        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N,
-                   "global_batch_tokens": M * world,
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (629 MB bf16 inputs, ~1.6 GB touched per step)",
-                   "recipe": "X,dY 1x16; W 16x16; SR on dY; 16-pt RHT on wgrad operands"},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
-        "clocks": clk.summary(),
-        "e2e": e2e,
-        "cpu_baseline": cpu,
-    }
-    line.update(out)
+    line = bench_line(world, args.steps, args.warmup, ms, value, clk.summary(), e2e, cpu, out)
     print(json.dumps(line), flush=True)
 
 

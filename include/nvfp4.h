@@ -248,8 +248,11 @@ int nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int block_
                            int rounding, uint64_t seed, uint8_t* packed, uint8_t* scales,
                            float* tensor_scale, nvfp4_stream_t stream);
 
-/* Status word of a quantize or linear workspace (synchronizes `stream`, then
- * clears the word).  *status = NVFP4_OK or the first device error recorded.    */
+/* Status word of a quantize or linear workspace: synchronizes `stream`, then
+ * copies the word to *status (host): NVFP4_OK or the first device error recorded
+ * since the word was last cleared.  Every call that takes the workspace clears
+ * the word on its stream before its first kernel, so the word describes the
+ * latest such call; reading it does not change it.                            */
 int nvfp4_read_status(void* workspace, int* status, nvfp4_stream_t stream);
 
 const char* nvfp4_status_string(int status);
