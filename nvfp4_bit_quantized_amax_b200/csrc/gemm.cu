@@ -17,12 +17,14 @@
 //                   tensor pipe spends no cycles on scale copies.
 //   warp 1 lane 0   MMA issuer: four tcgen05.mma kind::mxf4nvf4 block_scale
 //                   (K = 64 each) per stage into the fp32 accumulator in TMEM;
-//                   tcgen05.commit frees the stage and the scale region, and a
-//                   commit per tile hands the accumulator to the epilogue.
+//                   one tcgen05.commit per stage frees the stage (and with it the
+//                   scale region of the same index), and a commit per tile hands
+//                   the accumulator to the epilogue.
 //   warps 6-13      epilogue: two warps per TMEM quadrant, 128 columns each; they
 //                   drain the accumulator into registers (scaled by alpha*gA*gB and
 //                   rounded to bf16), release TMEM so the next tile's MMAs start,
-//                   then store while the next tile's mainloop runs.
+//                   then write the tile through a swizzled shared-memory buffer
+//                   with bulk tensor stores while the next tile's mainloop runs.
 // Every wait is bounded: after ~1 s the kernel records NVFP4_ERR_TIMEOUT in the
 // status word, stops issuing work, drains its own copies and frees TMEM.
 #include <cuda.h>
@@ -179,7 +181,6 @@ struct __align__(1024) GemmSmem {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t sf_full[4];   // scale region r written (4 scale-writer warps arrive)
-    uint64_t sf_empty[4];  // scale region r free again (MMA commit)
     uint64_t acc_full;   // accumulator of the current tile complete (MMA commit)
     uint64_t acc_empty;  // accumulator drained by the 8 epilogue warps
     uint32_t tmem_base;
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     using TL = TmemLayout<BN>;
     constexpr int R = TL::kRegions;
     constexpr int G = BN / 128;  // 128-row groups of B per tile
+    static_assert(R == STAGES, "scale regions are freed with their shared-memory stage");
     extern __shared__ uint8_t smem_raw[];
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -223,7 +225,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int r = 0; r < R; ++r) {
             mbar_init(smem_addr(&S.sf_full[r]), 4);
-            mbar_init(smem_addr(&S.sf_empty[r]), 1);
         }
         mbar_init(smem_addr(&S.acc_full), 1);
         mbar_init(smem_addr(&S.acc_empty), 8);
@@ -314,7 +315,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                     idesc, t_sfa + 4 * j, t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
                     }
                     tc_commit(smem_addr(&S.empty[s]));
-                    tc_commit(smem_addr(&S.sf_empty[r]));
                 }
                 tc_commit(smem_addr(&S.acc_full));
                 if (bad) {
@@ -335,12 +335,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int64_t total = ((tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) * KT;
         for (int64_t it = 0; it < total; ++it) {
             const int s = (int)(it % STAGES), r = (int)(it % R);
-            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u) ||
-                (it >= R && !mbar_wait(smem_addr(&S.sf_empty[r]), ((uint32_t)(it / R) & 1u) ^ 1u))) {
+            // Region r was last read by the MMAs of k-tile it - R.  With R == STAGES
+            // those MMAs completed before the producer could refill stage s (it
+            // waited for their commit), so the arrival of k-tile it in stage s
+            // also means that region r is free.
+            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u)) {
                 timed_out = 1;
                 break;
             }
-            tc_fence_after();  // the MMAs that read this region before are complete
+            tc_fence_after();
             const uint32_t col = (uint32_t)(BN + r * TL::kRegion);
             uint32_t v[16];
 #pragma unroll
