@@ -128,6 +128,34 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// The four K = 64 MMAs of one 256-deep k-tile in one statement: descriptors
+// advance by 32 bytes (2 in the >> 4 address field), the A scales by 4 TMEM
+// columns and the B scales by 4 * G columns per step; only the first MMA takes
+// `accumulate` (0 on the first k-tile of a tile), the rest always accumulate.
+template <int G>
+__device__ __forceinline__ void tc_mma_nvf4_x4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        ".reg .b32 sa1, sa2, sa3, sb1, sb2, sb3;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "setp.eq.b32 q, %3, %3;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.u32 sa1, %4, 4;\n\tadd.u32 sa2, %4, 8;\n\tadd.u32 sa3, %4, 12;\n\t"
+        "add.u32 sb1, %5, %7;\n\tadd.u32 sb2, %5, %8;\n\tadd.u32 sb3, %5, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a1, b1, %3, [sa1], [sb1], q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a2, b2, %3, [sa2], [sb2], q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a3, b3, %3, [sa3], [sb3], q;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate), "n"(4 * G),
+        "n"(8 * G), "n"(12 * G)
+        : "memory");
+}
+
 // Bulk tensor store of a shared-memory box to global memory (async proxy), and
 // its completion groups: .read waits until the source buffer may be reused.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
@@ -286,8 +314,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
+            // The block-scaled MMA does not queue ahead of its issuing thread:
+            // every instruction this thread runs between two MMAs idles the
+            // tensor pipe.  So the loop keeps stage, phase and descriptors in
+            // registers and waits on one barrier per k-tile: the scale writers
+            // arrive on sf_full only after they saw the stage's bytes land.
             constexpr uint32_t idesc = nvf4_idesc<BN>();
-            int64_t it = 0;
+            constexpr uint64_t kAStep = (kBM * kBKBytes) >> 4, kBStep = (BN * kBKBytes) >> 4;
+            const uint64_t adesc0 = operand_desc(smem_addr(S.a[0]));
+            const uint64_t bdesc0 = operand_desc(smem_addr(S.b[0]));
+            const uint32_t tsf0 = tmem + (uint32_t)BN;
+            const uint32_t sf_full0 = smem_addr(&S.sf_full[0]), empty0 = smem_addr(&S.empty[0]);
+            const int KT_full = (int)(p.K / 256);   // k-tiles with all four K = 64 steps
+            uint32_t s = 0, ph = 0;                 // stage (= scale region) and its phase
             uint32_t local = 0;  // tiles of this CTA so far
             for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
                 // the epilogue has drained the accumulator of the previous tile
@@ -297,24 +336,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_after();
                 bool bad = false;
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = (int)(it % STAGES), r = (int)(it % R);
-                    if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u) ||
-                        !mbar_wait(smem_addr(&S.sf_full[r]), (uint32_t)(it / R) & 1u)) {
+                for (int kt = 0; kt < KT; ++kt) {
+                    if (!mbar_wait(sf_full0 + 8u * s, ph)) {
                         bad = true;
                         break;
                     }
                     tc_fence_after();
-                    const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
-                    const int nks = rem < 4 ? (int)rem : 4;
-                    const uint32_t t_sfa = tmem + (uint32_t)(BN + r * TL::kRegion);
+                    const uint64_t ad = adesc0 + kAStep * s, bd = bdesc0 + kBStep * s;
+                    const uint32_t t_sfa = tsf0 + (uint32_t)TL::kRegion * s;
                     const uint32_t t_sfb = t_sfa + TL::kSfaCols;
-                    const uint32_t a_base = smem_addr(S.a[s]), b_base = smem_addr(S.b[s]);
-                    for (int j = 0; j < nks; ++j) {
-                        tc_mma_nvf4(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
-                                    idesc, t_sfa + 4 * j, t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
+                    if (kt < KT_full) {
+                        tc_mma_nvf4_x4<G>(tmem, ad, bd, idesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
+                    } else {  // K tail: 1 to 3 steps of 64
+                        const int nks = (int)((p.K - (int64_t)kt * 256) / kKStep);
+                        for (int j = 0; j < nks; ++j)
+                            tc_mma_nvf4(tmem, ad + 2u * j, bd + 2u * j, idesc, t_sfa + 4 * j,
+                                        t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
                     }
-                    tc_commit(smem_addr(&S.empty[s]));
+                    tc_commit(empty0 + 8u * s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 tc_commit(smem_addr(&S.acc_full));
                 if (bad) {
