@@ -48,6 +48,8 @@ def check(D32, D16, ref, bound, what):
     (128, 256, 64),       # one MMA
     (256, 512, 1024),     # several tiles, k-tiles > stages
     (200, 136, 320),      # ragged M, N; partial last k-tile
+    (256, 256, 768),      # odd number of 256-deep k-tiles (last stage half empty)
+    (128, 512, 1344),     # K % 256 == 64: k-tile slabs loaded one by one
     (384, 1024, 4096),
     (1, 8, 128),          # degenerate tiny output
 ])
