@@ -225,6 +225,92 @@ struct TmemLayout {
                                 : kUsed <= 256 ? 256 : 512;
 };
 
+// ---------------------------------------------------------------- epilogue
+// One epilogue warp's share of a finished tile: its 32 TMEM lanes (rows row0 ..
+// row0+31, lane = row) by BN/2 columns from col0.  Drains the accumulator into
+// registers (times alpha, rounded to bf16; the fp32 checking output is stored
+// before the release), arrives on the accumulator-empty barrier (local, or the
+// leader's at a cluster address when `remote`), then writes the bf16 tile 32 rows x 16 columns
+// at a time through this warp's 1 KB buffer: 16-byte half j of a row at half
+// j ^ ((row / 4) % 2), the 32-byte swizzle the store's tensor map undoes
+// (conflict-free), one bulk tensor store each; rows and columns past M and N are
+// clipped by the tensor map.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, int64_t col0,
+                                              const GemmParams& p, float alpha, bool bad,
+                                              uint32_t acc_empty, uint32_t remote, uint32_t buf,
+                                              const CUtensorMap* tmD) {
+    constexpr int HC = BN / 2;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = row0 + lane;
+    uint32_t packed[HC / 2];  // bf16 pairs of this thread's row
+#pragma unroll
+    for (int c = 0; c < HC / 32; ++c) {
+        uint32_t r[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+            "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+              "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+              "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+              "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+              "=r"(r[31])
+            : "r"(lane_base + (uint32_t)(c * 32)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+        if (p.D_f32 && !bad && row < p.M) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int64_t col = col0 + c * 32 + 8 * g;
+                if (col >= p.N) break;
+                float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
+                d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
+                d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+    }
+    // accumulator drained: the next tile's MMAs may overwrite it
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+        // a peer CTA's arrival needs no cluster-scope release: tcgen05.wait::ld
+        // has completed the reads of the accumulator it announces
+        if (remote)
+            asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(acc_empty)
+                         : "memory");
+        else
+            mbar_arrive(acc_empty);
+    }
+    if (p.D_bf16 && !bad && row0 < p.M) {
+        const uint32_t sw = (uint32_t)((lane >> 2) & 1);
+#pragma unroll
+        for (int h = 0; h < HC / 16; ++h) {
+            if (col0 + 16 * h >= p.N) break;
+            if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                st_shared_v4(buf + (uint32_t)lane * 32u + (((uint32_t)j ^ sw) << 4),
+                             packed[8 * h + 4 * j], packed[8 * h + 4 * j + 1],
+                             packed[8 * h + 4 * j + 2], packed[8 * h + 4 * j + 3]);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(tmD, buf, (int)(col0 + 16 * h), (int)row0);
+                bulk_commit();
+            }
+        }
+    }
+}
+
 constexpr int kGemmThreads = 448;
 
 template <int BN, int STAGES>
@@ -430,72 +516,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             __syncwarp();
             if (!acc_ok) timed_out = 1;
             const bool bad = *(volatile int*)&timed_out != 0;
-            const int64_t row = m0 + 32 * q + lane;
-            const int64_t col0 = n0 + half * HC;
-            uint32_t packed[HC / 2];  // bf16 pairs of this thread's row
-#pragma unroll
-            for (int c = 0; c < HC / 32; ++c) {
-                uint32_t r[32];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-                    "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                    : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                      "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-                      "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-                      "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-                      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-                      "=r"(r[31])
-                    : "r"(lane_base + (uint32_t)(c * 32)));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-                if (p.D_f32 && !bad && row < p.M) {
-                    // fp32 output (checking path): stored before TMEM is released
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int64_t col = col0 + c * 32 + 8 * g;
-                        if (col >= p.N) break;
-                        float4* d = reinterpret_cast<float4*>(p.D_f32 + row * p.N + col);
-                        d[0] = make_float4(v[8 * g], v[8 * g + 1], v[8 * g + 2], v[8 * g + 3]);
-                        d[1] = make_float4(v[8 * g + 4], v[8 * g + 5], v[8 * g + 6], v[8 * g + 7]);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-                    packed[c * 16 + i] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-            }
-            // accumulator drained: the next tile's MMAs may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&S.acc_empty));
-            if (p.D_bf16 && !bad && m0 + 32 * q < p.M) {
-                // stage 32 rows x 16 columns at a time in this warp's buffer (row = lane,
-                // 16-byte half j of a row at half j ^ ((row / 4) % 2): the 32-byte swizzle
-                // the store's tensor map undoes; conflict-free), then one bulk tensor
-                // store; rows and columns past M and N are clipped by the tensor map.
-                const uint32_t buf = smem_addr(S.dstage[warp - 6]);
-                const uint32_t sw = (uint32_t)((lane >> 2) & 1);
-#pragma unroll
-                for (int h = 0; h < HC / 16; ++h) {
-                    if (col0 + 16 * h >= p.N) break;
-                    if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 2; ++j)
-                        st_shared_v4(buf + (uint32_t)lane * 32u + (((uint32_t)j ^ sw) << 4),
-                                     packed[8 * h + 4 * j], packed[8 * h + 4 * j + 1],
-                                     packed[8 * h + 4 * j + 2], packed[8 * h + 4 * j + 3]);
-                    fence_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmD, buf, (int)(col0 + 16 * h), (int)(m0 + 32 * q));
-                        bulk_commit();
-                    }
-                }
-            }
+            epilogue_tile<BN>(lane_base, m0 + 32 * q, n0 + half * HC, p, alpha, bad,
+                              smem_addr(&S.acc_empty), 0u, smem_addr(S.dstage[warp - 6]), &tmD);
         }
         if (lane == 0) bulk_wait_all();  // every store of this warp has landed
         __syncwarp();
@@ -508,6 +530,374 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"((uint32_t)TL::kAlloc)
+                     : "memory");
+    }
+}
+
+// ============================================================================
+// Two-SM variant.  A cluster of two CTAs computes 256 x 256 output tiles with
+// tcgen05.mma.cta_group::2 (M = 256, 128 rows per CTA; N = 256).  Each CTA
+// loads its own 128 rows of A and its own 128 of the tile's 256 rows of B, so an
+// SM streams 32 KB of operands per 256-deep k-tile instead of 48 KB, and the
+// pair's MMA reads both halves of B.  The roles are those of the kernel above in
+// each CTA; the leader (cluster rank 0) issues the MMAs, the operand copies of
+// both CTAs complete on the leader's stage barrier, the scale writers and
+// epilogue warps of both CTAs arrive on the leader's barriers, and the leader's
+// commits arrive on the barriers of both CTAs.  No copy is multicast.
+// ============================================================================
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on the peer's barrier without a cluster-scope release: used after
+// tcgen05.wait::st, which has already completed the TMEM writes it announces.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Tile load into this CTA's shared memory whose bytes complete on a barrier of
+// either CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+// Arrive (once the pair's MMAs issued so far complete) on the barrier at this
+// shared-memory offset in both CTAs.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+// The four K = 64 steps of one k-tile, as tc_mma_nvf4_x4 (N = 256: B scales
+// advance by 8 columns per step).
+__device__ __forceinline__ void tc_mma_nvf4_pair_x4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                    uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                                    uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        ".reg .b32 sa1, sa2, sa3, sb1, sb2, sb3;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "setp.eq.b32 q, %3, %3;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.u32 sa1, %4, 4;\n\tadd.u32 sa2, %4, 8;\n\tadd.u32 sa3, %4, 12;\n\t"
+        "add.u32 sb1, %5, 8;\n\tadd.u32 sb2, %5, 16;\n\tadd.u32 sb3, %5, 24;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a1, b1, %3, [sa1], [sb1], q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a2, b2, %3, [sa2], [sb2], q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], a3, b3, %3, [sa3], [sb3], q;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+// Pair MMA: M = 256 (both CTAs), N = 256, E2M1 x E2M1, UE4M3 scales, K-major.
+constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                ((uint32_t)(256 >> 4) << 24);
+
+template <int STAGES>
+struct __align__(1024) PairSmem {
+    uint8_t a[STAGES][128 * kBKBytes];       // this CTA's 128 rows of A, 16 KB / stage
+    uint8_t b[STAGES][128 * kBKBytes];       // this CTA's 128 rows of B, 16 KB / stage
+    uint8_t dstage[8][32 * 32];              // per epilogue warp: 32 rows x 16 bf16, 32B-swizzled
+    uint8_t sfa[STAGES][4 * 512];            // scales of this CTA's A rows
+    uint8_t sfb[STAGES][2][4 * 512];         // scales of all 256 B rows of the tile
+    uint64_t full[STAGES];       // leader: A/B bytes of both CTAs landed
+    uint64_t sf_loaded[STAGES];  // this CTA's scale atoms landed
+    uint64_t empty[STAGES];      // stage free (leader's commit, both CTAs)
+    uint64_t sf_full[STAGES];    // leader: TMEM scales of both CTAs written (8 warps)
+    uint64_t acc_full;           // accumulator ready (leader's commit, both CTAs)
+    uint64_t acc_empty;          // leader: accumulators of both CTAs drained (16 warps)
+    uint32_t tmem_base;
+};
+
+constexpr int kPairThreads = 480;  // the warps of the one-SM kernel + a scale-copy producer
+
+template <int STAGES>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
+    using Smem = PairSmem<STAGES>;
+    constexpr int BN = 256, G = 2, HC = BN / 2;
+    constexpr int kSfaCols = 16, kRegion = 48;              // per stage: A scales, then B scales
+    constexpr int kUsed = BN + STAGES * kRegion;
+    static_assert(kUsed <= 512, "TMEM holds 512 columns");
+    constexpr uint32_t kAlloc = 512;
+    extern __shared__ uint8_t smem_raw[];
+    Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int64_t katoms = p.K / 64;
+    const int KT = (int)((p.K + 255) / 256);
+    const int64_t na_groups = (p.M + 127) / 128, nb_groups = (p.N + 127) / 128;
+    const int64_t tiles_n = (p.N + BN - 1) / BN;
+    const int64_t tiles = ((p.M + 255) / 256) * tiles_n;
+    const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_addr(&S.full[s]), 1);
+            mbar_init(smem_addr(&S.sf_loaded[s]), 1);
+            mbar_init(smem_addr(&S.empty[s]), 1);
+            mbar_init(smem_addr(&S.sf_full[s]), 8);
+        }
+        mbar_init(smem_addr(&S.acc_full), 1);
+        mbar_init(smem_addr(&S.acc_empty), 16);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&S.tmem_base)),
+                     "r"(kAlloc)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    __shared__ int timed_out;
+    if (threadIdx.x == 0) timed_out = 0;
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ A/B producer (both CTAs)
+            const uint32_t full_l0 = mapa_shared(smem_addr(&S.full[0]), 0);
+            const uint32_t empty0 = smem_addr(&S.empty[0]);
+            uint32_t s = 0, ph = 0;
+            int64_t issued = 0;
+            for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
+                const int64_t m0 = (pt / tiles_n) * 256, n0 = (pt % tiles_n) * BN;
+                for (int kt = 0; kt < KT; ++kt, ++issued) {
+                    if (issued >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u)) {
+                        timed_out = 1;
+                        break;
+                    }
+                    // A and B boxes of both CTAs (rows past M / N are zero-filled and count)
+                    if (leader) mbar_expect_tx(smem_addr(&S.full[s]), 4u * 128u * kBKBytes);
+                    tma_load_2d_pair(smem_addr(S.a[s]), &tmA, kt * kBKBytes, (int)(m0 + 128 * rank),
+                                     full_l0 + 8u * s);
+                    tma_load_2d_pair(smem_addr(S.b[s]), &tmB, kt * kBKBytes, (int)(n0 + 128 * rank),
+                                     full_l0 + 8u * s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (*(volatile int*)&timed_out && leader) {
+                // let copies already issued land before the CTA can exit
+                for (int64_t k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k)
+                    mbar_wait(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 14) {
+        if (lane == 0) {
+            // ------------------------------------------------ scale-atom producer (both CTAs)
+            // One thread issuing every copy of a stage was the pipeline's limit;
+            // the scale atoms have their own thread and barrier.
+            const uint32_t sfl0 = smem_addr(&S.sf_loaded[0]), empty0 = smem_addr(&S.empty[0]);
+            uint32_t s = 0, ph = 0;
+            int64_t issued = 0;
+            for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
+                const int64_t m0 = (pt / tiles_n) * 256, n0 = (pt % tiles_n) * BN;
+                const int64_t a_group = (m0 + 128 * rank) / 128;
+                for (int kt = 0; kt < KT; ++kt, ++issued) {
+                    if (issued >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u)) {
+                        timed_out = 1;
+                        break;
+                    }
+                    const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
+                    const uint32_t sf_bytes = (uint32_t)(rem < 4 ? rem : 4) * 512u;
+                    uint32_t bytes = a_group < na_groups ? sf_bytes : 0u;
+                    for (int g = 0; g < G; ++g)
+                        if (n0 / 128 + g < nb_groups) bytes += sf_bytes;
+                    const uint32_t sb = sfl0 + 8u * s;
+                    mbar_expect_tx(sb, bytes);
+                    if (a_group < na_groups)
+                        bulk_load(smem_addr(S.sfa[s]), p.sfA + (a_group * katoms + (int64_t)kt * 4) * 512,
+                                  sf_bytes, sb);
+                    for (int g = 0; g < G; ++g)
+                        if (n0 / 128 + g < nb_groups)
+                            bulk_load(smem_addr(S.sfb[s][g]),
+                                      p.sfB + ((n0 / 128 + g) * katoms + (int64_t)kt * 4) * 512, sf_bytes, sb);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (*(volatile int*)&timed_out) {
+                for (int64_t k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k)
+                    mbar_wait(sfl0 + 8u * (uint32_t)(k % STAGES), (uint32_t)(k / STAGES) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (leader)
+            constexpr uint64_t kStep = (128 * kBKBytes) >> 4;
+            const uint64_t adesc0 = operand_desc(smem_addr(S.a[0]));
+            const uint64_t bdesc0 = operand_desc(smem_addr(S.b[0]));
+            const uint32_t tsf0 = tmem + (uint32_t)BN;
+            const uint32_t sf_full0 = smem_addr(&S.sf_full[0]), empty0 = smem_addr(&S.empty[0]);
+            const int KT_full = (int)(p.K / 256);
+            uint32_t s = 0, ph = 0;
+            uint32_t local = 0;
+            for (int64_t pt = cid; pt < tiles; pt += ncl, ++local) {
+                if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u)) {
+                    timed_out = 1;
+                    break;
+                }
+                tc_fence_after();
+                bool bad = false;
+                for (int kt = 0; kt < KT; ++kt) {
+                    if (!mbar_wait(sf_full0 + 8u * s, ph)) {
+                        bad = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = adesc0 + kStep * s, bd = bdesc0 + kStep * s;
+                    const uint32_t t_sfa = tsf0 + (uint32_t)kRegion * s;
+                    const uint32_t t_sfb = t_sfa + kSfaCols;
+                    if (kt < KT_full) {
+                        tc_mma_nvf4_pair_x4(tmem, ad, bd, kIdescPair, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
+                    } else {  // K tail: 1 to 3 steps of 64
+                        const int nks = (int)((p.K - (int64_t)kt * 256) / kKStep);
+                        for (int j = 0; j < nks; ++j)
+                            tc_mma_nvf4_pair(tmem, ad + 2u * j, bd + 2u * j, kIdescPair, t_sfa + 4 * j,
+                                             t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(empty0 + 8u * s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                tc_commit_pair(smem_addr(&S.acc_full));
+                if (bad) {
+                    timed_out = 1;
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ---------------------------------------------------- scale writers (warps 2-5, both CTAs)
+        // Into this CTA's TMEM: the A scales of its own 128 rows and the B scales
+        // of all 256 rows of the tile, in the layout of the one-SM kernel.  The
+        // leader's writers also wait for the A/B bytes of both CTAs, so the
+        // issuer needs only the sf_full barrier.  Region s was last read by the
+        // previous use of stage s, whose commit the producer waited for before
+        // refilling the stage's scale atoms.
+        const int q = warp & 3;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        const int64_t my_tiles = cid < tiles ? (tiles - cid + ncl - 1) / ncl : 0;
+        const int64_t total = my_tiles * KT;
+        const uint32_t sfl0 = smem_addr(&S.sf_loaded[0]), full0 = smem_addr(&S.full[0]);
+        const uint32_t sf_full_local0 = smem_addr(&S.sf_full[0]);
+        const uint32_t sf_full_l0 = mapa_shared(sf_full_local0, 0);
+        uint32_t s = 0, ph = 0;
+        for (int64_t it = 0; it < total; ++it) {
+            if (!mbar_wait(sfl0 + 8u * s, ph) || (leader && !mbar_wait(full0 + 8u * s, ph))) {
+                timed_out = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t col = (uint32_t)(BN + kRegion * s);
+            uint32_t v[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 w = *reinterpret_cast<const uint4*>(S.sfa[s] + j * 512 + lane * 16);
+                v[4 * j] = w.x; v[4 * j + 1] = w.y; v[4 * j + 2] = w.z; v[4 * j + 3] = w.w;
+            }
+            tc_st16(lane_base + col, v);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {  // 16 columns: k-steps and groups, order 4*G*j + 4*g
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int idx = h * 4 + jj;
+                    const int j = idx / G, g = idx % G;
+                    const uint4 w = *reinterpret_cast<const uint4*>(S.sfb[s][g] + j * 512 + lane * 16);
+                    v[4 * jj] = w.x; v[4 * jj + 1] = w.y; v[4 * jj + 2] = w.z; v[4 * jj + 3] = w.w;
+                }
+                tc_st16(lane_base + col + kSfaCols + 16 * h, v);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(sf_full_local0 + 8u * s);
+                else
+                    mbar_arrive_cluster_relaxed(sf_full_l0 + 8u * s);
+            }
+            if (++s == STAGES) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (warps 6-13, both CTAs)
+        const int q = warp & 3;
+        const int half = (warp - 6) >> 2;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
+        const uint32_t acc_empty_l = leader ? smem_addr(&S.acc_empty) : mapa_shared(smem_addr(&S.acc_empty), 0);
+        float alpha = p.alpha;
+        if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
+        if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
+        uint32_t local = 0;
+        for (int64_t pt = cid; pt < tiles; pt += ncl, ++local) {
+            if (*(volatile int*)&timed_out) break;
+            const int64_t m0 = (pt / tiles_n) * 256, n0 = (pt % tiles_n) * BN;
+            const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u);
+            tc_fence_after();
+            __syncwarp();
+            if (!acc_ok) timed_out = 1;
+            const bool bad = *(volatile int*)&timed_out != 0;
+            epilogue_tile<BN>(lane_base, m0 + 128 * rank + 32 * q, n0 + half * HC, p, alpha, bad,
+                              acc_empty_l, leader ? 0u : 1u, smem_addr(S.dstage[warp - 6]), &tmD);
+        }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && *(volatile int*)&timed_out) set_status(p.status, kStatusTimeout);
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs done: no MMA, commit or remote arrive pending
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAlloc)
                      : "memory");
     }
 }
@@ -576,7 +966,48 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream
     return cudaGetLastError();
 }
 
+template <int STAGES>
+static cudaError_t launch_gemm_pair(const GemmParams& p, int sm_count, cudaStream_t st) {
+    CUtensorMap ma, mb, md;
+    if (!make_operand_map(&ma, p.A, p.M, p.K / 2, 128) || !make_operand_map(&mb, p.B, p.N, p.K / 2, 128))
+        return cudaErrorInvalidValue;
+    memset(&md, 0, sizeof(md));
+    if (p.D_bf16 && !make_output_map(&md, p.D_bf16, p.M, p.N)) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(PairSmem<STAGES>) + 1024;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<STAGES>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int64_t tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kPairThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many clusters as can be resident at once (an SM left over
+    // in a GPC cannot host half a pair), never more than there are tiles
+    static int resident = 0;
+    if (resident == 0) {
+        cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
+        if (cudaOccupancyMaxActiveClusters(&resident, gemm_nvf4_pair_kernel<STAGES>, &cfg) != cudaSuccess ||
+            resident < 1)
+            resident = sm_count / 2;
+    }
+    cfg.gridDim = dim3((unsigned)(2 * (tiles < resident ? tiles : resident)));
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<STAGES>, ma, mb, md, p);
+}
+
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
+    if (p.M > 128 && sm_count >= 2) return launch_gemm_pair<5>(p, sm_count, st);
     return launch_gemm_cfg<256, 4>(p, sm_count, st);
 }
 
