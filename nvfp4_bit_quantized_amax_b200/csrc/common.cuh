@@ -141,24 +141,36 @@ __device__ __forceinline__ uint32_t draw16(const Philox4& p, int j) {
     return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
 }
 
-// Stochastic rounding of v straight to its E2M1 code.  Let a = min(|v|, 6) and
-// lo <= a <= hi the adjacent grid points; the rule rounds up iff r < p * 2^16
-// with p = (a - lo) / (hi - lo) and r the 16-bit draw.  The map c(a) = 2a on
-// [0, 2], a + 2 on [2, 4], a / 2 + 4 on [4, 6] is affine between grid points and
-// sends the grid {0, .5, 1, 1.5, 2, 3, 4, 6} to the codes 0..7, so floor(c(a))
-// is the code of lo and frac(c(a)) is p.  With C = ceil(c(a) * 2^16), one fp32
-// FMA rounded upward (a times a power of two plus an integer, below 2^24, so the
-// only rounding is the ceiling), the code is floor(c) + [r < p * 2^16] =
-// (C + 65535 - r) >> 16; grid points (p = 0) never move.  The sign bit of v is
-// kept, zero included.
-__device__ __forceinline__ uint32_t sr_e2m1_code(float v, uint32_t r16) {
-    const float a = fminf(fabsf(v), 6.0f);
-    const bool lo2 = a < 2.0f, lo4 = a < 4.0f;
-    const float rs = lo2 ? 131072.0f : (lo4 ? 65536.0f : 32768.0f);      // slope * 2^16
-    const float b = lo2 ? 8388608.0f : (lo4 ? 8519680.0f : 8650752.0f);  // 2^23 + offset * 2^16
-    const uint32_t c = __float_as_uint(__fmaf_ru(a, rs, b));             // bits of 2^23 + C
-    const uint32_t code = (c - (0x4B000000u - 65535u) - r16) >> 16;
-    return code | ((__float_as_uint(v) >> 28) & 8u);
+// Stochastic rounding of eight values straight to packed E2M1 codes (element i
+// in bits [4i, 4i+4), sign bit of v kept, zero included).  Let a = min(|v|, 6)
+// and lo <= a <= hi the adjacent grid points; the rule rounds up iff
+// r < p * 2^16 with p = (a - lo) / (hi - lo) and r the 16-bit draw.  The map
+// c(a) = min(2a, a + 2, a / 2 + 4, 7) is affine between grid points and sends the
+// grid {0, .5, 1, 1.5, 2, 3, 4, 6} to the codes 0..7, so floor(c(a)) is the code
+// of lo and frac(c(a)) is p; hence code = floor(c) + [r < p * 2^16] =
+// (ceil(c * 2^16) + 65535 - r) >> 16, and grid points (p = 0) never move.  Each
+// line is one fp32 FMA rounded upward with 2^23 + offset * 2^16 + 65535 as its
+// addend (integers below 2^24, so the only rounding is the ceiling, and the
+// ceiling commutes with the minimum); the float's bits minus r then carry the
+// code in byte 2.  Byte permutes gather the codes and the sign bits.
+__device__ __forceinline__ uint32_t sr_e2m1x8(const float (&v)[8], const Philox4& rnd) {
+    uint32_t e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float a = fabsf(v[i]);
+        const float t = fminf(fminf(__fmaf_ru(a, 131072.0f, 8454143.0f), __fmaf_ru(a, 65536.0f, 8585215.0f)),
+                              fminf(__fmaf_ru(a, 32768.0f, 8716287.0f), 8912895.0f));
+        e[i] = __float_as_uint(t) - draw16(rnd, i);
+    }
+    const uint32_t ce = __byte_perm(__byte_perm(e[0], e[2], 0x0062), __byte_perm(e[4], e[6], 0x0062), 0x5410);
+    const uint32_t co = __byte_perm(__byte_perm(e[1], e[3], 0x0062), __byte_perm(e[5], e[7], 0x0062), 0x5410);
+    const uint32_t se = __byte_perm(__byte_perm(__float_as_uint(v[0]), __float_as_uint(v[2]), 0x0073),
+                                    __byte_perm(__float_as_uint(v[4]), __float_as_uint(v[6]), 0x0073), 0x5410);
+    const uint32_t so = __byte_perm(__byte_perm(__float_as_uint(v[1]), __float_as_uint(v[3]), 0x0073),
+                                    __byte_perm(__float_as_uint(v[5]), __float_as_uint(v[7]), 0x0073), 0x5410);
+    const uint32_t even = ce | ((se >> 4) & 0x08080808u);  // element 2k in byte k, sign in bit 3
+    const uint32_t odd = co | ((so >> 4) & 0x08080808u);
+    return even + (odd << 4);
 }
 
 // ---------------------------------------------------------------- scale layout

@@ -126,11 +126,10 @@ __device__ __forceinline__ uint32_t encode8(const float (&v)[8], float inv, bool
         for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
         return e2m1x8_rn(q);
     }
-    const Philox4 r = sr_draws8(rk, stream, e0 >> 3);
-    uint32_t out = 0;
+    float q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) out |= sr_e2m1_code(__fmul_rn(v[i], inv), draw16(r, i)) << (4 * i);
-    return out;
+    for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
+    return sr_e2m1x8(q, sr_draws8(rk, stream, e0 >> 3));
 }
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&v)[8]) {
