@@ -334,13 +334,14 @@ def run_ours(args, rank, world, local_rank):
 
 
 def moe_step_bench(capi, syn, dev, stream, timed, max_over_ranks, world, iters):
-    """Expert layer of the MoE config: gather routed token rows, per-expert NVFP4
-    fprop / dgrad / wgrad, combine the routed input gradients.  Useful FLOPs count
-    the routed tokens only (padding rows excluded)."""
+    """Expert layer of the MoE config: gather routed token rows, NVFP4 fprop / dgrad /
+    wgrad of all experts (grouped: one launch per kernel kind over all experts), and
+    combine the routed input gradients.  Useful FLOPs count the routed tokens only
+    (padding rows excluded).  The per-expert calls are timed beside it."""
     import torch
     s = syn.MOE
     E, K, N, T, k = s["experts"], s["hidden"], s["ffn"], s["tokens"], s["topk"]
-    d = syn.moe_inputs(T, E, K, N, k, s["zipf_s"], seed=0)
+    d = syn.moe_inputs(T, E, K, N, k, s["zipf_s"], seed=0, pad=128)
     rows = int(d["group_rows"].sum())
 
     def to_dev(b):
@@ -356,24 +357,37 @@ def moe_step_bench(capi, syn, dev, stream, timed, max_over_ranks, world, iters):
     dX = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
     dX_tok = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
     dW = torch.empty((E, N, K), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(capi.moe_workspace_bytes(d["group_rows"], K, N), dtype=torch.uint8, device=dev)
+    gws = torch.empty(capi.moe_grouped_workspace_bytes(d["group_rows"], K, N), dtype=torch.uint8,
+                      device=dev)
     signs = syn.rht_signs(0)
 
     def step():
         capi.nvfp4_moe_gather(x_tok, row_src, X_perm)
-        capi.nvfp4_moe_linear_fprop(X_perm, W, Y, d["group_rows"], signs, ws)
-        capi.nvfp4_moe_linear_dgrad(dY, dX, d["group_rows"], 7, signs, ws)
+        capi.nvfp4_moe_grouped_fprop(X_perm, W, Y, d["group_rows"], signs, gws)
+        capi.nvfp4_moe_grouped_dgrad(dY, dX, d["group_rows"], 7, signs, gws)
         capi.nvfp4_moe_combine(dX, slots, dX_tok)
-        capi.nvfp4_moe_linear_wgrad(dW, d["group_rows"], 7, signs, ws)
+        capi.nvfp4_moe_grouped_wgrad(dW, d["group_rows"], gws)
 
     ms = max_over_ranks(timed(step, iters, 3))
+    assert capi.nvfp4_read_status(gws) == 0
+    pws = torch.empty(capi.moe_workspace_bytes(d["group_rows"], K, N), dtype=torch.uint8, device=dev)
+
+    def step_per_expert():
+        capi.nvfp4_moe_gather(x_tok, row_src, X_perm)
+        capi.nvfp4_moe_linear_fprop(X_perm, W, Y, d["group_rows"], signs, pws)
+        capi.nvfp4_moe_linear_dgrad(dY, dX, d["group_rows"], 7, signs, pws)
+        capi.nvfp4_moe_combine(dX, slots, dX_tok)
+        capi.nvfp4_moe_linear_wgrad(dW, d["group_rows"], 7, signs, pws)
+
+    ms_pe = max_over_ranks(timed(step_per_expert, 3, 1))
     useful = 3 * 2.0 * T * k * K * N
     padded = 3 * 2.0 * rows * K * N
     return {"workload": "MoE expert layer: 64 experts, hidden 2048, FFN 1024, 16384 tokens, "
-                        "top-4 of Zipf(1.1)",
+                        "top-4 of Zipf(1.1), expert segments padded to 128 rows",
             "ms_per_step": round(ms, 4),
             "useful_tflops": round(world * useful / (ms * 1e-3) / 1e12, 1),
             "executed_tflops_incl_padding": round(world * padded / (ms * 1e-3) / 1e12, 1),
+            "per_expert_calls_ms_per_step": round(ms_pe, 4),
             "routed_rows": T * k, "padded_rows": rows,
             "group_rows_max_min": [int(d["group_rows"].max()), int(d["group_rows"].min())]}
 

@@ -204,6 +204,36 @@ int nvfp4_moe_linear_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K
                            uint64_t seed, const int8_t* rht_signs, void* ws, size_t ws_bytes,
                            nvfp4_stream_t stream);
 /*
+ * Grouped expert layer: the computation of nvfp4_moe_linear_* (each expert a linear
+ * layer with its own tensor scales; expert e draws stochastic rounding with seed + e
+ * and counts element indices inside its own tensors, so the codes, scales and
+ * outputs equal the per-expert calls'), with every step one launch over all experts:
+ * the permuted tensors are quantized whole, in both orientations, with per-expert
+ * tensor scales, and one persistent GEMM walks the tiles of all experts.  (The
+ * explainer's "The model underneath": most of the FP4 FLOPs are expert GEMMs.)
+ *   group_rows: HOST array of E entries, each a multiple of 128 (0 allowed), their
+ *   sum R >= 128; K, N multiples of 128.  X_perm [R][K], Y_perm / dY_perm [R][N],
+ *   dX_perm [R][K] bf16 in expert order; W, dW [E][N][K] bf16.
+ *   ws: nvfp4_moe_grouped_workspace_bytes() bytes, 256-byte aligned; its status word
+ *   is read with nvfp4_read_status.  fprop fills the X and W operands, dgrad the dY
+ *   operands and wgrad reads both (call them in that order on one workspace).  The
+ *   dW of an expert with no rows is written as zero.
+ *   nvfp4_moe_grouped_operand: views (NVFP4_LIN_*) of the whole quantized tensors,
+ *   X [R][K], X^T [K][R], W [E*N][K], W^T [K][E*N], dY [R][N], dY^T [N][R]; a view's
+ *   tensor_scale points at E floats, one per expert.  No device access.
+ */
+size_t nvfp4_moe_grouped_workspace_bytes(const int64_t* group_rows, int E, int64_t K, int64_t N);
+int nvfp4_moe_grouped_operand(void* ws, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                              int which, nvfp4_tensor* out);
+int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, const int64_t* group_rows,
+                            int E, int64_t K, int64_t N, const int8_t* rht_signs, void* ws,
+                            size_t ws_bytes, nvfp4_stream_t stream);
+int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
+                            int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
+                            size_t ws_bytes, nvfp4_stream_t stream);
+int nvfp4_moe_grouped_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                            void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+/*
  * nvfp4_moe_gather: dst[i] = src[row_src[i]] for rows of `cols` bf16 (row_src device
  * int32 [rows]; -1 writes a zero row).  cols % 8 == 0.
  * nvfp4_moe_combine: dst[t] = bf16(sum over j < topk of src[slots[t*topk + j]]) with an

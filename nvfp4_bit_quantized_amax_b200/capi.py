@@ -29,6 +29,8 @@ EXPORTS = (
     "nvfp4_status_string", "nvfp4_version", "nvfp4_quantize_noalloc",
     "nvfp4_moe_workspace_bytes", "nvfp4_moe_expert_workspace", "nvfp4_moe_linear_fprop",
     "nvfp4_moe_linear_dgrad", "nvfp4_moe_linear_wgrad", "nvfp4_moe_gather", "nvfp4_moe_combine",
+    "nvfp4_moe_grouped_workspace_bytes", "nvfp4_moe_grouped_operand", "nvfp4_moe_grouped_fprop",
+    "nvfp4_moe_grouped_dgrad", "nvfp4_moe_grouped_wgrad",
 )
 
 
@@ -88,6 +90,11 @@ def load(path: str = LIB_PATH):
         "nvfp4_moe_linear_wgrad": (ci, [vp, vp, ci, i64, i64, u64, vp, vp, sz, vp]),
         "nvfp4_moe_gather": (ci, [vp, vp, i64, i64, vp, vp]),
         "nvfp4_moe_combine": (ci, [vp, vp, i64, ci, i64, vp, vp]),
+        "nvfp4_moe_grouped_workspace_bytes": (sz, [vp, ci, i64, i64]),
+        "nvfp4_moe_grouped_operand": (ci, [vp, vp, ci, i64, i64, ci, C.POINTER(Tensor)]),
+        "nvfp4_moe_grouped_fprop": (ci, [vp, vp, vp, vp, ci, i64, i64, vp, vp, sz, vp]),
+        "nvfp4_moe_grouped_dgrad": (ci, [vp, vp, vp, ci, i64, i64, u64, vp, vp, sz, vp]),
+        "nvfp4_moe_grouped_wgrad": (ci, [vp, vp, ci, i64, i64, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -280,6 +287,48 @@ def nvfp4_moe_linear_wgrad(dW, group_rows, seed, rht_signs, ws, stream=None):
         _ptr(dW), gp, E, K, N, seed, sp, _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
     del keep, g
+
+
+def moe_grouped_workspace_bytes(group_rows, K, N):
+    g, gp = _rows(group_rows)
+    return load().nvfp4_moe_grouped_workspace_bytes(gp, len(g), K, N)
+
+
+def nvfp4_moe_grouped_operand(ws, group_rows, K, N, which):
+    g, gp = _rows(group_rows)
+    t = Tensor()
+    _check("nvfp4_moe_grouped_operand", load().nvfp4_moe_grouped_operand(
+        C.c_void_p(ws.data_ptr()), gp, len(g), K, N, which, C.byref(t)))
+    return t
+
+
+def nvfp4_moe_grouped_fprop(X_perm, W, Y_perm, group_rows, rht_signs, ws, stream=None):
+    g, gp = _rows(group_rows)
+    E, N, K = W.shape
+    keep, sp = _signs(rht_signs)
+    _check("nvfp4_moe_grouped_fprop", load().nvfp4_moe_grouped_fprop(
+        _ptr(X_perm), _ptr(W), _ptr(Y_perm), gp, E, K, N, sp, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep, g
+
+
+def nvfp4_moe_grouped_dgrad(dY_perm, dX_perm, group_rows, seed, rht_signs, ws, stream=None):
+    g, gp = _rows(group_rows)
+    K = dX_perm.shape[1]
+    N = dY_perm.shape[1]
+    keep, sp = _signs(rht_signs)
+    _check("nvfp4_moe_grouped_dgrad", load().nvfp4_moe_grouped_dgrad(
+        _ptr(dY_perm), _ptr(dX_perm), gp, len(g), K, N, seed, sp, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep, g
+
+
+def nvfp4_moe_grouped_wgrad(dW, group_rows, ws, stream=None):
+    g, gp = _rows(group_rows)
+    E, N, K = dW.shape
+    _check("nvfp4_moe_grouped_wgrad", load().nvfp4_moe_grouped_wgrad(
+        _ptr(dW), gp, E, K, N, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del g
 
 
 def nvfp4_moe_gather(src, row_src, dst, stream=None):

@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <vector>
+
 #include "../../include/nvfp4.h"
 #include "internal.h"
 
@@ -126,7 +128,7 @@ int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_
 int gemm_call(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
               const float* sa, const float* sb, float alpha, int64_t M, int64_t N, int64_t K,
               void* Dbf, float* Df, int* status, int sms, cudaStream_t st) {
-    GemmParams g;
+    GemmParams g{};
     g.A = A;
     g.sfA = sfA;
     g.B = B;
@@ -519,6 +521,279 @@ int nvfp4_read_status(void* workspace, int* status, nvfp4_stream_t stream) {
         return NVFP4_ERR_CUDA;
     *status = v;
     return NVFP4_OK;
+}
+
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- grouped mixture of experts
+namespace {
+// Workspace of the grouped expert layer: a header (status), per-group amax words
+// and tensor scales, the group tables, then every quantized operand of the whole
+// permuted tensors (rows R = sum of group rows):
+//   X row [R][K], X^T col [K][R] (RHT), W row [E*N][K], W^T col [K][E*N],
+//   dY row [R][N], dY^T col [N][R] (RHT).
+struct MoeLayout {
+    int64_t words_x, words_w, words_dy;          // 2E words each
+    int64_t gx_row, gx_col, gw_row, gw_col, gdy_row, gdy_col;  // E floats each
+    int64_t mtile_group, group_row0, group_nrows;
+    int64_t x_row, x_row_sf, x_col, x_col_sf, w_row, w_row_sf, w_col, w_col_sf;
+    int64_t dy_row, dy_row_sf, dy_col, dy_col_sf, total;
+    int64_t R;
+};
+MoeLayout moe_layout(const int64_t* group_rows, int E, int64_t K, int64_t N) {
+    MoeLayout L;
+    L.R = 0;
+    for (int e = 0; e < E; ++e) L.R += group_rows[e];
+    int64_t off = 256;  // header: status word
+    auto take = [&](int64_t bytes) {
+        const int64_t o = off;
+        off = pad(off + (bytes > 0 ? bytes : 1), 256);
+        return o;
+    };
+    L.words_x = take(8 * E);
+    L.words_w = take(8 * E);
+    L.words_dy = take(8 * E);
+    L.gx_row = take(4 * E);
+    L.gx_col = take(4 * E);
+    L.gw_row = take(4 * E);
+    L.gw_col = take(4 * E);
+    L.gdy_row = take(4 * E);
+    L.gdy_col = take(4 * E);
+    L.mtile_group = take(4 * (L.R / 128));
+    L.group_row0 = take(8 * E);
+    L.group_nrows = take(8 * E);
+    const int64_t R = L.R, EN = (int64_t)E * N;
+    L.x_row = take(R * K / 2);
+    L.x_row_sf = take((int64_t)nvfp4_scale_bytes(R, K));
+    L.x_col = take(K * R / 2);
+    L.x_col_sf = take((int64_t)nvfp4_scale_bytes(K, R));
+    L.w_row = take(EN * K / 2);
+    L.w_row_sf = take((int64_t)nvfp4_scale_bytes(EN, K));
+    L.w_col = take(K * EN / 2);
+    L.w_col_sf = take((int64_t)nvfp4_scale_bytes(K, EN));
+    L.dy_row = take(R * N / 2);
+    L.dy_row_sf = take((int64_t)nvfp4_scale_bytes(R, N));
+    L.dy_col = take(N * R / 2);
+    L.dy_col_sf = take((int64_t)nvfp4_scale_bytes(N, R));
+    L.total = off;
+    return L;
+}
+
+int moe_grouped_check(const int64_t* group_rows, int E, int64_t K, int64_t N) {
+    if (!group_rows || E < 1) return NVFP4_ERR_ARG;
+    if (K < 128 || N < 128 || K % 128 || N % 128) return NVFP4_ERR_SHAPE;
+    int64_t R = 0;
+    for (int e = 0; e < E; ++e) {
+        if (group_rows[e] < 0 || group_rows[e] % 128) return NVFP4_ERR_SHAPE;
+        R += group_rows[e];
+    }
+    if (R < 128 || R > (1ll << 31) - 256) return NVFP4_ERR_SHAPE;
+    return NVFP4_OK;
+}
+
+// Common checks; writes the group tables into the workspace (copied from a host
+// staging buffer on `st`).
+int moe_grouped_begin(const int64_t* group_rows, int E, int64_t K, int64_t N, void* ws,
+                      size_t ws_bytes, cudaStream_t st, MoeLayout* L, int* sms) {
+    int rc = moe_grouped_check(group_rows, E, K, N);
+    if (rc) return rc;
+    *L = moe_layout(group_rows, E, K, N);
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return NVFP4_ERR_ALIGN;
+    if (ws_bytes < (size_t)L->total) return NVFP4_ERR_WORKSPACE;
+    if ((rc = device_check(sms))) return rc;
+    std::vector<int32_t> mt((size_t)(L->R / 128));
+    std::vector<int64_t> r0((size_t)E), nr((size_t)E);
+    int64_t row = 0;
+    for (int e = 0; e < E; ++e) {
+        r0[e] = row;
+        nr[e] = group_rows[e];
+        for (int64_t b = row / 128; b < (row + group_rows[e]) / 128; ++b) mt[(size_t)b] = e;
+        row += group_rows[e];
+    }
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    if (cudaMemcpyAsync(b + L->mtile_group, mt.data(), mt.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(b + L->group_row0, r0.data(), r0.size() * 8, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(b + L->group_nrows, nr.data(), nr.size() * 8, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+// Grouped quantize of one tensor: amax per group, then both orientations.
+int run_quantize_grouped(const void* x, int64_t rows, int64_t cols, bool two_d, int row_sr, int col_sr,
+                         uint64_t seed, int col_rht, uint32_t mask, uint8_t* rd, uint8_t* rsf, float* rg,
+                         uint8_t* cd, uint8_t* csf, float* cg, uint32_t* words, int* status,
+                         const int32_t* row_group, const int64_t* row0, const int64_t* nrows,
+                         int64_t uniform, int sms, cudaStream_t st) {
+    QuantParams p;
+    memset(&p, 0, sizeof p);
+    p.x = static_cast<const uint16_t*>(x);
+    p.rows = rows;
+    p.cols = cols;
+    p.row_data = rd;
+    p.row_sf = rsf;
+    p.row_g = rg;
+    p.col_data = cd;
+    p.col_sf = csf;
+    p.col_g = cg;
+    p.amax_words = words;
+    p.status = status;
+    p.seed = seed;
+    p.row_sr = row_sr;
+    p.col_sr = col_sr;
+    p.col_rht = (col_rht && cd) ? 1 : 0;
+    p.sign_mask = mask;
+    p.row_group = row_group;
+    p.group_row0 = row0;
+    p.group_nrows = nrows;
+    p.group_rows_uniform = uniform;
+    cudaError_t e = launch_amax_grouped(p, sms, st);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    e = launch_quant_tile(p, two_d, st);
+    return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+int moe_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, const float* sa,
+             const float* sb, float alpha, int64_t M, int64_t N, int64_t K, void* D, int* status, int mode,
+             const int32_t* mtile_group, int64_t b_group_rows, int64_t b_group_k, int64_t Kb,
+             const int64_t* k_start, const int64_t* k_len, int groups, int sms, cudaStream_t st) {
+    GemmParams g{};
+    g.A = A;
+    g.sfA = sfA;
+    g.B = B;
+    g.sfB = sfB;
+    g.scale_a = sa;
+    g.scale_b = sb;
+    g.alpha = alpha;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.D_bf16 = D;
+    g.status = status;
+    g.group_mode = mode;
+    g.mtile_group = mtile_group;
+    g.b_group_rows = b_group_rows;
+    g.b_group_k = b_group_k;
+    g.Kb = Kb;
+    g.k_start = k_start;
+    g.k_len = k_len;
+    g.num_groups = groups;
+    return cuda_status(launch_gemm(g, sms, st));
+}
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_moe_grouped_workspace_bytes(const int64_t* group_rows, int E, int64_t K, int64_t N) {
+    if (moe_grouped_check(group_rows, E, K, N)) return 0;
+    return (size_t)moe_layout(group_rows, E, K, N).total;
+}
+
+int nvfp4_moe_grouped_operand(void* ws, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                              int which, nvfp4_tensor* out) {
+    int rc = moe_grouped_check(group_rows, E, K, N);
+    if (rc) return rc;
+    if (!ws || !out || which < 0 || which > 5) return NVFP4_ERR_ARG;
+    const MoeLayout L = moe_layout(group_rows, E, K, N);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    const int64_t R = L.R, EN = (int64_t)E * N;
+    switch (which) {
+        case NVFP4_LIN_X_ROW: *out = {b + L.x_row, b + L.x_row_sf, (float*)(b + L.gx_row), R, K}; break;
+        case NVFP4_LIN_X_COL: *out = {b + L.x_col, b + L.x_col_sf, (float*)(b + L.gx_col), K, R}; break;
+        case NVFP4_LIN_W_ROW: *out = {b + L.w_row, b + L.w_row_sf, (float*)(b + L.gw_row), EN, K}; break;
+        case NVFP4_LIN_W_COL: *out = {b + L.w_col, b + L.w_col_sf, (float*)(b + L.gw_col), K, EN}; break;
+        case NVFP4_LIN_DY_ROW: *out = {b + L.dy_row, b + L.dy_row_sf, (float*)(b + L.gdy_row), R, N}; break;
+        default: *out = {b + L.dy_col, b + L.dy_col_sf, (float*)(b + L.gdy_col), N, R}; break;
+    }
+    return NVFP4_OK;
+}
+
+int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, const int64_t* group_rows,
+                            int E, int64_t K, int64_t N, const int8_t* rht_signs, void* ws,
+                            size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!X_perm || !W || !Y_perm) return NVFP4_ERR_ARG;
+    if (!aligned(X_perm, 16) || !aligned(W, 16) || !aligned(Y_perm, 16)) return NVFP4_ERR_ALIGN;
+    uint32_t mask = 0;
+    if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    MoeLayout L;
+    int sms = 0;
+    int rc = moe_grouped_begin(group_rows, E, K, N, ws, ws_bytes, st, &L, &sms);
+    if (rc) return rc;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(b + 32);  // the word nvfp4_read_status reads
+    if (cudaMemsetAsync(b, 0, 256, st) != cudaSuccess ||
+        cudaMemsetAsync(b + L.words_x, 0, 8 * (size_t)E, st) != cudaSuccess ||
+        cudaMemsetAsync(b + L.words_w, 0, 8 * (size_t)E, st) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const int32_t* mt = reinterpret_cast<const int32_t*>(b + L.mtile_group);
+    const int64_t* r0 = reinterpret_cast<const int64_t*>(b + L.group_row0);
+    const int64_t* nr = reinterpret_cast<const int64_t*>(b + L.group_nrows);
+    // X: rows (1x16 RNE) for fprop, RHT columns (1x16 RNE) for wgrad, per expert
+    rc = run_quantize_grouped(X_perm, L.R, K, false, 0, 0, 0, 1, mask, b + L.x_row, b + L.x_row_sf,
+                              (float*)(b + L.gx_row), b + L.x_col, b + L.x_col_sf, (float*)(b + L.gx_col),
+                              (uint32_t*)(b + L.words_x), status, mt, r0, nr, 0, sms, st);
+    if (rc) return rc;
+    // W [E][N][K] as [E*N][K]: 16x16 RNE, both orientations, per expert
+    rc = run_quantize_grouped(W, (int64_t)E * N, K, true, 0, 0, 0, 0, 0, b + L.w_row, b + L.w_row_sf,
+                              (float*)(b + L.gw_row), b + L.w_col, b + L.w_col_sf, (float*)(b + L.gw_col),
+                              (uint32_t*)(b + L.words_w), status, nullptr, nullptr, nullptr, N, sms, st);
+    if (rc) return rc;
+    // Y rows of expert e = X rows of e times W_e^T
+    return moe_gemm(b + L.x_row, b + L.x_row_sf, b + L.w_row, b + L.w_row_sf, (float*)(b + L.gx_row),
+                    (float*)(b + L.gw_row), 1.0f, L.R, N, K, Y_perm, status, 1, mt, N, 0, 0, nullptr,
+                    nullptr, E, sms, st);
+}
+
+int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
+                            int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
+                            size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!dY_perm || !dX_perm) return NVFP4_ERR_ARG;
+    if (!aligned(dY_perm, 16) || !aligned(dX_perm, 16)) return NVFP4_ERR_ALIGN;
+    uint32_t mask = 0;
+    if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    MoeLayout L;
+    int sms = 0;
+    int rc = moe_grouped_begin(group_rows, E, K, N, ws, ws_bytes, st, &L, &sms);
+    if (rc) return rc;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(b + 32);  // the word nvfp4_read_status reads
+    if (cudaMemsetAsync(b, 0, 256, st) != cudaSuccess ||
+        cudaMemsetAsync(b + L.words_dy, 0, 8 * (size_t)E, st) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const int32_t* mt = reinterpret_cast<const int32_t*>(b + L.mtile_group);
+    const int64_t* r0 = reinterpret_cast<const int64_t*>(b + L.group_row0);
+    const int64_t* nr = reinterpret_cast<const int64_t*>(b + L.group_nrows);
+    // dY: rows (1x16 SR, stream 0) for dgrad, RHT columns (1x16 SR, stream 1) for wgrad;
+    // expert e draws with seed + e
+    rc = run_quantize_grouped(dY_perm, L.R, N, false, 1, 1, seed, 1, mask, b + L.dy_row, b + L.dy_row_sf,
+                              (float*)(b + L.gdy_row), b + L.dy_col, b + L.dy_col_sf, (float*)(b + L.gdy_col),
+                              (uint32_t*)(b + L.words_dy), status, mt, r0, nr, 0, sms, st);
+    if (rc) return rc;
+    // dX rows of expert e = dY rows of e times W_e (B = W^T [K][E*N], columns of e)
+    return moe_gemm(b + L.dy_row, b + L.dy_row_sf, b + L.w_col, b + L.w_col_sf, (float*)(b + L.gdy_row),
+                    (float*)(b + L.gw_col), 1.0f, L.R, K, N, dX_perm, status, 1, mt, 0, N, (int64_t)E * N,
+                    nullptr, nullptr, E, sms, st);
+}
+
+int nvfp4_moe_grouped_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                            void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!dW) return NVFP4_ERR_ARG;
+    if (!aligned(dW, 16)) return NVFP4_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    MoeLayout L;
+    int sms = 0;
+    int rc = moe_grouped_begin(group_rows, E, K, N, ws, ws_bytes, st, &L, &sms);
+    if (rc) return rc;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(b + 32);  // the word nvfp4_read_status reads
+    // dW_e = (dY_e^T D H)(X_e^T D H)^T / 16 over expert e's rows (zero if it has none)
+    return moe_gemm(b + L.dy_col, b + L.dy_col_sf, b + L.x_col, b + L.x_col_sf, (float*)(b + L.gdy_col),
+                    (float*)(b + L.gx_col), 1.0f / 16.0f, N, K, L.R, dW, status, 2, nullptr, 0, 0, 0,
+                    reinterpret_cast<const int64_t*>(b + L.group_row0),
+                    reinterpret_cast<const int64_t*>(b + L.group_nrows), E, sms, st);
 }
 
 }  // extern "C"

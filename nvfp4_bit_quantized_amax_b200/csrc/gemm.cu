@@ -227,7 +227,8 @@ struct TmemLayout {
 
 // ---------------------------------------------------------------- epilogue
 // One epilogue warp's share of a finished tile: its 32 TMEM lanes (rows row0 ..
-// row0+31, lane = row) by BN/2 columns from col0.  Drains the accumulator into
+// row0+31 of D, lane = row) by BN/2 columns from col0; nothing is stored unless
+// `store`, and `zero` writes zeros without reading the accumulator.  Drains the accumulator into
 // registers (times alpha, rounded to bf16; the fp32 checking output is stored
 // before the release), arrives on the accumulator-empty barrier (local, or the
 // leader's at a cluster address when `remote`), then writes the bf16 tile 32 rows x 16 columns
@@ -237,7 +238,7 @@ struct TmemLayout {
 // clipped by the tensor map.
 template <int BN>
 __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, int64_t col0,
-                                              const GemmParams& p, float alpha, bool bad,
+                                              const GemmParams& p, float alpha, bool store, bool zero,
                                               uint32_t acc_empty, uint32_t remote, uint32_t buf,
                                               const CUtensorMap* tmD) {
     constexpr int HC = BN / 2;
@@ -246,6 +247,11 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, 
     uint32_t packed[HC / 2];  // bf16 pairs of this thread's row
 #pragma unroll
     for (int c = 0; c < HC / 32; ++c) {
+        if (zero) {  // a tile with an empty reduction: D = 0, the accumulator is not read
+#pragma unroll
+            for (int i = 0; i < 16; ++i) packed[c * 16 + i] = 0u;
+            continue;
+        }
         uint32_t r[32];
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -261,7 +267,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, 
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-        if (p.D_f32 && !bad && row < p.M) {
+        if (p.D_f32 && store && row < p.M) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 const int64_t col = col0 + c * 32 + 8 * g;
@@ -289,7 +295,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, 
         else
             mbar_arrive(acc_empty);
     }
-    if (p.D_bf16 && !bad && row0 < p.M) {
+    if (p.D_bf16 && store) {
         const uint32_t sw = (uint32_t)((lane >> 2) & 1);
 #pragma unroll
         for (int h = 0; h < HC / 16; ++h) {
@@ -313,6 +319,42 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, 
 
 constexpr int kGemmThreads = 448;
 
+// Operands and result of one 128 x BN output tile (see GemmParams' group modes).
+struct TileJob {
+    int64_t a_row, b_row, d_row, n0;  // first A / B / D row, first D column
+    int64_t k0, k_len;                // reduction range
+    int64_t bk0;                      // extra reduction offset into B
+    int group;                        // -1 when not grouped
+    bool valid;                       // the tile's first row lies inside its problem
+};
+template <int BN>
+__device__ __forceinline__ TileJob tile_job(const GemmParams& p, int64_t tile, int64_t tiles_n,
+                                            int64_t tiles_per_group) {
+    TileJob j;
+    const int64_t t = p.group_mode == 2 ? tile % tiles_per_group : tile;
+    const int64_t m0 = (t / tiles_n) * kBM;
+    j.n0 = (t % tiles_n) * BN;
+    j.a_row = m0;
+    j.b_row = j.n0;
+    j.d_row = m0;
+    j.k0 = 0;
+    j.k_len = p.K;
+    j.bk0 = 0;
+    j.group = -1;
+    j.valid = m0 < p.M;
+    if (p.group_mode == 1) {
+        j.group = p.mtile_group[m0 / kBM];
+        j.b_row = (int64_t)j.group * p.b_group_rows + j.n0;
+        j.bk0 = (int64_t)j.group * p.b_group_k;
+    } else if (p.group_mode == 2) {
+        j.group = (int)(tile / tiles_per_group);
+        j.k0 = p.k_start[j.group];
+        j.k_len = p.k_len[j.group];
+        j.d_row = (int64_t)j.group * p.M + m0;
+    }
+    return j;
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -326,11 +368,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t katoms = p.K / 64;                 // scale atoms per 128-row group
-    const int KT = (int)((p.K + 255) / 256);         // k-tiles of 256
-    const int64_t nb_groups = (p.N + 127) / 128;     // 128-row groups of B
+    const int64_t katoms = p.K / 64;                 // scale atoms per 128-row group of A
+    const int64_t katoms_b = (p.Kb ? p.Kb : p.K) / 64;  // ... and of B
+    const int64_t nb_groups = (p.N + 127) / 128;     // 128-row groups of B (per group)
     const int64_t tiles_n = (p.N + BN - 1) / BN;
-    const int64_t tiles = ((p.M + kBM - 1) / kBM) * tiles_n;
+    const int64_t tiles_per_group = ((p.M + kBM - 1) / kBM) * tiles_n;
+    const int64_t tiles = p.group_mode == 2 ? tiles_per_group * p.num_groups : tiles_per_group;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -363,30 +406,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // ------------------------------------------------ TMA producer
             int64_t it = 0;  // k-tiles issued by this CTA so far (all tiles)
             for (int64_t tile = blockIdx.x; tile < tiles && !*(volatile int*)&timed_out; tile += gridDim.x) {
-                const int64_t m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * BN;
-                for (int kt = 0; kt < KT; ++kt, ++it) {
+                const TileJob jb = tile_job<BN>(p, tile, tiles_n, tiles_per_group);
+                const int KTt = (int)((jb.k_len + 255) / 256);
+                for (int kt = 0; kt < KTt; ++kt, ++it) {
                     const int s = (int)(it % STAGES);
                     const uint32_t use = (uint32_t)(it / STAGES);
                     if (it >= STAGES && !mbar_wait(smem_addr(&S.empty[s]), (use & 1u) ^ 1u)) {
                         timed_out = 1;
                         break;
                     }
-                    const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
+                    const int64_t rem = (jb.k_len - (int64_t)kt * 256) / kKStep;
                     const int nks = rem < 4 ? (int)rem : 4;
                     const uint32_t sf_bytes = (uint32_t)nks * 512u;
                     uint32_t bytes = kBM * kBKBytes + BN * kBKBytes + sf_bytes;
                     for (int g = 0; g < G; ++g)
-                        if (n0 / 128 + g < nb_groups) bytes += sf_bytes;
+                        if (jb.n0 / 128 + g < nb_groups) bytes += sf_bytes;
                     const uint32_t fb = smem_addr(&S.full[s]);
+                    const int64_t katom = jb.k0 / 64 + (int64_t)kt * 4;  // first scale atom of the k-tile
                     mbar_expect_tx(fb, bytes);
-                    tma_load_2d(smem_addr(S.a[s]), &tmA, kt * kBKBytes, (int)m0, fb);
-                    tma_load_2d(smem_addr(S.b[s]), &tmB, kt * kBKBytes, (int)n0, fb);
-                    bulk_load(smem_addr(S.sfa[s]), p.sfA + ((m0 / 128) * katoms + (int64_t)kt * 4) * 512,
+                    tma_load_2d(smem_addr(S.a[s]), &tmA, (int)((jb.k0 / 2) + kt * kBKBytes), (int)jb.a_row, fb);
+                    tma_load_2d(smem_addr(S.b[s]), &tmB, (int)((jb.bk0 + jb.k0) / 2 + kt * kBKBytes), (int)jb.b_row, fb);
+                    bulk_load(smem_addr(S.sfa[s]), p.sfA + ((jb.a_row / 128) * katoms + katom) * 512,
                               sf_bytes, fb);
                     for (int g = 0; g < G; ++g)
-                        if (n0 / 128 + g < nb_groups)
+                        if (jb.n0 / 128 + g < nb_groups)
                             bulk_load(smem_addr(S.sfb[s] + g * 2048),
-                                      p.sfB + ((n0 / 128 + g) * katoms + (int64_t)kt * 4) * 512,
+                                      p.sfB + ((jb.b_row / 128 + g) * katoms_b + jb.bk0 / 64 + katom) * 512,
                                       sf_bytes, fb);
                 }
             }
@@ -411,10 +456,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t bdesc0 = operand_desc(smem_addr(S.b[0]));
             const uint32_t tsf0 = tmem + (uint32_t)BN;
             const uint32_t sf_full0 = smem_addr(&S.sf_full[0]), empty0 = smem_addr(&S.empty[0]);
-            const int KT_full = (int)(p.K / 256);   // k-tiles with all four K = 64 steps
             uint32_t s = 0, ph = 0;                 // stage (= scale region) and its phase
             uint32_t local = 0;  // tiles of this CTA so far
             for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+                const TileJob jb = tile_job<BN>(p, tile, tiles_n, tiles_per_group);
+                const int KT = (int)((jb.k_len + 255) / 256);
+                const int KT_full = (int)(jb.k_len / 256);  // k-tiles with all four K = 64 steps
                 // the epilogue has drained the accumulator of the previous tile
                 if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u)) {
                     timed_out = 1;
@@ -434,7 +481,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (kt < KT_full) {
                         tc_mma_nvf4_x4<G>(tmem, ad, bd, idesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
                     } else {  // K tail: 1 to 3 steps of 64
-                        const int nks = (int)((p.K - (int64_t)kt * 256) / kKStep);
+                        const int nks = (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
                         for (int j = 0; j < nks; ++j)
                             tc_mma_nvf4(tmem, ad + 2u * j, bd + 2u * j, idesc, t_sfa + 4 * j,
                                         t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
@@ -461,8 +508,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // layout the block-scaled MMA reads (row l + 32i in column i).
         const int q = warp & 3;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        const int64_t total = ((tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) * KT;
-        for (int64_t it = 0; it < total; ++it) {
+        int64_t it = 0;
+        bool stop = false;
+        for (int64_t tile = blockIdx.x; tile < tiles && !stop; tile += gridDim.x)
+        for (int kt = (int)((tile_job<BN>(p, tile, tiles_n, tiles_per_group).k_len + 255) / 256); kt > 0; --kt, ++it) {
             const int s = (int)(it % STAGES), r = (int)(it % R);
             // Region r was last read by the MMAs of k-tile it - R.  With R == STAGES
             // those MMAs completed before the producer could refill stage s (it
@@ -470,6 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // also means that region r is free.
             if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u)) {
                 timed_out = 1;
+                stop = true;
                 break;
             }
             tc_fence_after();
@@ -504,20 +554,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int half = (warp - 6) >> 2;        // columns [half * BN/2, +BN/2)
         constexpr int HC = BN / 2;               // columns per epilogue warp
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
-        float alpha = p.alpha;
-        if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
-        if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
         uint32_t local = 0;
         for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
             if (*(volatile int*)&timed_out) break;  // a stage failed: no further tiles arrive
-            const int64_t m0 = (tile / tiles_n) * kBM, n0 = (tile % tiles_n) * BN;
+            const TileJob jb = tile_job<BN>(p, tile, tiles_n, tiles_per_group);
+            float alpha = p.alpha;
+            const int gs = jb.group < 0 ? 0 : jb.group;
+            if (p.scale_a) alpha = __fmul_rn(alpha, p.scale_a[gs]);
+            if (p.scale_b) alpha = __fmul_rn(alpha, p.scale_b[gs]);
             const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u);
             tc_fence_after();
             __syncwarp();
             if (!acc_ok) timed_out = 1;
             const bool bad = *(volatile int*)&timed_out != 0;
-            epilogue_tile<BN>(lane_base, m0 + 32 * q, n0 + half * HC, p, alpha, bad,
-                              smem_addr(&S.acc_empty), 0u, smem_addr(S.dstage[warp - 6]), &tmD);
+            const int64_t m_in = (jb.d_row - (jb.group >= 0 && p.group_mode == 2 ? (int64_t)jb.group * p.M : 0)) + 32 * q;
+            epilogue_tile<BN>(lane_base, jb.d_row + 32 * q, jb.n0 + half * HC, p, alpha,
+                              !bad && m_in < p.M, jb.k_len == 0, smem_addr(&S.acc_empty), 0u,
+                              smem_addr(S.dstage[warp - 6]), &tmD);
         }
         if (lane == 0) bulk_wait_all();  // every store of this warp has landed
         __syncwarp();
@@ -885,8 +938,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             __syncwarp();
             if (!acc_ok) timed_out = 1;
             const bool bad = *(volatile int*)&timed_out != 0;
-            epilogue_tile<BN>(lane_base, m0 + 128 * rank + 32 * q, n0 + half * HC, p, alpha, bad,
-                              acc_empty_l, leader ? 0u : 1u, smem_addr(S.dstage[warp - 6]), &tmD);
+            epilogue_tile<BN>(lane_base, m0 + 128 * rank + 32 * q, n0 + half * HC, p, alpha,
+                              !bad && m0 + 128 * rank + 32 * q < p.M, false, acc_empty_l, leader ? 0u : 1u,
+                              smem_addr(S.dstage[warp - 6]), &tmD);
         }
         if (lane == 0) bulk_wait_all();
         __syncwarp();
@@ -948,10 +1002,13 @@ static bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) 
 template <int BN, int STAGES>
 static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream_t st) {
     CUtensorMap ma, mb, md;
-    if (!make_operand_map(&ma, p.A, p.M, p.K / 2, kBM) || !make_operand_map(&mb, p.B, p.N, p.K / 2, BN))
+    const int64_t b_rows = p.group_mode == 1 && p.b_group_rows ? p.b_group_rows * p.num_groups : p.N;
+    const int64_t kb = p.Kb ? p.Kb : p.K;
+    if (!make_operand_map(&ma, p.A, p.M, p.K / 2, kBM) || !make_operand_map(&mb, p.B, b_rows, kb / 2, BN))
         return cudaErrorInvalidValue;
     memset(&md, 0, sizeof(md));
-    if (p.D_bf16 && !make_output_map(&md, p.D_bf16, p.M, p.N)) return cudaErrorInvalidValue;
+    const int64_t d_rows = p.group_mode == 2 ? p.M * p.num_groups : p.M;
+    if (p.D_bf16 && !make_output_map(&md, p.D_bf16, d_rows, p.N)) return cudaErrorInvalidValue;
     const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
     static bool configured = false;
     if (!configured) {
@@ -960,7 +1017,8 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
+    int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
+    if (p.group_mode == 2) tiles *= p.num_groups;
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
     gemm_nvf4_kernel<BN, STAGES><<<grid, kGemmThreads, smem, st>>>(ma, mb, md, p);
     return cudaGetLastError();
@@ -1007,7 +1065,7 @@ static cudaError_t launch_gemm_pair(const GemmParams& p, int sm_count, cudaStrea
 }
 
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
-    if (p.M > 128 && sm_count >= 2) return launch_gemm_pair<5>(p, sm_count, st);
+    if (p.group_mode == 0 && p.M > 128 && sm_count >= 2) return launch_gemm_pair<5>(p, sm_count, st);
     return launch_gemm_cfg<256, 4>(p, sm_count, st);
 }
 

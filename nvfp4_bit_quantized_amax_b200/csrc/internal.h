@@ -22,7 +22,18 @@ struct QuantParams {
     int row_sr, col_sr, col_rht;
     uint32_t sign_mask;  // bit i set: rotation sign i is -1
     uint32_t rk[20];     // Philox4x32-10 round keys of `seed` (filled by the launchers)
+    // Grouped tensors (mixture of experts): row r belongs to group
+    // row_group[r / 128] (table) or r / group_rows_uniform; group g owns rows
+    // [row0_g, row0_g + rows_g) and has its own amax words (amax_words + 2g), tensor
+    // scales (row_g[g], col_g[g]), Philox key seed + g, and element indices counted
+    // inside its rows.  Groups are whole 128-row blocks.
+    const int32_t* row_group;
+    const int64_t* group_row0;
+    const int64_t* group_nrows;
+    int64_t group_rows_uniform;
 };
+
+cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t st);
 
 // Philox4x32-10 key schedule of a 64-bit seed: round r uses
 // (lo(seed) + r * 0x9E3779B9, hi(seed) + r * 0xBB67AE85), mod 2^32.
@@ -61,6 +72,22 @@ struct GemmParams {
     void* D_bf16;
     float* D_f32;
     int* status;
+    // Grouped problems (mixture of experts), one launch for all groups:
+    //  group_mode 1: A rows are grouped in 128-row tiles (mtile_group[m / 128] is the
+    //    group of A row m); a tile of group g reads B rows g * b_group_rows + n.
+    //  group_mode 2: group g reduces over k in [k_start[g], k_start[g] + k_len[g]) of
+    //    A and B (both multiples of 128) and writes D rows g * M + m.
+    //  scale_a / scale_b then hold one tensor scale per group; no fp32 output.
+    //  In mode 1 a tile of group g also starts its reduction over B at column
+    //  g * b_group_k, and B's rows are Kb wide (0: K).
+    int group_mode;
+    const int32_t* mtile_group;
+    int64_t b_group_rows;
+    int64_t b_group_k;
+    int64_t Kb;
+    const int64_t* k_start;
+    const int64_t* k_len;
+    int num_groups;
 };
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st);
 

@@ -47,10 +47,14 @@ __device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t f
 // bf16 magnitude; NaN patterns sort above Inf), word 1 max |RHT16 down the
 // rows| (column orientation), as fp32 bits.  Both are combined with atomicMax.
 // ============================================================================
-template <bool kColRht>
+// Grouped (kGrouped): the rows of a unit lie in one group, whose words are
+// words[2g] and words[2g+1]; each unit is folded into them by the warp.
+template <bool kColRht, bool kGrouped>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, uint32_t sign_mask,
-                                                   uint32_t* __restrict__ words) {
+                                                   uint32_t* __restrict__ words,
+                                                   const int32_t* __restrict__ row_group,
+                                                   int64_t group_rows_uniform) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t col_units = (cols + 255) >> 8;
     const int64_t units = ((rows + 15) >> 4) * col_units;
@@ -59,7 +63,11 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += (int64_t)gridDim.x * 8) {
         const int64_t r0 = (u / col_units) * 16;
         const int64_t c0 = (u % col_units) * 256 + lane * 8;
-        if (c0 >= cols) continue;
+        if (kGrouped) {
+            m_row = 0;
+            m_col = 0.0;
+        }
+        if (c0 < cols) {
         uint4 v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -87,7 +95,20 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
                 for (int i = 0; i < 16; ++i) m_col = fmax(m_col, fabs(y[i]));
             }
         }
+        }
+        if (kGrouped) {
+            const int64_t g = row_group ? (int64_t)row_group[r0 >> 7] : r0 / group_rows_uniform;
+            uint32_t ur = max(m_row & 0xFFFFu, m_row >> 16) << 16;
+            uint32_t uc = kColRht ? __float_as_uint(__double2float_rn(m_col)) : 0u;
+            ur = __reduce_max_sync(0xFFFFFFFFu, ur);
+            uc = __reduce_max_sync(0xFFFFFFFFu, uc);
+            if (lane == 0) {
+                if (ur) atomicMax(words + 2 * g, ur);
+                if (kColRht && uc) atomicMax(words + 2 * g + 1, uc);
+            }
+        }
     }
+    if (kGrouped) return;
     uint32_t a_row = max(m_row & 0xFFFFu, m_row >> 16) << 16;
     uint32_t a_col = kColRht ? __float_as_uint(__double2float_rn(m_col)) : 0u;
     a_row = __reduce_max_sync(0xFFFFFFFFu, a_row);
@@ -214,17 +235,53 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 // ============================================================================
 constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;
 
-template <bool k2D, bool kRht>
+// Grouped (kGrouped): the tile's rows lie in one group g (see QuantParams), which
+// supplies the tensor scales, the Philox key seed + g and the origin of the
+// element indices.
+template <bool k2D, bool kRht, bool kGrouped>
 __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
     __shared__ __align__(16) uint16_t tile[kTR][kPitch];
     __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
     __shared__ float tile_inv[kTR / 16][kTC / 16];
 
-    TensorScale tr, tc;
-    if (!load_tensor_scales(p, tr, tc)) return;
-
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = (int64_t)blockIdx.y * kTR, c0 = (int64_t)blockIdx.x * kTC;
+    TensorScale tr, tc;
+    int64_t g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
+    uint32_t rkg[20];                     // the group's Philox round keys
+    if (kGrouped) {
+        const int64_t g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
+        g_row0 = p.row_group ? p.group_row0[g] : g * p.group_rows_uniform;
+        g_rows = p.row_group ? p.group_nrows[g] : p.group_rows_uniform;
+        const uint32_t wr = p.amax_words[2 * g];
+        const uint32_t wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
+        const bool first = r0 == g_row0 && c0 == 0 && tid == 0;
+        if (!finite_bits(wr) || !finite_bits(wc)) {
+            if (first) {
+                set_status(p.status, kStatusNonFinite);
+                if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
+                if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
+            }
+            return;
+        }
+        tr = tensor_scale_from_amax(__uint_as_float(wr));
+        tc = tensor_scale_from_amax(__uint_as_float(wc));
+        if (first) {
+            if (p.row_g) p.row_g[g] = tr.g;
+            if (p.col_g) p.col_g[g] = tc.g;
+        }
+        uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
+#pragma unroll
+        for (int r = 0; r < 10; ++r) {
+            rkg[2 * r] = k0;
+            rkg[2 * r + 1] = k1;
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+    } else {
+        if (!load_tensor_scales(p, tr, tc)) return;
+    }
+    const uint32_t (&rk)[20] = kGrouped ? rkg : p.rk;
     const bool want_row = p.row_data != nullptr;
     const bool want_col = p.col_data != nullptr;
     const bool use_smem = want_col || k2D;
@@ -283,15 +340,15 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
                 block_scale(amax, tc, s, inv);
             }
             if (want_col) {
-                const uint64_t e0 = (uint64_t)c * (uint64_t)p.rows + (uint64_t)(r0 + 16 * j);
+                const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
                 float lo8[8], hi8[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     lo8[i] = y[i];
                     hi8[i] = y[8 + i];
                 }
-                out[2 * jj] = encode8(lo8, inv, p.col_sr, p.rk, 1u, e0);
-                out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, p.rk, 1u, e0 + 8);
+                out[2 * jj] = encode8(lo8, inv, p.col_sr, rk, 1u, e0);
+                out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, rk, 1u, e0 + 8);
                 if (c < p.cols && r0 + 16 * j < p.rows)
                     p.col_sf[sf_offset(c, (r0 >> 4) + j, katoms_c)] = (uint8_t)s;
             }
@@ -327,7 +384,7 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
             float v[8];
             unpack8(reg[k], v);
             const uint32_t codes =
-                encode8(v, inv, p.row_sr, p.rk, 0u, (uint64_t)r * (uint64_t)p.cols + (uint64_t)c);
+                encode8(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
             if (r < p.rows && c < p.cols) {
                 *reinterpret_cast<uint32_t*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
                 if ((lc & 15) == 0) p.row_sf[sf_offset(r, c >> 4, katoms_r)] = (uint8_t)s;
@@ -426,9 +483,22 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
     const int64_t units = ((rows + 15) / 16) * ((cols + 255) / 256);
     const int grid = grid_for(units, 8, sm_count, 8);
     if (col_rht)
-        amax_kernel<true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words);
+        amax_kernel<true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
     else
-        amax_kernel<false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words);
+        amax_kernel<false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t st) {
+    const int64_t units = ((p.rows + 15) >> 4) * ((p.cols + 255) >> 8);
+    const int grid = grid_for(units, 8, sm_count, 8);
+    uint32_t* words = const_cast<uint32_t*>(p.amax_words);
+    if (p.col_rht)
+        amax_kernel<true, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
+                                                     p.group_rows_uniform);
+    else
+        amax_kernel<false, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
+                                                      p.group_rows_uniform);
     return cudaGetLastError();
 }
 
@@ -445,12 +515,20 @@ cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, cudaStream_
     QuantParams p = params;
     philox_round_keys(p.seed, p.rk);
     const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
-    if (two_d)
-        quant_tile_kernel<true, false><<<grid, 256, 0, st>>>(p);
+    const bool grouped = p.row_group != nullptr || p.group_rows_uniform > 0;
+    if (grouped) {
+        if (two_d)
+            quant_tile_kernel<true, false, true><<<grid, 256, 0, st>>>(p);
+        else if (p.col_rht && p.col_data)
+            quant_tile_kernel<false, true, true><<<grid, 256, 0, st>>>(p);
+        else
+            quant_tile_kernel<false, false, true><<<grid, 256, 0, st>>>(p);
+    } else if (two_d)
+        quant_tile_kernel<true, false, false><<<grid, 256, 0, st>>>(p);
     else if (p.col_rht && p.col_data)
-        quant_tile_kernel<false, true><<<grid, 256, 0, st>>>(p);
+        quant_tile_kernel<false, true, false><<<grid, 256, 0, st>>>(p);
     else
-        quant_tile_kernel<false, false><<<grid, 256, 0, st>>>(p);
+        quant_tile_kernel<false, false, false><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
