@@ -211,8 +211,8 @@ int nvfp4_moe_linear_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K
  * the permuted tensors are quantized whole, in both orientations, with per-expert
  * tensor scales, and one persistent GEMM walks the tiles of all experts.  (The
  * explainer's "The model underneath": most of the FP4 FLOPs are expert GEMMs.)
- *   group_rows: HOST array of E entries, each a multiple of 128 (0 allowed), their
- *   sum R >= 128; K, N multiples of 128.  X_perm [R][K], Y_perm / dY_perm [R][N],
+ *   group_rows: HOST array of E <= 1024 entries, each a multiple of 128 (0 allowed),
+ *   their sum R >= 128; K, N multiples of 128.  X_perm [R][K], Y_perm / dY_perm [R][N],
  *   dX_perm [R][K] bf16 in expert order; W, dW [E][N][K] bf16.
  *   ws: nvfp4_moe_grouped_workspace_bytes() bytes, 256-byte aligned; its status word
  *   is read with nvfp4_read_status.  fprop fills the X and W operands, dgrad the dY

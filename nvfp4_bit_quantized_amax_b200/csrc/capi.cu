@@ -7,8 +7,6 @@
 #include <stdint.h>
 #include <string.h>
 
-#include <vector>
-
 #include "../../include/nvfp4.h"
 #include "internal.h"
 
@@ -581,7 +579,7 @@ MoeLayout moe_layout(const int64_t* group_rows, int E, int64_t K, int64_t N) {
 }
 
 int moe_grouped_check(const int64_t* group_rows, int E, int64_t K, int64_t N) {
-    if (!group_rows || E < 1) return NVFP4_ERR_ARG;
+    if (!group_rows || E < 1 || E > kMaxGroups) return NVFP4_ERR_ARG;
     if (K < 128 || N < 128 || K % 128 || N % 128) return NVFP4_ERR_SHAPE;
     int64_t R = 0;
     for (int e = 0; e < E; ++e) {
@@ -603,19 +601,10 @@ int moe_grouped_begin(const int64_t* group_rows, int E, int64_t K, int64_t N, vo
     if (!aligned(ws, 256)) return NVFP4_ERR_ALIGN;
     if (ws_bytes < (size_t)L->total) return NVFP4_ERR_WORKSPACE;
     if ((rc = device_check(sms))) return rc;
-    std::vector<int32_t> mt((size_t)(L->R / 128));
-    std::vector<int64_t> r0((size_t)E), nr((size_t)E);
-    int64_t row = 0;
-    for (int e = 0; e < E; ++e) {
-        r0[e] = row;
-        nr[e] = group_rows[e];
-        for (int64_t b = row / 128; b < (row + group_rows[e]) / 128; ++b) mt[(size_t)b] = e;
-        row += group_rows[e];
-    }
     uint8_t* b = static_cast<uint8_t*>(ws);
-    if (cudaMemcpyAsync(b + L->mtile_group, mt.data(), mt.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(b + L->group_row0, r0.data(), r0.size() * 8, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(b + L->group_nrows, nr.data(), nr.size() * 8, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    if (launch_group_tables(group_rows, E, reinterpret_cast<int32_t*>(b + L->mtile_group),
+                            reinterpret_cast<int64_t*>(b + L->group_row0),
+                            reinterpret_cast<int64_t*>(b + L->group_nrows), st) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }

@@ -35,6 +35,13 @@ struct QuantParams {
 
 cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t st);
 
+// Group tables of a grouped tensor from its group sizes (host array of E <=
+// kMaxGroups entries, multiples of 128): group of every 128-row block, first row
+// and rows of every group, written on `st`.
+constexpr int kMaxGroups = 1024;
+cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block_group, int64_t* row0,
+                                int64_t* nrows, cudaStream_t st);
+
 // Philox4x32-10 key schedule of a 64-bit seed: round r uses
 // (lo(seed) + r * 0x9E3779B9, hi(seed) + r * 0xBB67AE85), mod 2^32.
 inline void philox_round_keys(uint64_t seed, uint32_t (&rk)[20]) {

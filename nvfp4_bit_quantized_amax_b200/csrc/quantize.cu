@@ -10,6 +10,8 @@
 // ("NVIDIA's 4-bit floating point pushes AI training limits", artiverse.ca).
 #include <cuda_bf16.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -499,6 +501,59 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
     else
         amax_kernel<false, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
                                                       p.group_rows_uniform);
+    return cudaGetLastError();
+}
+
+// ============================================================================
+// Group tables of a grouped tensor, built on the device from the group sizes
+// (carried in the kernel's parameters): the group of every 128-row block, and
+// each group's first row and row count.
+// ============================================================================
+struct GroupSizes {
+    int64_t rows[kMaxGroups];
+};
+__global__ void group_tables_kernel(GroupSizes gs, int E, int32_t* __restrict__ block_group,
+                                    int64_t* __restrict__ row0, int64_t* __restrict__ nrows) {
+    __shared__ int64_t start[kMaxGroups + 1];
+    if (threadIdx.x == 0) {
+        int64_t r = 0;
+        for (int e = 0; e < E; ++e) {
+            start[e] = r;
+            r += gs.rows[e];
+        }
+        start[E] = r;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        row0[e] = start[e];
+        nrows[e] = gs.rows[e];
+    }
+    const int64_t blocks = start[E] / 128;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < blocks;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        int lo = 0, hi = E - 1;  // last group whose start is <= the block's first row
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (start[mid] <= b * 128) lo = mid; else hi = mid - 1;
+        }
+        while (lo < E - 1 && start[lo + 1] <= b * 128) ++lo;
+        block_group[b] = lo;
+    }
+}
+
+cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block_group, int64_t* row0,
+                                int64_t* nrows, cudaStream_t st) {
+    if (E < 1 || E > kMaxGroups) return cudaErrorInvalidValue;
+    GroupSizes gs;
+    memset(&gs, 0, sizeof gs);
+    int64_t total = 0;
+    for (int e = 0; e < E; ++e) {
+        gs.rows[e] = group_rows[e];
+        total += group_rows[e];
+    }
+    const int64_t blocks = total / 128;
+    const int grid = (int)((blocks + 255) / 256 < 64 ? (blocks + 255) / 256 : 64);
+    group_tables_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(gs, E, block_group, row0, nrows);
     return cudaGetLastError();
 }
 
