@@ -34,6 +34,11 @@ FLOPS_PER_GEMM = 2.0 * M * K * N
 FLOPS_PER_STEP = 3 * FLOPS_PER_GEMM
 KERNELS_PER_STEP = 9  # 2 amax + 2 quantize (fprop), 1 + 1 (dgrad), 3 GEMMs
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
+# DRAM bytes (read + write) of one fprop GEMM launch at this workload, from one ncu
+# capture (profiles/gemm_nvf4_pair_fprop_8192x20480x5120_traffic.md); reported only
+# while the GEMM source is the one that was captured.
+GEMM_TRAFFIC = {"gemm_cu_sha256_16": "dd3efb8a564996a2", "bytes": 382145024 + 311861504,
+                "launch": "fprop M=8192 N=20480 K=5120"}
 
 
 def env_rank():
@@ -276,10 +281,17 @@ def run_ours(args, rank, world, local_rank):
                  for k, v in q_ms.items()}
         q_total_bytes = sum(q_bytes_per_el * v[1] for v in q_ms.values())
         q_total_ms = sum(v[0] for v in q_ms.values())
+        traffic = args.traffic
+        if traffic is None:
+            import hashlib
+            with open(os.path.join(ROOT, "nvfp4_bit_quantized_amax_b200", "csrc", "gemm.cu"), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest()[:16] == GEMM_TRAFFIC["gemm_cu_sha256_16"]:
+                    traffic = GEMM_TRAFFIC["bytes"]
         out["roofline"] = {
-            "bound": "tensor", "kernel": "gemm_nvf4_kernel (fprop/dgrad/wgrad average)",
+            "bound": "tensor", "kernel": "gemm_nvf4_pair_kernel (fprop/dgrad/wgrad average)",
             "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-            "frac": round(achieved / fp4_peak, 4), "traffic": args.traffic,
+            "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
+            "traffic_launch": GEMM_TRAFFIC["launch"] if traffic is not None else None,
             "peak_source": f"{peak_kind}: FP4 = {FP4_OVER_BF16:g} x bf16 burst "
                            f"{peaks['bf16_tflops']} TFLOP/s (nominal 9 / 2.25 PFLOP/s ratio)",
         }
@@ -462,7 +474,8 @@ def run_reference(args, rank, world):
 def run_kernel(args):
     """Single-kernel mode for profilers: quantize synthetic bf16 inputs of the given
     shape, then launch one kernel `--steps` times.  --kernel gemm (M,N,K),
-    quant-x / quant-w / quant-dy (rows,cols): the three fused quantize passes."""
+    quant-x / quant-w / quant-dy (rows,cols): the three fused quantize passes;
+    moe-step: the grouped MoE expert-layer step (no shape)."""
     import torch
 
     from nvfp4_bit_quantized_amax_b200 import capi
@@ -484,7 +497,30 @@ def run_kernel(args):
         capi.nvfp4_quantize(x, 0, 0, 0, *op, ws)
         return op
 
-    if args.kernel == "gemm":
+    if args.kernel == "moe-step":
+        s_ = syn.MOE
+        E, K_, N_, T_, k_ = s_["experts"], s_["hidden"], s_["ffn"], s_["tokens"], s_["topk"]
+        d = syn.moe_inputs(T_, E, K_, N_, k_, s_["zipf_s"], seed=0, pad=128)
+        rows = int(d["group_rows"].sum())
+        x_tok, dY = to_dev(d["X"]), to_dev(d["dY"])
+        Wm = to_dev(d["W"].reshape(E * N_, K_)).view(E, N_, K_)
+        row_src = torch.from_numpy(d["row_src"]).to(dev)
+        slots = torch.from_numpy(d["slots"]).to(dev)
+        X_perm = torch.empty((rows, K_), dtype=torch.bfloat16, device=dev)
+        Y = torch.empty((rows, N_), dtype=torch.bfloat16, device=dev)
+        dX = torch.empty((rows, K_), dtype=torch.bfloat16, device=dev)
+        dX_tok = torch.empty((T_, K_), dtype=torch.bfloat16, device=dev)
+        dW = torch.empty((E, N_, K_), dtype=torch.bfloat16, device=dev)
+        gws = torch.empty(capi.moe_grouped_workspace_bytes(d["group_rows"], K_, N_), dtype=torch.uint8,
+                          device=dev)
+
+        def fn():
+            capi.nvfp4_moe_gather(x_tok, row_src, X_perm)
+            capi.nvfp4_moe_grouped_fprop(X_perm, Wm, Y, d["group_rows"], signs, gws)
+            capi.nvfp4_moe_grouped_dgrad(dY, dX, d["group_rows"], 7, signs, gws)
+            capi.nvfp4_moe_combine(dX, slots, dX_tok)
+            capi.nvfp4_moe_grouped_wgrad(dW, d["group_rows"], gws)
+    elif args.kernel == "gemm":
         Mk, Nk, Kk = dims
         a, b = operand(Mk, Kk, 1), operand(Nk, Kk, 2)
         D = torch.empty((Mk, Nk), dtype=torch.bfloat16, device=dev)
@@ -511,7 +547,7 @@ def run_kernel(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", default=None, choices=["gemm", "quant-x", "quant-w", "quant-dy"],
+    ap.add_argument("--kernel", default=None, choices=["gemm", "quant-x", "quant-w", "quant-dy", "moe-step"],
                     help="profiler mode: launch one kernel kind only")
     ap.add_argument("--shape", default="4096,8192,5120")
     ap.add_argument("--gpus", type=int, default=1)
