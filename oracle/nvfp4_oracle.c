@@ -30,6 +30,10 @@
  *      p = (|v| - lo) / (hi - lo); round up iff r < p * 2^16, with r the element's
  *      16-bit Philox draw (see ora_sr_draw16).
  *  R9  amax == 0 gives g = 0, enc = 0, all scales 0 and all codes +-0.
+ *  R14 RHT on both backward GEMMs ([LTD] "Main findings", the Mosaic recipe): the
+ *      dgrad operands dY and W^T are rotated along N, their shared reduction axis,
+ *      i.e. along the rows of the quantized view (orient 0 with rht); the dgrad
+ *      alpha takes the 1/16.
  */
 #include "nvfp4_oracle.h"
 
@@ -256,9 +260,20 @@ int ora_rht(const uint16_t* x, int64_t rows, int64_t cols, int axis,
  * falls outside the exact domain of ora_rht16.                                */
 static int ora_v_row(const uint16_t* x, int64_t rows, int64_t cols, int orient, int rht,
                      const int8_t signs[16], int64_t vr, float* out) {
-    if (orient == 0) {
+    if (orient == 0 && !rht) {
         for (int64_t c = 0; c < cols; ++c) out[c] = ora_bf16_to_f32(x[vr * cols + c]);
         return 0;
+    }
+    if (orient == 0) {
+        /* R14: the rotation along the row (dgrad operands rotated along N) */
+        int bad = 0;
+        for (int64_t j = 0; j < cols / 16; ++j) {
+            double in[16], y[16];
+            for (int i = 0; i < 16; ++i) in[i] = ora_bf16_to_f32(x[vr * cols + 16 * j + i]);
+            if (ora_rht16(in, signs, y) != 0) bad = 1;
+            for (int t = 0; t < 16; ++t) out[16 * j + t] = (float)y[t];
+        }
+        return bad ? -1 : 0;
     }
     /* orient 1: V row vr is column vr of x, blocks along the rows of x */
     if (!rht) {
@@ -277,11 +292,11 @@ static int ora_v_row(const uint16_t* x, int64_t rows, int64_t cols, int orient, 
 
 int ora_tensor_amax(const uint16_t* x, int64_t rows, int64_t cols, int orient, int rht,
                     const int8_t signs[16], float* amax, int nthreads) {
-    if (orient == 1 && rht && rows % 16 != 0) return -2;
+    if (rht && (orient ? rows : cols) % 16 != 0) return -2;
     int64_t vrows = orient ? cols : rows, vcols = orient ? rows : cols;
     float m = 0.0f;
     int bad = 0;
-    if (!(orient == 1 && rht)) {
+    if (!rht) {
         /* the same set of elements either way */
 #pragma omp parallel for num_threads(ora_threads(nthreads)) reduction(max : m)
         for (int64_t i = 0; i < rows * cols; ++i) {

@@ -67,6 +67,7 @@ int  ora_rht(const uint16_t* x, int64_t rows, int64_t cols, int axis,
  *   orient 0: V = x                      ([rows][cols], blocks along cols)
  *   orient 1: V = x^T                    ([cols][rows], blocks along rows of x)
  *   orient 1 with rht: V[c][16j+t] = RHT16(x[16j..16j+15][c], signs)[t]
+ *   orient 0 with rht: V[r][16j+t] = RHT16(x[r][16j..16j+15], signs)[t]    (R14)
  * amax of V as fp32 (max |V|).  Returns 0, or -1 if the RHT domain check fails. */
 int   ora_tensor_amax(const uint16_t* x, int64_t rows, int64_t cols, int orient,
                       int rht, const int8_t signs[16], float* amax, int nthreads);

@@ -251,3 +251,40 @@ def test_gemm_matches_numpy_and_pairs(ora, tables):
     ni = rng.integers(0, N, 50)
     out, bnd = ora.gemm_pairs(A, sa, B, sb, alpha, mi, ni)
     assert np.array_equal(out, D[mi, ni]) and np.array_equal(bnd, bound[mi, ni])
+
+
+# ---- R14: RHT along the row of the quantized view (dgrad operands rotated along N) ----
+def test_row_rht_equals_column_rht_of_transpose(ora):
+    """The rotation along a view row is the same whether the view is x (orient 0) or
+    the transpose of x^T (orient 1, pinned above): same amax, codes and scales (RNE;
+    SR draws differ by stream)."""
+    x = syn.normal_bf16((48, 64), 21, outlier_prob=0.02)
+    s = syn.rht_signs(3)
+    xt = np.ascontiguousarray(x.T)
+    for bm in (0, 1):
+        p0, sf0, g0, a0 = ora.quantize(x, 0, True, s, bm, 0)
+        p1, sf1, g1, a1 = ora.quantize(xt, 1, True, s, bm, 0)
+        assert a0 == a1 and g0 == g1
+        assert np.array_equal(p0, p1) and np.array_equal(sf0, sf1)
+
+
+def test_row_rht_amax_is_max_of_standalone_rht(ora):
+    x = syn.normal_bf16((32, 96), 22)
+    s = syn.rht_signs(4)
+    y = ora.rht(x, 1, s)                  # 16-chunks along the contiguous columns
+    _, _, _, amax = ora.quantize(x, 0, True, s, 0, 0)
+    assert amax == np.float32(np.abs(y).max())
+
+
+def test_dgrad_rotation_identity_fp64():
+    """(dY D H)(W^T D H)^T = 16 dY W on unquantized data: the rotation along N cancels
+    in dgrad with alpha 1/16."""
+    rng = np.random.default_rng(7)
+    M, N, K = 8, 32, 12
+    dY = rng.standard_normal((M, N))
+    W = rng.standard_normal((N, K))
+    s = syn.rht_signs(6).astype(np.float64)
+    H = np.array([[(-1.0) ** bin(i & j).count("1") for j in range(16)] for i in range(16)])
+    R = np.kron(np.eye(N // 16), np.diag(s) @ H)      # block-diagonal rotation along N
+    lhs = (dY @ R) @ (W.T @ R).T / 16.0
+    assert np.allclose(lhs, dY @ W, rtol=1e-12, atol=1e-12)
