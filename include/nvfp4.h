@@ -244,6 +244,32 @@ int nvfp4_moe_gather(const void* src, const int32_t* row_src, int64_t rows, int6
 int nvfp4_moe_combine(const void* src, const int32_t* slots, int64_t tokens, int topk,
                       int64_t cols, void* dst, nvfp4_stream_t stream);
 
+/*
+ * Recipe options of the linear layer (NULL = the defaults above).
+ *   weight_block_mode  NVFP4_BLOCK_16X16 (default): one quantization of W shared by
+ *                      fprop and dgrad; NVFP4_BLOCK_1X16: the 1D-weight recipe, W
+ *                      quantized 1x16 along K for fprop and, separately, 1x16 along N
+ *                      for dgrad (the 1D-versus-2D weight comparison of "Paper of the
+ *                      day: What matters for NVFP4 training?", "The problem").
+ *   dgrad_rht          1: rotate both dgrad operands (dY and W^T) along N with the same
+ *                      16-point RHT, dgrad alpha 1/16 (RHT on both backward GEMMs, the
+ *                      Mosaic recipe of "Paper of the day: What matters for NVFP4
+ *                      training?", "Main findings"); needs weight_block_mode 1X16.
+ * The options change fprop's quantization of W and dgrad's of dY; pass the same
+ * options to both calls on one workspace (wgrad is unaffected).  Invalid options:
+ * NVFP4_ERR_ARG.
+ */
+typedef struct {
+    int weight_block_mode;
+    int dgrad_rht;
+} nvfp4_linear_opts;
+int nvfp4_linear_fprop_ex(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
+                          const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
+                          size_t ws_bytes, nvfp4_stream_t stream);
+int nvfp4_linear_dgrad_ex(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                          const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
+                          size_t ws_bytes, nvfp4_stream_t stream);
+
 /* Views of the quantized operands a linear workspace holds (no device access). */
 enum {
     NVFP4_LIN_X_ROW = 0,  /* X,   M x K, 1x16 RNE                 */

@@ -29,6 +29,7 @@ EXPORTS = (
     "nvfp4_status_string", "nvfp4_version", "nvfp4_quantize_noalloc",
     "nvfp4_moe_workspace_bytes", "nvfp4_moe_expert_workspace", "nvfp4_moe_linear_fprop",
     "nvfp4_moe_linear_dgrad", "nvfp4_moe_linear_wgrad", "nvfp4_moe_gather", "nvfp4_moe_combine",
+    "nvfp4_linear_fprop_ex", "nvfp4_linear_dgrad_ex",
     "nvfp4_moe_grouped_workspace_bytes", "nvfp4_moe_grouped_operand", "nvfp4_moe_grouped_fprop",
     "nvfp4_moe_grouped_dgrad", "nvfp4_moe_grouped_wgrad",
 )
@@ -44,6 +45,11 @@ class Tensor(C.Structure):
     """nvfp4_tensor: one quantized operand (device pointers)."""
     _fields_ = [("data", C.c_void_p), ("scales", C.c_void_p), ("tensor_scale", C.c_void_p),
                 ("rows", C.c_int64), ("cols", C.c_int64)]
+
+
+class LinearOpts(C.Structure):
+    """nvfp4_linear_opts: weight block mode, RHT on the dgrad operands."""
+    _fields_ = [("weight_block_mode", C.c_int), ("dgrad_rht", C.c_int)]
 
 
 class QuantizeOpts(C.Structure):
@@ -90,6 +96,8 @@ def load(path: str = LIB_PATH):
         "nvfp4_moe_linear_wgrad": (ci, [vp, vp, ci, i64, i64, u64, vp, vp, sz, vp]),
         "nvfp4_moe_gather": (ci, [vp, vp, i64, i64, vp, vp]),
         "nvfp4_moe_combine": (ci, [vp, vp, i64, ci, i64, vp, vp]),
+        "nvfp4_linear_fprop_ex": (ci, [vp, vp, vp, i64, i64, i64, vp, C.POINTER(LinearOpts), vp, sz, vp]),
+        "nvfp4_linear_dgrad_ex": (ci, [vp, vp, i64, i64, i64, u64, vp, C.POINTER(LinearOpts), vp, sz, vp]),
         "nvfp4_moe_grouped_workspace_bytes": (sz, [vp, ci, i64, i64]),
         "nvfp4_moe_grouped_operand": (ci, [vp, vp, ci, i64, i64, ci, C.POINTER(Tensor)]),
         "nvfp4_moe_grouped_fprop": (ci, [vp, vp, vp, vp, ci, i64, i64, vp, vp, sz, vp]),
@@ -228,6 +236,28 @@ def nvfp4_linear_wgrad(dY, dW, M, seed, rht_signs, ws, stream=None):
     _check("nvfp4_linear_wgrad", load().nvfp4_linear_wgrad(
         _ptr(dY), _ptr(dW), M, K, N, seed, sp, _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+    del keep
+
+
+def nvfp4_linear_fprop_ex(X, W, Y, rht_signs, ws, weight_block_mode=1, dgrad_rht=0, stream=None):
+    M, K = X.shape
+    N = W.shape[0]
+    keep, sp = _signs(rht_signs)
+    o = LinearOpts(weight_block_mode, dgrad_rht)
+    _check("nvfp4_linear_fprop_ex", load().nvfp4_linear_fprop_ex(
+        _ptr(X), _ptr(W), _ptr(Y), M, K, N, sp, C.byref(o), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def nvfp4_linear_dgrad_ex(dY, dX, seed, rht_signs, ws, weight_block_mode=1, dgrad_rht=0, stream=None):
+    M, N = dY.shape
+    K = dX.shape[1]
+    keep, sp = _signs(rht_signs)
+    o = LinearOpts(weight_block_mode, dgrad_rht)
+    _check("nvfp4_linear_dgrad_ex", load().nvfp4_linear_dgrad_ex(
+        _ptr(dY), _ptr(dX), M, K, N, seed, sp, C.byref(o), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
     del keep
 
 

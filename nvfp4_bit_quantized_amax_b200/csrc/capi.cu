@@ -94,9 +94,9 @@ LinLayout lin_layout(int64_t M, int64_t K, int64_t N) {
 int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_sr, int col_sr,
                  uint64_t seed, int col_rht, uint32_t mask, uint8_t* rd, uint8_t* rsf, float* rg,
                  uint8_t* cd, uint8_t* csf, float* cg, uint32_t* words, int* status, int sms,
-                 cudaStream_t st, bool rows_only_kernel) {
+                 cudaStream_t st, bool rows_only_kernel, int row_rht = 0) {
     cudaError_t e = launch_amax(static_cast<const uint16_t*>(x), rows, cols, col_rht && cd, mask,
-                                words, sms, st);
+                                words, sms, st, row_rht != 0);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     QuantParams p;
     memset(&p, 0, sizeof p);
@@ -115,8 +115,9 @@ int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_
     p.row_sr = row_sr;
     p.col_sr = col_sr;
     p.col_rht = (col_rht && cd) ? 1 : 0;
+    p.row_rht = row_rht;
     p.sign_mask = mask;
-    e = rows_only_kernel ? launch_quant_rows(p, sms, st) : launch_quant_tile(p, two_d, st);
+    e = rows_only_kernel && !row_rht ? launch_quant_rows(p, sms, st) : launch_quant_tile(p, two_d, st);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     if (rsf && (e = launch_sf_pad(rsf, rows, cols / 16, sms, st)) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (csf && (e = launch_sf_pad(csf, cols, rows / 16, sms, st)) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -343,13 +344,26 @@ static int lin_check(int64_t M, int64_t K, int64_t N, void* ws, size_t ws_bytes)
     return NVFP4_OK;
 }
 
-int nvfp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
-                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+static int opts_check(const nvfp4_linear_opts* o) {
+    if (!o) return NVFP4_OK;
+    if (o->weight_block_mode != NVFP4_BLOCK_16X16 && o->weight_block_mode != NVFP4_BLOCK_1X16)
+        return NVFP4_ERR_ARG;
+    if (o->dgrad_rht != 0 && o->dgrad_rht != 1) return NVFP4_ERR_ARG;
+    if (o->dgrad_rht && o->weight_block_mode != NVFP4_BLOCK_1X16) return NVFP4_ERR_ARG;
+    return NVFP4_OK;
+}
+
+int nvfp4_linear_fprop_ex(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
+                          const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
+                          size_t ws_bytes, nvfp4_stream_t stream) {
     if (!X || !W || !Y) return NVFP4_ERR_ARG;
     uint32_t mask = 0;
     if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
-    int rc = lin_check(M, K, N, ws, ws_bytes);
+    int rc = opts_check(opts);
     if (rc) return rc;
+    const bool w1d = opts && opts->weight_block_mode == NVFP4_BLOCK_1X16;
+    const int dgrad_rht = opts ? opts->dgrad_rht : 0;
+    if ((rc = lin_check(M, K, N, ws, ws_bytes))) return rc;
     if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16)) return NVFP4_ERR_ALIGN;
     int sms = 0;
     if ((rc = device_check(&sms))) return rc;
@@ -366,21 +380,32 @@ int nvfp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t
     rc = run_quantize(X, M, K, false, 0, 0, 0, 1, mask, xr.data, xr.scales, xr.tensor_scale, xc.data,
                       xc.scales, xc.tensor_scale, words + kWX, status, sms, st, false);
     if (rc) return rc;
-    // W: 16x16 RNE, both orientations -- one read
-    rc = run_quantize(W, N, K, true, 0, 0, 0, 0, 0, wr.data, wr.scales, wr.tensor_scale, wc.data,
-                      wc.scales, wc.tensor_scale, words + kWW, status, sms, st, false);
+    // W -- one read: 16x16 RNE shared by both orientations, or (1D-weight recipe) 1x16
+    // RNE along K for fprop and, separately, 1x16 RNE along N for dgrad, rotated
+    // along N under the Mosaic recipe
+    rc = run_quantize(W, N, K, !w1d, 0, 0, 0, w1d ? dgrad_rht : 0, mask, wr.data, wr.scales,
+                      wr.tensor_scale, wc.data, wc.scales, wc.tensor_scale, words + kWW, status, sms, st,
+                      false);
     if (rc) return rc;
     return gemm_call(xr.data, xr.scales, wr.data, wr.scales, xr.tensor_scale, wr.tensor_scale, 1.0f,
                      M, N, K, Y, nullptr, status, sms, st);
 }
 
-int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
+int nvfp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
                        const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    return nvfp4_linear_fprop_ex(X, W, Y, M, K, N, rht_signs, nullptr, ws, ws_bytes, stream);
+}
+
+int nvfp4_linear_dgrad_ex(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                          const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
+                          size_t ws_bytes, nvfp4_stream_t stream) {
     if (!dY || !dX) return NVFP4_ERR_ARG;
     uint32_t mask = 0;
     if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
-    int rc = lin_check(M, K, N, ws, ws_bytes);
+    int rc = opts_check(opts);
     if (rc) return rc;
+    const int dgrad_rht = opts ? opts->dgrad_rht : 0;
+    if ((rc = lin_check(M, K, N, ws, ws_bytes))) return rc;
     if (!aligned(dY, 16) || !aligned(dX, 16)) return NVFP4_ERR_ALIGN;
     int sms = 0;
     if ((rc = device_check(&sms))) return rc;
@@ -392,12 +417,19 @@ int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N
     uint32_t* words = static_cast<uint32_t*>(ws);
     int* status = reinterpret_cast<int*>(words + kWordStatus);
     if (cudaMemsetAsync(words, 0, kClearBytes, st) != cudaSuccess) return NVFP4_ERR_CUDA;
-    // dY: rows (1x16 SR, stream 0) for dgrad, RHT columns (1x16 SR, stream 1) for wgrad
+    // dY: rows (1x16 SR, stream 0; rotated along N under the Mosaic recipe) for dgrad,
+    // RHT columns (1x16 SR, stream 1) for wgrad
     rc = run_quantize(dY, M, N, false, 1, 1, seed, 1, mask, dr.data, dr.scales, dr.tensor_scale,
-                      dc.data, dc.scales, dc.tensor_scale, words + kWDY, status, sms, st, false);
+                      dc.data, dc.scales, dc.tensor_scale, words + kWDY, status, sms, st, false, dgrad_rht);
     if (rc) return rc;
-    return gemm_call(dr.data, dr.scales, wc.data, wc.scales, dr.tensor_scale, wc.tensor_scale, 1.0f,
-                     M, K, N, dX, nullptr, status, sms, st);
+    // with both operands rotated along N the rotation cancels: H H^T = 16 I
+    return gemm_call(dr.data, dr.scales, wc.data, wc.scales, dr.tensor_scale, wc.tensor_scale,
+                     dgrad_rht ? 1.0f / 16.0f : 1.0f, M, K, N, dX, nullptr, status, sms, st);
+}
+
+int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                       const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    return nvfp4_linear_dgrad_ex(dY, dX, M, K, N, seed, rht_signs, nullptr, ws, ws_bytes, stream);
 }
 
 int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N, uint64_t seed,

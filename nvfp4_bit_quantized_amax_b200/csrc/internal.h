@@ -20,6 +20,7 @@ struct QuantParams {
     int* status;
     uint64_t seed;
     int row_sr, col_sr, col_rht;
+    int row_rht;         // rotate the row orientation too (tile kernel, ungrouped, 1x16)
     uint32_t sign_mask;  // bit i set: rotation sign i is -1
     uint32_t rk[20];     // Philox4x32-10 round keys of `seed` (filled by the launchers)
     // Grouped tensors (mixture of experts): row r belongs to group
@@ -55,7 +56,8 @@ inline void philox_round_keys(uint64_t seed, uint32_t (&rk)[20]) {
 }
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
-                        uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st);
+                        uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st,
+                        bool row_rht = false);
 cudaError_t launch_quant_rows(const QuantParams& p, int sm_count, cudaStream_t st);
 cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, cudaStream_t st);
 cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st);

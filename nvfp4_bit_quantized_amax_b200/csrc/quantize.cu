@@ -38,6 +38,37 @@ __device__ __forceinline__ void fwht16(double (&y)[16]) {
     }
 }
 
+// 16-point rotation of a row chunk held by a lane pair (even lane: elements 0-7,
+// odd lane: 8-15; both lanes of every pair call this together): three butterfly
+// stages inside the lane, the last across the pair.  In fp64, exact like fwht16;
+// y receives the lane's eight outputs.
+__device__ __forceinline__ void rht16_lane_pair(const uint4& w, uint32_t sign_mask, int lane,
+                                                double (&y)[8]) {
+    const int base = (lane & 1) * 8;
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t b = (k & 1) ? (ws[k >> 1] >> 16) : (ws[k >> 1] & 0xFFFFu);
+        y[k] = (double)__uint_as_float((b ^ (((sign_mask >> (base + k)) & 1u) << 15)) << 16);
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if ((k & h) == 0) {
+                const double a = y[k], b = y[k + h];
+                y[k] = a + b;
+                y[k + h] = a - b;
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const double o = __shfl_xor_sync(0xFFFFFFFFu, y[k], 1);
+        y[k] = (lane & 1) ? o - y[k] : y[k] + o;
+    }
+}
+
 // bf16 bit pattern with its sign flipped where the rotation sign is -1.
 __device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t flip) {
     return (double)__uint_as_float((bits16 ^ (flip << 15)) << 16);
@@ -51,7 +82,9 @@ __device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t f
 // ============================================================================
 // Grouped (kGrouped): the rows of a unit lie in one group, whose words are
 // words[2g] and words[2g+1]; each unit is folded into them by the warp.
-template <bool kColRht, bool kGrouped>
+// kRowRht: word 0 (or 2g) is max |RHT16 along the rows| instead of max |x| (the
+// row orientation is rotated); a non-finite input still makes it non-finite.
+template <bool kColRht, bool kGrouped, bool kRowRht>
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, uint32_t sign_mask,
                                                    uint32_t* __restrict__ words,
@@ -62,6 +95,7 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     const int64_t units = ((rows + 15) >> 4) * col_units;
     uint32_t m_row = 0;   // two packed 16-bit magnitudes
     double m_col = 0.0;
+    double m_rrht = 0.0;  // kRowRht: max |rotated row|
     for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += (int64_t)gridDim.x * 8) {
         const int64_t r0 = (u / col_units) * 16;
         const int64_t c0 = (u % col_units) * 256 + lane * 8;
@@ -69,11 +103,21 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
             m_row = 0;
             m_col = 0.0;
         }
-        if (c0 < cols) {
+        if (kRowRht || c0 < cols) {
         uint4 v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-            v[i] = (r0 + i < rows) ? ld_stream_v4(x + (r0 + i) * cols + c0) : make_uint4(0, 0, 0, 0);
+            v[i] = (c0 < cols && r0 + i < rows) ? ld_stream_v4(x + (r0 + i) * cols + c0)
+                                                : make_uint4(0, 0, 0, 0);
+        if (kRowRht) {  // every lane takes part (zeros past the columns)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                double y[8];
+                rht16_lane_pair(v[i], sign_mask, lane, y);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m_rrht = fmax(m_rrht, fabs(y[k]));
+            }
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             m_row = __vmaxu2(m_row, v[i].x & 0x7FFF7FFFu);
@@ -112,6 +156,7 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     }
     if (kGrouped) return;
     uint32_t a_row = max(m_row & 0xFFFFu, m_row >> 16) << 16;
+    if (kRowRht && a_row < 0x7F800000u) a_row = __float_as_uint(__double2float_rn(m_rrht));
     uint32_t a_col = kColRht ? __float_as_uint(__double2float_rn(m_col)) : 0u;
     a_row = __reduce_max_sync(0xFFFFFFFFu, a_row);
     a_col = __reduce_max_sync(0xFFFFFFFFu, a_col);
@@ -240,7 +285,10 @@ constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;
 // Grouped (kGrouped): the tile's rows lie in one group g (see QuantParams), which
 // supplies the tensor scales, the Philox key seed + g and the origin of the
 // element indices.
-template <bool k2D, bool kRht, bool kGrouped>
+// kRowRht: the row orientation is rotated too (16-point RHT along each row block,
+// the block's lane pair exchanging halves), e.g. dgrad operands under the Mosaic
+// recipe.
+template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
 __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
     __shared__ __align__(16) uint16_t tile[kTR][kPitch];
     __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
@@ -375,16 +423,28 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
             const int64_t r = r0 + lr, c = c0 + lc;
             uint32_t s;
             float inv;
-            if (k2D) {
+            float v[8];
+            if (kRowRht) {
+                double y[8];
+                rht16_lane_pair(reg[k], p.sign_mask, lane, y);
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    v[i] = __double2float_rn(y[i]);
+                    amax = fmaxf(amax, fabsf(v[i]));
+                }
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+                block_scale(amax, tr, s, inv);
+            } else if (k2D) {
                 s = tile_s[lr >> 4][lc >> 4];
                 inv = tile_inv[lr >> 4][lc >> 4];
+                unpack8(reg[k], v);
             } else {
                 float amax = absmax8(reg[k]);
                 amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
                 block_scale(amax, tr, s, inv);
+                unpack8(reg[k], v);
             }
-            float v[8];
-            unpack8(reg[k], v);
             const uint32_t codes =
                 encode8(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
             if (r < p.rows && c < p.cols) {
@@ -481,13 +541,18 @@ static int grid_for(int64_t work_items, int per_block, int sm_count, int blocks_
 }
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
-                        uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st) {
+                        uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st,
+                        bool row_rht) {
     const int64_t units = ((rows + 15) / 16) * ((cols + 255) / 256);
     const int grid = grid_for(units, 8, sm_count, 8);
-    if (col_rht)
-        amax_kernel<true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+    if (row_rht && col_rht)
+        amax_kernel<true, false, true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+    else if (row_rht)
+        amax_kernel<false, false, true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+    else if (col_rht)
+        amax_kernel<true, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
     else
-        amax_kernel<false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+        amax_kernel<false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
     return cudaGetLastError();
 }
 
@@ -496,10 +561,10 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
     const int grid = grid_for(units, 8, sm_count, 8);
     uint32_t* words = const_cast<uint32_t*>(p.amax_words);
     if (p.col_rht)
-        amax_kernel<true, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
+        amax_kernel<true, true, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
                                                      p.group_rows_uniform);
     else
-        amax_kernel<false, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
+        amax_kernel<false, true, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
                                                       p.group_rows_uniform);
     return cudaGetLastError();
 }
@@ -571,19 +636,25 @@ cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, cudaStream_
     philox_round_keys(p.seed, p.rk);
     const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
     const bool grouped = p.row_group != nullptr || p.group_rows_uniform > 0;
+    if (p.row_rht && (grouped || two_d)) return cudaErrorInvalidValue;
+    const bool col_rht = p.col_rht && p.col_data;
     if (grouped) {
         if (two_d)
-            quant_tile_kernel<true, false, true><<<grid, 256, 0, st>>>(p);
-        else if (p.col_rht && p.col_data)
-            quant_tile_kernel<false, true, true><<<grid, 256, 0, st>>>(p);
+            quant_tile_kernel<true, false, true, false><<<grid, 256, 0, st>>>(p);
+        else if (col_rht)
+            quant_tile_kernel<false, true, true, false><<<grid, 256, 0, st>>>(p);
         else
-            quant_tile_kernel<false, false, true><<<grid, 256, 0, st>>>(p);
+            quant_tile_kernel<false, false, true, false><<<grid, 256, 0, st>>>(p);
     } else if (two_d)
-        quant_tile_kernel<true, false, false><<<grid, 256, 0, st>>>(p);
-    else if (p.col_rht && p.col_data)
-        quant_tile_kernel<false, true, false><<<grid, 256, 0, st>>>(p);
+        quant_tile_kernel<true, false, false, false><<<grid, 256, 0, st>>>(p);
+    else if (p.row_rht && col_rht)
+        quant_tile_kernel<false, true, false, true><<<grid, 256, 0, st>>>(p);
+    else if (p.row_rht)
+        quant_tile_kernel<false, false, false, true><<<grid, 256, 0, st>>>(p);
+    else if (col_rht)
+        quant_tile_kernel<false, true, false, false><<<grid, 256, 0, st>>>(p);
     else
-        quant_tile_kernel<false, false, false><<<grid, 256, 0, st>>>(p);
+        quant_tile_kernel<false, false, false, false><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
