@@ -34,6 +34,10 @@
  *      dgrad operands dY and W^T are rotated along N, their shared reduction axis,
  *      i.e. along the rows of the quantized view (orient 0 with rht); the dgrad
  *      alpha takes the 1/16.
+ *  R15 MXFP4 ([NVX] "What NVFP4 actually is" names it: E2M1 elements, a power-of-two
+ *      E8M0 scale per 32 elements, no tensor scale): the block scale is the smallest
+ *      power of two 2^k with amax_b <= 6 * 2^k (nothing clipped), E8M0 code
+ *      k + 127; elements round to nearest even.
  */
 #include "nvfp4_oracle.h"
 
@@ -487,4 +491,88 @@ void ora_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
             ora_dot(A, sfA, B, sfB, K, alpha, m, n, &D[m * N + n], &bound[m * N + n]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4, the comparison format ([NVX] "What NVFP4 actually is": E2M1 elements,  */
+/* one power-of-two E8M0 scale per 32-element block, 4.25 bits per element)     */
+/* ------------------------------------------------------------------------ */
+
+/* E8M0: value 2^(e - 127) for e in 0..254; 255 is NaN. */
+double ora_e8m0_decode(unsigned code) {
+    code &= 0xFFu;
+    if (code == 255u) return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* R15: the block scale is the smallest power of two 2^k with amax_b <= 6 * 2^k,
+ * so no element is clipped; e = k + 127 clamped to [0, 254] (an all-zero block
+ * takes e = 0).  Found by brute force over k.                                  */
+unsigned ora_mx_scale_code(double amax_b) {
+    if (!(amax_b > 0.0)) return 0u;
+    for (int k = -127; k <= 127; ++k)
+        if (amax_b <= 6.0 * ldexp(1.0, k)) {
+            int e = k + 127;
+            return (unsigned)(e < 0 ? 0 : (e > 254 ? 254 : e));
+        }
+    return 254u;
+}
+
+/* Row orientation, 1x32 blocks along the columns, round-to-nearest-even: each
+ * element is x / 2^(e - 127) (exact in fp64) encoded to E2M1.  packed: rows x
+ * cols/2 bytes (low nibble = even element); sf: rows x cols/32 logical codes.   */
+int ora_mx_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* packed,
+                         uint8_t* sf) {
+    if (cols % 32 != 0) return -2;
+    const int64_t nkb = cols / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t kb = 0; kb < nkb; ++kb) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs((double)ora_bf16_to_f32(x[r * cols + kb * 32 + i]));
+                if (isnan(a)) return -3;
+                if (a > amax) amax = a;
+            }
+            if (isinf(amax)) return -3;
+            const unsigned e = ora_mx_scale_code(amax);
+            sf[r * nkb + kb] = (uint8_t)e;
+            const double scale = ora_e8m0_decode(e);
+            for (int i = 0; i < 32; ++i) {
+                const int64_t c = kb * 32 + i;
+                const double v = (double)ora_bf16_to_f32(x[r * cols + c]) / scale;
+                const unsigned code = ora_e2m1_encode_rne(v);
+                uint8_t* byte = &packed[r * (cols / 2) + c / 2];
+                if (c & 1)
+                    *byte = (uint8_t)((*byte & 0x0Fu) | (code << 4));
+                else
+                    *byte = (uint8_t)((*byte & 0xF0u) | code);
+            }
+        }
+    }
+    return 0;
+}
+
+/* D[m][n] = alpha * sum_k a(m,k) * b(n,k), a = e2m1 * 2^(e - 127) per 32-block,
+ * in fp64 (every product exact); bound = |alpha| * sum |a * b|.                */
+static double ora_mx_deq(const uint8_t* P, const uint8_t* sf, int64_t row, int64_t k, int64_t K) {
+    uint8_t byte = P[row * (K / 2) + k / 2];
+    unsigned code = (k & 1) ? (byte >> 4) : (byte & 15u);
+    return ora_e2m1_decode(code) * ora_e8m0_decode(sf[row * (K / 32) + k / 32]);
+}
+
+void ora_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                 int64_t M, int64_t N, int64_t K, double alpha, double* D, double* bound,
+                 int nthreads) {
+#pragma omp parallel for num_threads(ora_threads(nthreads)) schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = ora_mx_deq(A, sfA, m, k, K) * ora_mx_deq(B, sfB, n, k, K);
+                acc += p;
+                mag += fabs(p);
+            }
+            D[m * N + n] = alpha * acc;
+            bound[m * N + n] = fabs(alpha) * mag;
+        }
 }

@@ -104,4 +104,17 @@ void ora_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B,
 #ifdef __cplusplus
 }
 #endif
+/* ---- MXFP4, the comparison format --------------------------------------- */
+/* E8M0 scale 2^(e-127) (255 NaN); R15: block scale = smallest 2^k with
+ * amax_b <= 6 * 2^k (e clamped to [0, 254]; all-zero block: e = 0).  Row
+ * orientation, 1x32 blocks, RNE.  Scale layout: the atoms of ora_sf_swizzle over
+ * 32-element blocks (call it with vcols / 2).                                   */
+double   ora_e8m0_decode(unsigned code);
+unsigned ora_mx_scale_code(double amax_b);
+int  ora_mx_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* packed,
+                          uint8_t* sf);
+void ora_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                 int64_t M, int64_t N, int64_t K, double alpha, double* D, double* bound,
+                 int nthreads);
+
 #endif

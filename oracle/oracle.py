@@ -41,6 +41,10 @@ def lib():
             "ora_sf_swizzle": (None, [vp, i64, i64, vp]),
             "ora_gemm_pairs": (None, [vp, vp, vp, vp, i64, f64, i64, vp, vp, vp, vp, ci]),
             "ora_gemm": (None, [vp, vp, vp, vp, i64, i64, i64, f64, vp, vp, ci]),
+            "ora_e8m0_decode": (f64, [C.c_uint]),
+            "ora_mx_scale_code": (C.c_uint, [f64]),
+            "ora_mx_quantize_rows": (ci, [vp, i64, i64, vp, vp]),
+            "ora_mx_gemm": (None, [vp, vp, vp, vp, i64, i64, i64, f64, vp, vp, ci]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -226,3 +230,42 @@ def gemm(A, sfA, B, sfB, alpha, nthreads=0):
 
 def num_threads_default():
     return os.cpu_count() or 1
+
+
+# ---- MXFP4 (the comparison format; reading R15) ------------------------------------
+def e8m0_decode(code):
+    return lib().ora_e8m0_decode(int(code))
+
+
+def mx_scale_code(amax_b):
+    return lib().ora_mx_scale_code(float(amax_b))
+
+
+def mx_quantize(x_bits):
+    """Row orientation, 1x32 E8M0 blocks, RNE: returns (packed, sf_logical)."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, cols = x.shape
+    packed = np.zeros((rows, cols // 2), dtype=np.uint8)
+    sf = np.zeros((rows, cols // 32), dtype=np.uint8)
+    rc = lib().ora_mx_quantize_rows(_p(x), rows, cols, _p(packed), _p(sf))
+    if rc != 0:
+        raise ValueError(f"ora_mx_quantize_rows failed: {rc}")
+    return packed, sf
+
+
+def mx_sf_swizzle(sf_logical, vcols):
+    """The block-scaled MMA's atom layout over 32-element blocks."""
+    return sf_swizzle(sf_logical, vcols // 2)
+
+
+def mx_gemm(A, sfA, B, sfB, alpha, nthreads=0):
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    sfA = np.ascontiguousarray(sfA, dtype=np.uint8)
+    sfB = np.ascontiguousarray(sfB, dtype=np.uint8)
+    M, N, K = A.shape[0], B.shape[0], A.shape[1] * 2
+    D = np.zeros((M, N), dtype=np.float64)
+    bound = np.zeros((M, N), dtype=np.float64)
+    lib().ora_mx_gemm(_p(A), _p(sfA), _p(B), _p(sfB), M, N, K, float(alpha), _p(D), _p(bound),
+                      int(nthreads))
+    return D, bound
