@@ -270,6 +270,28 @@ int nvfp4_linear_dgrad_ex(const void* dY, void* dX, int64_t M, int64_t K, int64_
                           const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
                           size_t ws_bytes, nvfp4_stream_t stream);
 
+/*
+ * MXFP4, the comparison format ("Nemotron NVFP4" explainer, "What NVFP4 actually
+ * is": E2M1 elements with one power-of-two E8M0 scale per 32 elements, 4.25 bits
+ * per element, no tensor scale).  The pages fix no scale rule; the block scale is
+ * the smallest power of two 2^k with amax_b <= 6 * 2^k, so no element clips (E8M0
+ * code k + 127; 0 for an all-zero block; 255 when the block holds Inf or NaN), and
+ * elements round to nearest even.
+ * nvfp4_mx_quantize: row orientation, blocks along cols (cols % 32 == 0); one read.
+ *   packed  out, rows * cols / 2 bytes; scales out, nvfp4_mx_scale_bytes(rows, cols)
+ *   bytes in the layout of nvfp4_scale_bytes' scales over 32-element blocks (512-byte
+ *   atoms of 128 rows x 4 blocks; padding written as 0).
+ * nvfp4_mx_gemm: D = alpha * A B^T over MXFP4 operands (tcgen05 block-scaled MMA,
+ *   scale_vec::2X with UE8M0 scales); K % 128 == 0, N % 8 == 0; D_bf16 and / or
+ *   D_f32 as in nvfp4_gemm; status (nullable) as in nvfp4_gemm.
+ */
+size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols);
+int nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* scales,
+                      nvfp4_stream_t stream);
+int nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, float alpha,
+                  int64_t M, int64_t N, int64_t K, void* D_bf16, float* D_f32, int* status,
+                  nvfp4_stream_t stream);
+
 /* Views of the quantized operands a linear workspace holds (no device access). */
 enum {
     NVFP4_LIN_X_ROW = 0,  /* X,   M x K, 1x16 RNE                 */

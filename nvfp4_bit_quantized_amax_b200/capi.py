@@ -30,6 +30,7 @@ EXPORTS = (
     "nvfp4_moe_workspace_bytes", "nvfp4_moe_expert_workspace", "nvfp4_moe_linear_fprop",
     "nvfp4_moe_linear_dgrad", "nvfp4_moe_linear_wgrad", "nvfp4_moe_gather", "nvfp4_moe_combine",
     "nvfp4_linear_fprop_ex", "nvfp4_linear_dgrad_ex",
+    "nvfp4_mx_scale_bytes", "nvfp4_mx_quantize", "nvfp4_mx_gemm",
     "nvfp4_moe_grouped_workspace_bytes", "nvfp4_moe_grouped_operand", "nvfp4_moe_grouped_fprop",
     "nvfp4_moe_grouped_dgrad", "nvfp4_moe_grouped_wgrad",
 )
@@ -98,6 +99,9 @@ def load(path: str = LIB_PATH):
         "nvfp4_moe_combine": (ci, [vp, vp, i64, ci, i64, vp, vp]),
         "nvfp4_linear_fprop_ex": (ci, [vp, vp, vp, i64, i64, i64, vp, C.POINTER(LinearOpts), vp, sz, vp]),
         "nvfp4_linear_dgrad_ex": (ci, [vp, vp, i64, i64, i64, u64, vp, C.POINTER(LinearOpts), vp, sz, vp]),
+        "nvfp4_mx_scale_bytes": (sz, [i64, i64]),
+        "nvfp4_mx_quantize": (ci, [vp, i64, i64, vp, vp, vp]),
+        "nvfp4_mx_gemm": (ci, [vp, vp, vp, vp, f32, i64, i64, i64, vp, vp, vp, vp]),
         "nvfp4_moe_grouped_workspace_bytes": (sz, [vp, ci, i64, i64]),
         "nvfp4_moe_grouped_operand": (ci, [vp, vp, ci, i64, i64, ci, C.POINTER(Tensor)]),
         "nvfp4_moe_grouped_fprop": (ci, [vp, vp, vp, vp, ci, i64, i64, vp, vp, sz, vp]),
@@ -259,6 +263,23 @@ def nvfp4_linear_dgrad_ex(dY, dX, seed, rht_signs, ws, weight_block_mode=1, dgra
         _ptr(dY), _ptr(dX), M, K, N, seed, sp, C.byref(o), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
     del keep
+
+
+def mx_scale_bytes(rows, cols):
+    return load().nvfp4_mx_scale_bytes(rows, cols)
+
+
+def nvfp4_mx_quantize(x, packed, scales, stream=None):
+    rows, cols = x.shape
+    _check("nvfp4_mx_quantize", load().nvfp4_mx_quantize(_ptr(x), rows, cols, _ptr(packed),
+                                                         _ptr(scales), _stream(stream)))
+
+
+def nvfp4_mx_gemm(A, sfA, B, sfB, alpha, M, N, K, D_bf16=None, D_f32=None, status=None,
+                  stream=None):
+    _check("nvfp4_mx_gemm", load().nvfp4_mx_gemm(
+        _ptr(A), _ptr(sfA), _ptr(B), _ptr(sfB), float(alpha), M, N, K, _ptr(D_bf16),
+        _ptr(D_f32), _ptr(status), _stream(stream)))
 
 
 def nvfp4_linear_operand(ws, M, K, N, which):

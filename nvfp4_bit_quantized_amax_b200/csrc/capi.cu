@@ -706,6 +706,53 @@ int moe_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8
 
 extern "C" {
 
+size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols) {
+    if (rows <= 0 || cols <= 0 || cols % 32) return 0;
+    return (size_t)(pad(rows, 128) * pad(cols / 32, 4));
+}
+
+int nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* scales,
+                      nvfp4_stream_t stream) {
+    if (!x || !packed || !scales) return NVFP4_ERR_ARG;
+    if (rows < 1 || cols < 32 || cols % 32 || rows > (1ll << 40) / cols) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(packed, 16)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_mx_quant_rows(static_cast<const uint16_t*>(x), rows, cols, packed, scales, sms, st);
+    if (e == cudaSuccess) e = launch_sf_pad(scales, rows, cols / 32, sms, st);
+    return cuda_status(e);
+}
+
+int nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, float alpha,
+                  int64_t M, int64_t N, int64_t K, void* D_bf16, float* D_f32, int* status,
+                  nvfp4_stream_t stream) {
+    if (!A || !sfA || !B || !sfB || (!D_bf16 && !D_f32)) return NVFP4_ERR_ARG;
+    if (M < 1 || N < 8 || K < 128 || K % 128 != 0 || N % 8 != 0) return NVFP4_ERR_SHAPE;
+    if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K / 2 > (1ll << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sfA, 16) || !aligned(sfB, 16) ||
+        (D_bf16 && !aligned(D_bf16, 16)) || (D_f32 && !aligned(D_f32, 16)))
+        return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    int rc = device_check(&sms);
+    if (rc) return rc;
+    GemmParams g{};
+    g.A = A;
+    g.sfA = sfA;
+    g.B = B;
+    g.sfB = sfB;
+    g.alpha = alpha;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.D_bf16 = D_bf16;
+    g.D_f32 = D_f32;
+    g.status = status;
+    g.mx = 1;
+    return cuda_status(launch_gemm(g, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t nvfp4_moe_grouped_workspace_bytes(const int64_t* group_rows, int E, int64_t K, int64_t N) {
     if (moe_grouped_check(group_rows, E, K, N)) return 0;
     return (size_t)moe_layout(group_rows, E, K, N).total;

@@ -156,6 +156,26 @@ __device__ __forceinline__ void tc_mma_nvf4_x4(uint32_t d_tmem, uint64_t adesc, 
         : "memory");
 }
 
+// MXFP4 (kMx): E2M1 operands with UE8M0 scales over 32-element blocks
+// (block_scale.scale_vec::2X).  A 512-byte scale atom holds 4 blocks of 32 per row,
+// i.e. two K = 64 steps; the instruction descriptor's scale-factor ids (bits 29-30
+// for A, 4-5 for B) pick the byte pair of the step: 0 for the first, 2 for the
+// second.  The four steps of a k-tile read atoms 0, 0, 1, 1.
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X"
+        " [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ uint32_t mx_sf_id(uint32_t idesc, uint32_t id) {
+    return idesc | (id << 29) | (id << 4);
+}
+
 // Bulk tensor store of a shared-memory box to global memory (async proxy), and
 // its completion groups: .read waits until the source buffer may be reused.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
@@ -192,9 +212,9 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
 // Instruction descriptor of kind::mxf4nvf4 block-scaled MMA: E2M1 A and B
 // (format 1), K-major both, UE4M3 scales (scale format 0), M = 128, N = BN,
 // K = 64 per instruction, dense.
-template <int BN>
+template <int BN, bool kMx = false>
 __host__ __device__ constexpr uint32_t nvf4_idesc() {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (0u << 23) |
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((kMx ? 1u : 0u) << 23) |
            ((uint32_t)(kBM >> 4) << 24);
 }
 
@@ -355,7 +375,7 @@ __device__ __forceinline__ TileJob tile_job(const GemmParams& p, int64_t tile, i
     return j;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool kMx>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
@@ -368,8 +388,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t katoms = p.K / 64;                 // scale atoms per 128-row group of A
-    const int64_t katoms_b = (p.Kb ? p.Kb : p.K) / 64;  // ... and of B
+    // scale atoms per 128-row group of A and of B (an atom covers 64, or for MX 128,
+    // reduction elements)
+    constexpr int64_t kAtomK = kMx ? 128 : 64;
+    const int64_t katoms = (p.K + kAtomK - 1) / kAtomK;
+    const int64_t katoms_b = ((p.Kb ? p.Kb : p.K) + kAtomK - 1) / kAtomK;
     const int64_t nb_groups = (p.N + 127) / 128;     // 128-row groups of B (per group)
     const int64_t tiles_n = (p.N + BN - 1) / BN;
     const int64_t tiles_per_group = ((p.M + kBM - 1) / kBM) * tiles_n;
@@ -417,12 +440,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     const int64_t rem = (jb.k_len - (int64_t)kt * 256) / kKStep;
                     const int nks = rem < 4 ? (int)rem : 4;
-                    const uint32_t sf_bytes = (uint32_t)nks * 512u;
+                    const uint32_t sf_bytes = (uint32_t)(kMx ? (nks + 1) / 2 : nks) * 512u;
                     uint32_t bytes = kBM * kBKBytes + BN * kBKBytes + sf_bytes;
                     for (int g = 0; g < G; ++g)
                         if (jb.n0 / 128 + g < nb_groups) bytes += sf_bytes;
                     const uint32_t fb = smem_addr(&S.full[s]);
-                    const int64_t katom = jb.k0 / 64 + (int64_t)kt * 4;  // first scale atom of the k-tile
+                    const int64_t katom = (jb.k0 + (int64_t)kt * 256) / kAtomK;  // first scale atom of the k-tile
                     mbar_expect_tx(fb, bytes);
                     tma_load_2d(smem_addr(S.a[s]), &tmA, (int)((jb.k0 / 2) + kt * kBKBytes), (int)jb.a_row, fb);
                     tma_load_2d(smem_addr(S.b[s]), &tmB, (int)((jb.bk0 + jb.k0) / 2 + kt * kBKBytes), (int)jb.b_row, fb);
@@ -431,7 +454,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int g = 0; g < G; ++g)
                         if (jb.n0 / 128 + g < nb_groups)
                             bulk_load(smem_addr(S.sfb[s] + g * 2048),
-                                      p.sfB + ((jb.b_row / 128 + g) * katoms_b + jb.bk0 / 64 + katom) * 512,
+                                      p.sfB + ((jb.b_row / 128 + g) * katoms_b + jb.bk0 / kAtomK + katom) * 512,
                                       sf_bytes, fb);
                 }
             }
@@ -450,7 +473,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // tensor pipe.  So the loop keeps stage, phase and descriptors in
             // registers and waits on one barrier per k-tile: the scale writers
             // arrive on sf_full only after they saw the stage's bytes land.
-            constexpr uint32_t idesc = nvf4_idesc<BN>();
+            constexpr uint32_t idesc = nvf4_idesc<BN, kMx>();
             constexpr uint64_t kAStep = (kBM * kBKBytes) >> 4, kBStep = (BN * kBKBytes) >> 4;
             const uint64_t adesc0 = operand_desc(smem_addr(S.a[0]));
             const uint64_t bdesc0 = operand_desc(smem_addr(S.b[0]));
@@ -478,7 +501,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint64_t ad = adesc0 + kAStep * s, bd = bdesc0 + kBStep * s;
                     const uint32_t t_sfa = tsf0 + (uint32_t)TL::kRegion * s;
                     const uint32_t t_sfb = t_sfa + TL::kSfaCols;
-                    if (kt < KT_full) {
+                    if (kMx) {
+                        const int nks = kt < KT_full ? 4 : (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
+                        for (int j = 0; j < nks; ++j)
+                            tc_mma_mx(tmem, ad + 2u * j, bd + 2u * j, mx_sf_id(idesc, 2u * (j & 1)),
+                                      t_sfa + 4 * (j >> 1), t_sfb + 4 * G * (j >> 1),
+                                      (kt > 0 || j > 0) ? 1u : 0u);
+                    } else if (kt < KT_full) {
                         tc_mma_nvf4_x4<G>(tmem, ad, bd, idesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
                     } else {  // K tail: 1 to 3 steps of 64
                         const int nks = (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
@@ -999,7 +1028,7 @@ static bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) 
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool kMx>
 static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream_t st) {
     CUtensorMap ma, mb, md;
     const int64_t b_rows = p.group_mode == 1 && p.b_group_rows ? p.b_group_rows * p.num_groups : p.N;
@@ -1012,7 +1041,7 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream
     const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel<BN, STAGES>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel<BN, STAGES, kMx>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -1020,7 +1049,7 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream
     int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
     if (p.group_mode == 2) tiles *= p.num_groups;
     const unsigned grid = (unsigned)(tiles < sm_count ? tiles : sm_count);
-    gemm_nvf4_kernel<BN, STAGES><<<grid, kGemmThreads, smem, st>>>(ma, mb, md, p);
+    gemm_nvf4_kernel<BN, STAGES, kMx><<<grid, kGemmThreads, smem, st>>>(ma, mb, md, p);
     return cudaGetLastError();
 }
 
@@ -1065,8 +1094,9 @@ static cudaError_t launch_gemm_pair(const GemmParams& p, int sm_count, cudaStrea
 }
 
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
-    if (p.group_mode == 0 && p.M > 128 && sm_count >= 2) return launch_gemm_pair<5>(p, sm_count, st);
-    return launch_gemm_cfg<256, 4>(p, sm_count, st);
+    if (!p.mx && p.group_mode == 0 && p.M > 128 && sm_count >= 2) return launch_gemm_pair<5>(p, sm_count, st);
+    if (p.mx) return launch_gemm_cfg<256, 4, true>(p, sm_count, st);
+    return launch_gemm_cfg<256, 4, false>(p, sm_count, st);
 }
 
 }  // namespace nvfp4

@@ -61,6 +61,8 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
 cudaError_t launch_quant_rows(const QuantParams& p, int sm_count, cudaStream_t st);
 cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, cudaStream_t st);
 cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st);
+cudaError_t launch_mx_quant_rows(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* packed,
+                                 uint8_t* sf, int sm_count, cudaStream_t st);
 cudaError_t launch_rht(const uint16_t* x, float* y, int64_t rows, int64_t cols, int axis,
                        uint32_t sign_mask, int sm_count, cudaStream_t st);
 
@@ -97,6 +99,7 @@ struct GemmParams {
     const int64_t* k_start;
     const int64_t* k_len;
     int num_groups;
+    int mx;  // MXFP4 operands: UE8M0 scales over 32-element blocks, no tensor scales
 };
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st);
 

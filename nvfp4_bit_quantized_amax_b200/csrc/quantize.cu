@@ -456,6 +456,64 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
 }
 
 // ============================================================================
+// MXFP4 (the comparison format): row orientation, E8M0 scale per 32 elements,
+// round-to-nearest-even, one pass (no tensor scale, so no amax prepass).  Every
+// lane owns 8 consecutive elements; a 32-block is a lane quad.  The scale is the
+// smallest power of two 2^k with amax <= 6 * 2^k: for amax = (1 + f) * 2^E, k =
+// E - 2 if f <= 1/2 else E - 1, code e = k + 127 (0 for a zero or subnormal
+// amax, 255 when the block holds Inf / NaN); elements are x * 2^-k, exact.
+// ============================================================================
+__global__ void __launch_bounds__(256) mx_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                            int64_t cols, uint8_t* __restrict__ packed,
+                                                            uint8_t* __restrict__ sf) {
+    const int64_t cpr = cols >> 3;  // 8-chunks per row (a multiple of 4)
+    const int64_t nchunks = rows * cpr;
+    const int64_t katoms = (cols / 32 + 3) >> 2;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < nchunks;
+         base += stride) {
+        const int64_t q = base + (threadIdx.x & 31);
+        const bool valid = q < nchunks;
+        const uint4 w = valid ? ld_stream_v4(x + q * 8) : make_uint4(0, 0, 0, 0);
+        float amax = absmax8(w);
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        const uint32_t ab = __float_as_uint(amax);
+        uint32_t e;
+        if (ab >= 0x7F800000u)
+            e = 255u;
+        else if ((ab >> 23) == 0u)
+            e = 0u;
+        else
+            e = (ab >> 23) - 2u + ((ab & 0x7FFFFFu) > 0x400000u ? 1u : 0u);
+        // 2^-k = 2^(127 - e) (e <= 253 for finite bf16 input, so this is a normal float)
+        const float mult = e == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float((254u - e) << 23);
+        float v[8];
+        unpack8(w, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], mult);
+        const uint32_t codes = e2m1x8_rn(v);
+        if (valid) {
+            reinterpret_cast<uint32_t*>(packed)[q] = codes;
+            if ((q & 3) == 0) {
+                const int64_t r = q / cpr, kb = (q % cpr) >> 2;
+                sf[sf_offset(r, kb, katoms)] = (uint8_t)e;
+            }
+        }
+    }
+}
+
+static int grid_for(int64_t work_items, int per_block, int sm_count, int blocks_per_sm);
+
+cudaError_t launch_mx_quant_rows(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* packed,
+                                 uint8_t* sf, int sm_count, cudaStream_t st) {
+    const int64_t nchunks = rows * (cols / 8);
+    const int grid = grid_for(nchunks, 256, sm_count, 8);
+    mx_quant_rows_kernel<<<grid, 256, 0, st>>>(x, rows, cols, packed, sf);
+    return cudaGetLastError();
+}
+
+// ============================================================================
 // Zero fill of the scale padding: rows [rows, pad128(rows)) and 16-blocks
 // [nb, pad4(nb)) of an operand with `rows` rows and `nb` 16-blocks per row.
 // ============================================================================
