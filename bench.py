@@ -304,6 +304,25 @@ def run_ours(args, rank, world, local_rank):
             "hbm_peak_GB/s": peaks["hbm_gbs"],
         }
 
+    # ---- MXFP4, the comparison format: one-pass quantize of X and W, MX GEMM (fprop shape)
+    if "kernels" in out:
+        xm = (torch.empty(M * K // 2, dtype=torch.uint8, device=dev),
+              torch.empty(capi.mx_scale_bytes(M, K), dtype=torch.uint8, device=dev))
+        wm = (torch.empty(N * K // 2, dtype=torch.uint8, device=dev),
+              torch.empty(capi.mx_scale_bytes(N, K), dtype=torch.uint8, device=dev))
+        iters_mx = max(10, min(50, args.steps))
+        qx_ms = timed(lambda: capi.nvfp4_mx_quantize(X, *xm), iters_mx, 3)
+        qw_ms = timed(lambda: capi.nvfp4_mx_quantize(W, *wm), iters_mx, 3)
+        g_mx = timed(lambda: capi.nvfp4_mx_gemm(xm[0], xm[1], wm[0], wm[1], 1.0, M, N, K, D_bf16=Y),
+                     iters_mx, 3)
+        mx_bytes_per_el = 2.0 + 0.5 + 1.0 / 32   # one read, codes + E8M0 scales written
+        out["kernels"]["mxfp4"] = {
+            "quantize_X_ms": round(qx_ms, 4), "quantize_W_ms": round(qw_ms, 4),
+            "quantize_GB/s": round(mx_bytes_per_el * (M * K + N * K) / ((qx_ms + qw_ms) * 1e-3) / 1e9, 1),
+            "gemm_fprop_ms": round(g_mx, 4),
+            "gemm_fprop_tflops": round(FLOPS_PER_GEMM / (g_mx * 1e-3) / 1e12, 1),
+            "note": "1-SM kernel, block_scale.scale_vec::2X, UE8M0 per 32 elements"}
+
     # ---- mixture-of-experts expert layer (64 experts, Zipf(1.1) top-4 routing)
     if not args.no_moe:
         out["moe"] = moe_step_bench(capi, syn, dev, stream, timed, max_over_ranks, world,
