@@ -34,11 +34,11 @@ FLOPS_PER_GEMM = 2.0 * M * K * N
 FLOPS_PER_STEP = 3 * FLOPS_PER_GEMM
 KERNELS_PER_STEP = 9  # 2 amax + 2 quantize (fprop), 1 + 1 (dgrad), 3 GEMMs
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
-# DRAM bytes (read + write) of one fprop GEMM launch at this workload, from one ncu
-# capture (profiles/gemm_nvf4_pair_fprop_8192x20480x5120_traffic.md); reported only
-# while the GEMM source is the one that was captured.
-GEMM_TRAFFIC = {"gemm_cu_sha256_16": "dd3efb8a564996a2", "bytes": 382145024 + 311861504,
-                "launch": "fprop M=8192 N=20480 K=5120"}
+# DRAM bytes (read + write) of one launch of each GEMM of the step, from one-pass ncu
+# captures (profiles/gemm_nvf4_pair_mlp12b_traffic.md); reported only while the GEMM
+# source is the one that was captured.
+GEMM_TRAFFIC = {"gemm_cu_sha256_16": "7ca9e5b2a0a54209", "bytes": {
+    "fprop": 87931136 + 293433088, "dgrad": 434238464 + 68137472, "wgrad": 118976256 + 175343360}}
 
 
 def env_rank():
@@ -281,17 +281,18 @@ def run_ours(args, rank, world, local_rank):
                  for k, v in q_ms.items()}
         q_total_bytes = sum(q_bytes_per_el * v[1] for v in q_ms.values())
         q_total_ms = sum(v[0] for v in q_ms.values())
-        traffic = args.traffic
+        traffic, traffic_by_gemm = args.traffic, None
         if traffic is None:
             import hashlib
             with open(os.path.join(ROOT, "nvfp4_bit_quantized_amax_b200", "csrc", "gemm.cu"), "rb") as f:
                 if hashlib.sha256(f.read()).hexdigest()[:16] == GEMM_TRAFFIC["gemm_cu_sha256_16"]:
-                    traffic = GEMM_TRAFFIC["bytes"]
+                    traffic_by_gemm = GEMM_TRAFFIC["bytes"]
+                    traffic = round(sum(traffic_by_gemm.values()) / 3)
         out["roofline"] = {
             "bound": "tensor", "kernel": "gemm_nvf4_pair_kernel (fprop/dgrad/wgrad average)",
             "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
             "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
-            "traffic_launch": GEMM_TRAFFIC["launch"] if traffic is not None else None,
+            "traffic_by_gemm": traffic_by_gemm,
             "peak_source": f"{peak_kind}: FP4 = {FP4_OVER_BF16:g} x bf16 burst "
                            f"{peaks['bf16_tflops']} TFLOP/s (nominal 9 / 2.25 PFLOP/s ratio)",
         }

@@ -740,9 +740,35 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int64_t katoms = p.K / 64;
     const int KT = (int)((p.K + 255) / 256);
     const int64_t na_groups = (p.M + 127) / 128, nb_groups = (p.N + 127) / 128;
-    const int64_t tiles_n = (p.N + BN - 1) / BN;
-    const int64_t tiles = ((p.M + 255) / 256) * tiles_n;
+    const int64_t tiles_n = (p.N + BN - 1) / BN, tiles_m = (p.M + 255) / 256;
+    const int64_t tiles = tiles_m * tiles_n;
     const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+    // Tile order, for reuse of the operands in L2 (measured on the DRAM counters):
+    // if the smaller operand (codes + scales) fits in a quarter of L2 the clusters
+    // sweep along its dimension first, so it is re-read from L2 while the larger one
+    // streams from DRAM once; otherwise neither stays resident across waves and
+    // the tiles go in bands of kBand 256-row tile rows (M fastest inside a band),
+    // so each wave reads about as many A bands as B bands.
+    constexpr int64_t kBand = 8;
+    const int64_t small_bytes = (p.M < p.N ? p.M : p.N) * (p.K / 2 + p.K / 16);
+    const int order = small_bytes <= (int64_t(32) << 20) ? (p.M < p.N ? 1 : 0) : 2;
+    auto tile_origin = [&](int64_t pt, int64_t& m0, int64_t& n0) {
+        int64_t tm, tn;
+        if (order == 0) {  // N fastest
+            tm = pt / tiles_n;
+            tn = pt % tiles_n;
+        } else if (order == 1) {  // M fastest
+            tm = pt % tiles_m;
+            tn = pt / tiles_m;
+        } else {
+            const int64_t band = pt / (kBand * tiles_n), w = pt % (kBand * tiles_n);
+            const int64_t rows = tiles_m - band * kBand < kBand ? tiles_m - band * kBand : kBand;
+            tm = band * kBand + w % rows;
+            tn = w / rows;
+        }
+        m0 = tm * 256;
+        n0 = tn * BN;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -777,7 +803,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t s = 0, ph = 0;
             int64_t issued = 0;
             for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
-                const int64_t m0 = (pt / tiles_n) * 256, n0 = (pt % tiles_n) * BN;
+                int64_t m0, n0;
+            tile_origin(pt, m0, n0);
                 for (int kt = 0; kt < KT; ++kt, ++issued) {
                     if (issued >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u)) {
                         timed_out = 1;
@@ -811,7 +838,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t s = 0, ph = 0;
             int64_t issued = 0;
             for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
-                const int64_t m0 = (pt / tiles_n) * 256, n0 = (pt % tiles_n) * BN;
+                int64_t m0, n0;
+            tile_origin(pt, m0, n0);
                 const int64_t a_group = (m0 + 128 * rank) / 128;
                 for (int kt = 0; kt < KT; ++kt, ++issued) {
                     if (issued >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u)) {
@@ -961,7 +989,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         uint32_t local = 0;
         for (int64_t pt = cid; pt < tiles; pt += ncl, ++local) {
             if (*(volatile int*)&timed_out) break;
-            const int64_t m0 = (pt / tiles_n) * 256, n0 = (pt % tiles_n) * BN;
+            int64_t m0, n0;
+            tile_origin(pt, m0, n0);
             const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u);
             tc_fence_after();
             __syncwarp();

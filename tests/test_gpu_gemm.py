@@ -120,6 +120,16 @@ def test_gemm_square_sweep_sampled(ora, n):
     sampled_gemm_check(ora, n, n, n, seed=n)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (2432, 2688, 25600),   # smaller operand > 32 MB: bands of 8 tile rows, last band 2 rows (one half tile)
+    (640, 2304, 1024),     # M < N, small operands: M fastest, ragged last tile row
+    (2304, 640, 1024),     # M >= N: N fastest, ragged last tile column
+])
+def test_gemm_tile_orders_sampled(ora, M, N, K):
+    """Every tile of the 2-SM kernel is computed once in each of its tile orders."""
+    sampled_gemm_check(ora, M, N, K, seed=M + 3 * N, nsamp=4096)
+
+
 @pytest.mark.parametrize("N,K", syn.GEMM_SKINNY_WGRAD)
 def test_gemm_skinny_wgrad_sampled(ora, N, K):
     """wgrad shapes: output N x K, reduction over 32768 tokens."""
