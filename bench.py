@@ -38,7 +38,7 @@ FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
 # captures (profiles/gemm_nvf4_pair_mlp12b_traffic.md); reported only while the GEMM
 # source is the one that was captured.
 GEMM_TRAFFIC = {"gemm_cu_sha256_16": "7ca9e5b2a0a54209", "bytes": {
-    "fprop": 87931136 + 293433088, "dgrad": 434238464 + 68137472, "wgrad": 118976256 + 175343360}}
+    "fprop": 86695168 + 296710656, "dgrad": 406735104 + 71220224, "wgrad": 118866944 + 178942720}}
 
 
 def env_rank():
