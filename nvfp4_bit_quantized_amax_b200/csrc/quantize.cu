@@ -293,6 +293,12 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
     __shared__ __align__(16) uint16_t tile[kTR][kPitch];
     __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
     __shared__ float tile_inv[kTR / 16][kTC / 16];
+    // The tile's scales, staged so that they leave in wide stores instead of one
+    // byte each: the column orientation's 128 columns x 4 blocks are exactly one
+    // 512-byte atom; the row orientation's 64 rows x 8 blocks are 8 bytes of each
+    // of the 32 lines of two atoms.  Entries past the tensor hold 0 (the padding).
+    __shared__ __align__(16) uint8_t col_atom[512];
+    __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t r0 = (int64_t)blockIdx.y * kTR, c0 = (int64_t)blockIdx.x * kTC;
@@ -354,7 +360,6 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
         const int lc = 32 * (warp & 3) + lane;
         const int j0 = 2 * (warp >> 2);
         const int64_t c = c0 + lc;
-        const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
         uint32_t out[4];
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
@@ -399,23 +404,26 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
                 }
                 out[2 * jj] = encode8(lo8, inv, p.col_sr, rk, 1u, e0);
                 out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, rk, 1u, e0 + 8);
-                if (c < p.cols && r0 + 16 * j < p.rows)
-                    p.col_sf[sf_offset(c, (r0 >> 4) + j, katoms_c)] = (uint8_t)s;
+                // atom byte of (column lc, block j): line lc % 32, group lc / 32
+                col_atom[lane * 16 + (warp & 3) * 4 + j] =
+                    (c < p.cols && r0 + 16 * j < p.rows) ? (uint8_t)s : (uint8_t)0;
             }
         }
         if (want_col && c < p.cols) {
             uint8_t* base = p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j0) >> 1);
-            if (r0 + 16 * j0 < p.rows)
-                *reinterpret_cast<uint2*>(base) = make_uint2(out[0], out[1]);
-            if (r0 + 16 * (j0 + 1) < p.rows)
-                *reinterpret_cast<uint2*>(base + 8) = make_uint2(out[2], out[3]);
+            const bool both = r0 + 16 * (j0 + 1) < p.rows;
+            if (both && (reinterpret_cast<uintptr_t>(base) & 15u) == 0) {
+                *reinterpret_cast<uint4*>(base) = make_uint4(out[0], out[1], out[2], out[3]);
+            } else {
+                if (r0 + 16 * j0 < p.rows) *reinterpret_cast<uint2*>(base) = make_uint2(out[0], out[1]);
+                if (both) *reinterpret_cast<uint2*>(base + 8) = make_uint2(out[2], out[3]);
+            }
         }
         if (k2D) __syncthreads();
     }
 
     // ---- row pass from registers: a 16-block is a lane pair
     if (want_row) {
-        const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int q = k * 256 + tid;
@@ -447,10 +455,33 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
             }
             const uint32_t codes =
                 encode8(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
-            if (r < p.rows && c < p.cols) {
-                *reinterpret_cast<uint32_t*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
-                if ((lc & 15) == 0) p.row_sf[sf_offset(r, c >> 4, katoms_r)] = (uint8_t)s;
-            }
+            const bool inside = r < p.rows && c < p.cols;
+            if (inside) *reinterpret_cast<uint32_t*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
+            // (row lr, block lc / 16): half-atom lc / 64, line lr % 32, byte 4 * (lr / 32) + block % 4
+            if ((lc & 15) == 0)
+                row_half_atoms[lc >> 6][lr & 31][(lr >> 5) * 4 + ((lc >> 4) & 3)] = inside ? (uint8_t)s : (uint8_t)0;
+        }
+    }
+
+    // ---- scale stores.  Every entry written lies inside the scale buffer: the
+    // column atom is (128-column group c0 / 128, blocks r0 / 16 .. + 3) with r0 a
+    // multiple of 64 below the rows; the row half-atoms cover 64 rows below
+    // pad128(rows), and the second is skipped when its blocks start past the
+    // padded block count.
+    __syncthreads();
+    if (want_col && warp == 0) {
+        const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
+        const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
+        *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) =
+            *reinterpret_cast<const uint4*>(col_atom + lane * 16);
+    }
+    if (want_row && (warp == 2 || warp == 3)) {
+        const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
+        const int a = warp - 2;
+        if ((c0 >> 6) + a < katoms_r) {
+            const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
+            *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
+                *reinterpret_cast<const uint2*>(row_half_atoms[a][lane]);
         }
     }
 }
