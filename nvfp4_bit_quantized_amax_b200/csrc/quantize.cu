@@ -288,8 +288,17 @@ constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;
 // kRowRht: the row orientation is rotated too (16-point RHT along each row block,
 // the block's lane pair exchanging halves), e.g. dgrad operands under the Mosaic
 // recipe.
+// Resident CTAs per SM that the register budget is sized for.  A CTA loads its
+// tile once and then only computes and stores, so more resident CTAs keep more
+// loads in flight; the grouped RHT variant keeps three (at four it spills).
+template <bool k2D, bool kRht, bool kGrouped>
+constexpr int quant_tile_min_blocks() {
+    return (kGrouped && kRht) ? 3 : 4;
+}
+
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
-__global__ void __launch_bounds__(256) quant_tile_kernel(QuantParams p) {
+__global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGrouped>()))
+    quant_tile_kernel(QuantParams p) {
     __shared__ __align__(16) uint16_t tile[kTR][kPitch];
     __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
     __shared__ float tile_inv[kTR / 16][kTC / 16];
