@@ -23,6 +23,9 @@
  *    are recorded in a status word in the caller's workspace; read it with
  *    nvfp4_read_status() (which synchronizes the stream).
  *  - No entry point traps, asserts on the device or throws across the ABI.
+ *  - A tensor quantized in both orientations or in 16x16 blocks (nvfp4_quantize_2d,
+ *    16x16 nvfp4_quantize, the linear and expert-layer calls) has at most
+ *    4,194,240 rows (65535 tiles of 64); larger ones return NVFP4_ERR_SHAPE.
  *
  * Numerics (fixed readings of points the pages leave open):
  *  - decode scale g = amax / (6 * 448) (fp32), encode factor 2688 / amax.

@@ -147,9 +147,9 @@ int gemm_call(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint
 // ---------------------------------------------------------------- mixture of experts
 int moe_check(const int64_t* group_rows, int E, int64_t K, int64_t N) {
     if (!group_rows || E < 1) return NVFP4_ERR_ARG;
-    if (K < 64 || N < 64 || K % 64 || N % 64) return NVFP4_ERR_SHAPE;
+    if (K < 64 || N < 64 || K % 64 || N % 64 || N > kMaxTileRows) return NVFP4_ERR_SHAPE;
     for (int e = 0; e < E; ++e)
-        if (group_rows[e] < 0 || group_rows[e] % 64) return NVFP4_ERR_SHAPE;
+        if (group_rows[e] < 0 || group_rows[e] % 64 || group_rows[e] > kMaxTileRows) return NVFP4_ERR_SHAPE;
     return NVFP4_OK;
 }
 
@@ -219,7 +219,7 @@ int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int block_mode, in
     if (block_mode != NVFP4_BLOCK_1X16 && block_mode != NVFP4_BLOCK_16X16) return NVFP4_ERR_ARG;
     if (rounding != NVFP4_ROUND_RNE && rounding != NVFP4_ROUND_SR) return NVFP4_ERR_ARG;
     if (rows < 1 || cols < 16 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
-    if (block_mode == NVFP4_BLOCK_16X16 && rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (block_mode == NVFP4_BLOCK_16X16 && (rows % 16 != 0 || rows > kMaxTileRows)) return NVFP4_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 16) || !aligned(workspace, 16) ||
         !aligned(tensor_scale, 4))
         return NVFP4_ERR_ALIGN;
@@ -248,7 +248,7 @@ int nvfp4_quantize_2d(const void* x, int64_t rows, int64_t cols, const nvfp4_qua
         if (o->block_mode != NVFP4_BLOCK_1X16) return NVFP4_ERR_ARG;
         if (sign_mask_of(o->rht_signs, &mask)) return NVFP4_ERR_ARG;
     }
-    if (rows < 1 || cols < 16 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (rows < 1 || cols < 16 || cols % 16 != 0 || rows > kMaxTileRows) return NVFP4_ERR_SHAPE;
     if ((col_out || o->block_mode == NVFP4_BLOCK_16X16) && rows % 16 != 0) return NVFP4_ERR_SHAPE;
     for (nvfp4_tensor* t : {row_out, col_out}) {
         if (!t) continue;
@@ -339,6 +339,7 @@ int nvfp4_linear_operand(void* ws, int64_t M, int64_t K, int64_t N, int which, n
 static int lin_check(int64_t M, int64_t K, int64_t N, void* ws, size_t ws_bytes) {
     if (!ws) return NVFP4_ERR_WORKSPACE;
     if (M < 64 || K < 64 || N < 64 || M % 64 || K % 64 || N % 64) return NVFP4_ERR_SHAPE;
+    if (M > kMaxTileRows || N > kMaxTileRows) return NVFP4_ERR_SHAPE;
     if (ws_bytes < nvfp4_linear_workspace_bytes(M, K, N)) return NVFP4_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return NVFP4_ERR_ALIGN;
     return NVFP4_OK;
@@ -618,7 +619,7 @@ int moe_grouped_check(const int64_t* group_rows, int E, int64_t K, int64_t N) {
         if (group_rows[e] < 0 || group_rows[e] % 128) return NVFP4_ERR_SHAPE;
         R += group_rows[e];
     }
-    if (R < 128 || R > (1ll << 31) - 256) return NVFP4_ERR_SHAPE;
+    if (R < 128 || R > kMaxTileRows || (int64_t)E * N > kMaxTileRows) return NVFP4_ERR_SHAPE;
     return NVFP4_OK;
 }
 

@@ -34,6 +34,11 @@ struct QuantParams {
     int64_t group_rows_uniform;
 };
 
+// Rows one launch of the quantize tile kernel covers: 64-row tiles along the
+// grid's y extent (at most 65535).  The entry points refuse larger tensors as a
+// shape error.
+constexpr int64_t kMaxTileRows = 65535ll * 64;
+
 cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t st);
 
 // Group tables of a grouped tensor from its group sizes (host array of E <=

@@ -73,7 +73,7 @@ extern "C" int nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols,
     if (block_mode != NVFP4_BLOCK_1X16 && block_mode != NVFP4_BLOCK_16X16) return NVFP4_ERR_ARG;
     if (rounding != NVFP4_ROUND_RNE && rounding != NVFP4_ROUND_SR) return NVFP4_ERR_ARG;
     if (rows < 1 || cols < 16 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
-    if (block_mode == NVFP4_BLOCK_16X16 && rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (block_mode == NVFP4_BLOCK_16X16 && (rows % 16 != 0 || rows > kMaxTileRows)) return NVFP4_ERR_SHAPE;
     // the scratch this call needs must fit the static array (it needs the same 64
     // bytes for every tensor size today; a larger need is refused, not truncated)
     const size_t needed = kNeededBytes;

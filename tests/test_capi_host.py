@@ -209,3 +209,27 @@ def test_moe_grouped_operand_views(lib):
     assert spans[0][0] >= (1 << 24) and spans[-1][1] <= (1 << 24) + total
     with pytest.raises(RuntimeError):
         capi.nvfp4_moe_grouped_operand(FakeWs(), groups, K, N, 6)
+
+
+def test_tile_row_limit(lib):
+    """Tensors quantized by the tile kernel (two orientations or 16x16 blocks) take at
+    most 65535 x 64 rows; one row tile more is a shape error, found on the host."""
+    from nvfp4_bit_quantized_amax_b200 import capi
+    p = C.c_void_p(4096)
+    big = 65535 * 64 + 64
+    q = lib.nvfp4_quantize
+    assert q(p, big, 16, 1, 0, 0, p, p, p, p, None) == capi.ERR_SHAPE
+    assert lib.nvfp4_quantize_noalloc(p, big, 16, 1, 0, 0, p, p, p, None) == capi.ERR_SHAPE
+    opts = capi.QuantizeOpts(0, 0, 0, 0, 0, None)
+    t = capi.Tensor(4096, 4096, 4096, 0, 0)
+    assert lib.nvfp4_quantize_2d(p, big, 16, C.byref(opts), C.byref(t), None, p, None) == capi.ERR_SHAPE
+    sp = np.array([1, -1] * 8, dtype=np.int8).ctypes.data_as(C.c_void_p)
+    assert lib.nvfp4_linear_fprop(p, p, p, big, 64, 64, sp, p, 1 << 62, None) == capi.ERR_SHAPE
+    assert lib.nvfp4_linear_fprop(p, p, p, 64, 64, big, sp, p, 1 << 62, None) == capi.ERR_SHAPE
+    assert capi.moe_grouped_workspace_bytes(np.array([65535 * 64 + 128], dtype=np.int64), 128, 128) == 0
+    # W of all experts [E*N][K] is one tile launch too: 1024 x 4096 rows is 64 too many
+    assert capi.moe_grouped_workspace_bytes(np.array([128] * 1024, dtype=np.int64), 128, 4096) == 0
+    assert capi.moe_grouped_workspace_bytes(np.array([128] * 1024, dtype=np.int64), 128, 3968) > 0
+    g = np.array([big], dtype=np.int64)
+    assert lib.nvfp4_moe_linear_fprop(p, p, p, g.ctypes.data_as(C.c_void_p), 1, 64, 64, sp, p,
+                                      1 << 62, None) == capi.ERR_SHAPE
