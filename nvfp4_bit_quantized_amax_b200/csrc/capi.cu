@@ -369,7 +369,7 @@ int nvfp4_linear_fprop_ex(const void* X, const void* W, void* Y, int64_t M, int6
     int sms = 0;
     if ((rc = device_check(&sms))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    nvfp4_tensor xr, xc, wr, wc;
+    nvfp4_tensor xr{}, xc{}, wr{}, wc{};
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_X_ROW, &xr);
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_X_COL, &xc);
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_W_ROW, &wr);
@@ -411,7 +411,7 @@ int nvfp4_linear_dgrad_ex(const void* dY, void* dX, int64_t M, int64_t K, int64_
     int sms = 0;
     if ((rc = device_check(&sms))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    nvfp4_tensor dr, dc, wc;
+    nvfp4_tensor dr{}, dc{}, wc{};
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_DY_ROW, &dr);
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_DY_COL, &dc);
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_W_COL, &wc);
@@ -444,7 +444,7 @@ int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N
     int sms = 0;
     if ((rc = device_check(&sms))) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    nvfp4_tensor dc, xc;
+    nvfp4_tensor dc{}, xc{};
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_DY_COL, &dc);
     nvfp4_linear_operand(ws, M, K, N, NVFP4_LIN_X_COL, &xc);
     uint32_t* words = static_cast<uint32_t*>(ws);
