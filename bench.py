@@ -229,100 +229,99 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_tflops(world, FLOPS_PER_STEP, ms)
 
     out = {}
-    if rank == 0 or True:
-        # ---- per-kernel timing on the same stream (each launch alone, back to back)
-        iters = max(10, min(50, args.steps))
-        ops = {w: capi.nvfp4_linear_operand(ws, M, K, N, w) for w in range(6)}
-        lib = capi.load()
+    # ---- per-kernel timing on the same stream (each launch alone, back to back); every
+    # rank runs it (timed() holds barriers)
+    iters = max(10, min(50, args.steps))
+    ops = {w: capi.nvfp4_linear_operand(ws, M, K, N, w) for w in range(6)}
+    lib = capi.load()
 
-        def gemm(a, b, alpha, D, Mx, Nx, Kx):
-            va, vb = ops[a], ops[b]
-            return lambda: lib.nvfp4_gemm(va.data, va.scales, vb.data, vb.scales,
-                                          va.tensor_scale, vb.tensor_scale, alpha, Mx, Nx, Kx,
-                                          D.data_ptr(), None, None, stream.cuda_stream)
+    def gemm(a, b, alpha, D, Mx, Nx, Kx):
+        va, vb = ops[a], ops[b]
+        return lambda: lib.nvfp4_gemm(va.data, va.scales, vb.data, vb.scales,
+                                      va.tensor_scale, vb.tensor_scale, alpha, Mx, Nx, Kx,
+                                      D.data_ptr(), None, None, stream.cuda_stream)
 
-        g_ms = {
-            "fprop": timed(gemm(capi.LIN_X_ROW, capi.LIN_W_ROW, 1.0, Y, M, N, K), iters, 3),
-            "dgrad": timed(gemm(capi.LIN_DY_ROW, capi.LIN_W_COL, 1.0, dX, M, K, N), iters, 3),
-            "wgrad": timed(gemm(capi.LIN_DY_COL, capi.LIN_X_COL, 1.0 / 16, dW, N, K, M), iters, 3),
-        }
-        qws = torch.empty(capi.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+    g_ms = {
+        "fprop": timed(gemm(capi.LIN_X_ROW, capi.LIN_W_ROW, 1.0, Y, M, N, K), iters, 3),
+        "dgrad": timed(gemm(capi.LIN_DY_ROW, capi.LIN_W_COL, 1.0, dX, M, K, N), iters, 3),
+        "wgrad": timed(gemm(capi.LIN_DY_COL, capi.LIN_X_COL, 1.0 / 16, dW, N, K, M), iters, 3),
+    }
+    qws = torch.empty(capi.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
 
-        def tview(w):
-            v = ops[w]
-            return (v.data, v.scales, v.tensor_scale)
+    def tview(w):
+        v = ops[w]
+        return (v.data, v.scales, v.tensor_scale)
 
-        def quant(x, bm, rr, cr, rht, row_w, col_w):
-            r = capi.Tensor(*tview(row_w), 0, 0) if row_w is not None else None
-            c = capi.Tensor(*tview(col_w), 0, 0) if col_w is not None else None
-            sgn = np.ascontiguousarray(signs)
-            opts = capi.QuantizeOpts(bm, rr, cr, seed, int(rht), sgn.ctypes.data)
-            import ctypes
-            args_ = (ctypes.c_void_p(x.data_ptr()), x.shape[0], x.shape[1], ctypes.byref(opts),
-                     ctypes.byref(r) if r is not None else None,
-                     ctypes.byref(c) if c is not None else None,
-                     ctypes.c_void_p(qws.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
-            return lambda: lib.nvfp4_quantize_2d(*args_)
+    def quant(x, bm, rr, cr, rht, row_w, col_w):
+        r = capi.Tensor(*tview(row_w), 0, 0) if row_w is not None else None
+        c = capi.Tensor(*tview(col_w), 0, 0) if col_w is not None else None
+        sgn = np.ascontiguousarray(signs)
+        opts = capi.QuantizeOpts(bm, rr, cr, seed, int(rht), sgn.ctypes.data)
+        import ctypes
+        args_ = (ctypes.c_void_p(x.data_ptr()), x.shape[0], x.shape[1], ctypes.byref(opts),
+                 ctypes.byref(r) if r is not None else None,
+                 ctypes.byref(c) if c is not None else None,
+                 ctypes.c_void_p(qws.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+        return lambda: lib.nvfp4_quantize_2d(*args_)
 
-        q_ms = {
-            "X_row+col_rht": (timed(quant(X, 0, 0, 0, True, capi.LIN_X_ROW, capi.LIN_X_COL), iters, 3), M * K),
-            "W_16x16_both": (timed(quant(W, 1, 0, 0, False, capi.LIN_W_ROW, capi.LIN_W_COL), iters, 3), N * K),
-            "dY_row_sr+col_rht_sr": (timed(quant(dY, 0, 1, 1, True, capi.LIN_DY_ROW, capi.LIN_DY_COL), iters, 3), M * N),
-        }
-        peaks, peak_kind = load_peaks()
-        fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-        gemm_avg_ms = sum(g_ms.values()) / 3
-        achieved = FLOPS_PER_GEMM / (gemm_avg_ms * 1e-3) / 1e12
-        # dual-orientation quantize: amax read 2 B + quantize read 2 B + 2 x (0.5 + 1/16) B written
-        q_bytes_per_el = 2.0 + 2.0 + 2 * (0.5 + 1.0 / 16)
-        quant = {k: {"ms": round(v[0], 4),
-                     "GB/s": round(q_bytes_per_el * v[1] / (v[0] * 1e-3) / 1e9, 1),
-                     "frac_hbm": round(q_bytes_per_el * v[1] / (v[0] * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
-                 for k, v in q_ms.items()}
-        q_total_bytes = sum(q_bytes_per_el * v[1] for v in q_ms.values())
-        q_total_ms = sum(v[0] for v in q_ms.values())
-        traffic, traffic_by_gemm = args.traffic, None
-        if traffic is None:
-            import hashlib
-            with open(os.path.join(ROOT, "nvfp4_bit_quantized_amax_b200", "csrc", "gemm.cu"), "rb") as f:
-                if hashlib.sha256(f.read()).hexdigest()[:16] == GEMM_TRAFFIC["gemm_cu_sha256_16"]:
-                    traffic_by_gemm = GEMM_TRAFFIC["bytes"]
-                    traffic = round(sum(traffic_by_gemm.values()) / 3)
-        out["roofline"] = {
-            "bound": "tensor", "kernel": "gemm_nvf4_pair_kernel (fprop/dgrad/wgrad average)",
-            "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-            "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
-            "traffic_by_gemm": traffic_by_gemm,
-            "peak_source": f"{peak_kind}: FP4 = {FP4_OVER_BF16:g} x bf16 burst "
-                           f"{peaks['bf16_tflops']} TFLOP/s (nominal 9 / 2.25 PFLOP/s ratio)",
-        }
-        out["kernels"] = {
-            "gemm_ms": {k: round(v, 4) for k, v in g_ms.items()},
-            "gemm_tflops": {k: round(FLOPS_PER_GEMM / (v * 1e-3) / 1e12, 1) for k, v in g_ms.items()},
-            "quantize": quant,
-            "quantize_GB/s": round(q_total_bytes / (q_total_ms * 1e-3) / 1e9, 1),
-            "quantize_frac_hbm": round(q_total_bytes / (q_total_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
-            "hbm_peak_GB/s": peaks["hbm_gbs"],
-        }
+    q_ms = {
+        "X_row+col_rht": (timed(quant(X, 0, 0, 0, True, capi.LIN_X_ROW, capi.LIN_X_COL), iters, 3), M * K),
+        "W_16x16_both": (timed(quant(W, 1, 0, 0, False, capi.LIN_W_ROW, capi.LIN_W_COL), iters, 3), N * K),
+        "dY_row_sr+col_rht_sr": (timed(quant(dY, 0, 1, 1, True, capi.LIN_DY_ROW, capi.LIN_DY_COL), iters, 3), M * N),
+    }
+    peaks, peak_kind = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_avg_ms = sum(g_ms.values()) / 3
+    achieved = FLOPS_PER_GEMM / (gemm_avg_ms * 1e-3) / 1e12
+    # dual-orientation quantize: amax read 2 B + quantize read 2 B + 2 x (0.5 + 1/16) B written
+    q_bytes_per_el = 2.0 + 2.0 + 2 * (0.5 + 1.0 / 16)
+    quant = {k: {"ms": round(v[0], 4),
+                 "GB/s": round(q_bytes_per_el * v[1] / (v[0] * 1e-3) / 1e9, 1),
+                 "frac_hbm": round(q_bytes_per_el * v[1] / (v[0] * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+             for k, v in q_ms.items()}
+    q_total_bytes = sum(q_bytes_per_el * v[1] for v in q_ms.values())
+    q_total_ms = sum(v[0] for v in q_ms.values())
+    traffic, traffic_by_gemm = args.traffic, None
+    if traffic is None:
+        import hashlib
+        with open(os.path.join(ROOT, "nvfp4_bit_quantized_amax_b200", "csrc", "gemm.cu"), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] == GEMM_TRAFFIC["gemm_cu_sha256_16"]:
+                traffic_by_gemm = GEMM_TRAFFIC["bytes"]
+                traffic = round(sum(traffic_by_gemm.values()) / 3)
+    out["roofline"] = {
+        "bound": "tensor", "kernel": "gemm_nvf4_pair_kernel (fprop/dgrad/wgrad average)",
+        "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+        "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
+        "traffic_by_gemm": traffic_by_gemm,
+        "peak_source": f"{peak_kind}: FP4 = {FP4_OVER_BF16:g} x bf16 burst "
+                       f"{peaks['bf16_tflops']} TFLOP/s (nominal 9 / 2.25 PFLOP/s ratio)",
+    }
+    out["kernels"] = {
+        "gemm_ms": {k: round(v, 4) for k, v in g_ms.items()},
+        "gemm_tflops": {k: round(FLOPS_PER_GEMM / (v * 1e-3) / 1e12, 1) for k, v in g_ms.items()},
+        "quantize": quant,
+        "quantize_GB/s": round(q_total_bytes / (q_total_ms * 1e-3) / 1e9, 1),
+        "quantize_frac_hbm": round(q_total_bytes / (q_total_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+        "hbm_peak_GB/s": peaks["hbm_gbs"],
+    }
 
     # ---- MXFP4, the comparison format: one-pass quantize of X and W, MX GEMM (fprop shape)
-    if "kernels" in out:
-        xm = (torch.empty(M * K // 2, dtype=torch.uint8, device=dev),
-              torch.empty(capi.mx_scale_bytes(M, K), dtype=torch.uint8, device=dev))
-        wm = (torch.empty(N * K // 2, dtype=torch.uint8, device=dev),
-              torch.empty(capi.mx_scale_bytes(N, K), dtype=torch.uint8, device=dev))
-        iters_mx = max(10, min(50, args.steps))
-        qx_ms = timed(lambda: capi.nvfp4_mx_quantize(X, *xm), iters_mx, 3)
-        qw_ms = timed(lambda: capi.nvfp4_mx_quantize(W, *wm), iters_mx, 3)
-        g_mx = timed(lambda: capi.nvfp4_mx_gemm(xm[0], xm[1], wm[0], wm[1], 1.0, M, N, K, D_bf16=Y),
-                     iters_mx, 3)
-        mx_bytes_per_el = 2.0 + 0.5 + 1.0 / 32   # one read, codes + E8M0 scales written
-        out["kernels"]["mxfp4"] = {
-            "quantize_X_ms": round(qx_ms, 4), "quantize_W_ms": round(qw_ms, 4),
-            "quantize_GB/s": round(mx_bytes_per_el * (M * K + N * K) / ((qx_ms + qw_ms) * 1e-3) / 1e9, 1),
-            "gemm_fprop_ms": round(g_mx, 4),
-            "gemm_fprop_tflops": round(FLOPS_PER_GEMM / (g_mx * 1e-3) / 1e12, 1),
-            "note": "1-SM kernel, block_scale.scale_vec::2X, UE8M0 per 32 elements"}
+    xm = (torch.empty(M * K // 2, dtype=torch.uint8, device=dev),
+          torch.empty(capi.mx_scale_bytes(M, K), dtype=torch.uint8, device=dev))
+    wm = (torch.empty(N * K // 2, dtype=torch.uint8, device=dev),
+          torch.empty(capi.mx_scale_bytes(N, K), dtype=torch.uint8, device=dev))
+    iters_mx = max(10, min(50, args.steps))
+    qx_ms = timed(lambda: capi.nvfp4_mx_quantize(X, *xm), iters_mx, 3)
+    qw_ms = timed(lambda: capi.nvfp4_mx_quantize(W, *wm), iters_mx, 3)
+    g_mx = timed(lambda: capi.nvfp4_mx_gemm(xm[0], xm[1], wm[0], wm[1], 1.0, M, N, K, D_bf16=Y),
+                 iters_mx, 3)
+    mx_bytes_per_el = 2.0 + 0.5 + 1.0 / 32   # one read, codes + E8M0 scales written
+    out["kernels"]["mxfp4"] = {
+        "quantize_X_ms": round(qx_ms, 4), "quantize_W_ms": round(qw_ms, 4),
+        "quantize_GB/s": round(mx_bytes_per_el * (M * K + N * K) / ((qx_ms + qw_ms) * 1e-3) / 1e9, 1),
+        "gemm_fprop_ms": round(g_mx, 4),
+        "gemm_fprop_tflops": round(FLOPS_PER_GEMM / (g_mx * 1e-3) / 1e12, 1),
+        "note": "1-SM kernel, block_scale.scale_vec::2X, UE8M0 per 32 elements"}
 
     # ---- mixture-of-experts expert layer (64 experts, Zipf(1.1) top-4 routing)
     if not args.no_moe:
