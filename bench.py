@@ -410,7 +410,7 @@ def moe_step_bench(capi, syn, dev, stream, timed, max_over_ranks, world, iters):
         capi.nvfp4_moe_combine(dX, slots, dX_tok)
         capi.nvfp4_moe_linear_wgrad(dW, d["group_rows"], 7, signs, pws)
 
-    ms_pe = max_over_ranks(timed(step_per_expert, 3, 1))
+    ms_pe = max_over_ranks(timed(step_per_expert, 3, 3))
     useful = 3 * 2.0 * T * k * K * N
     padded = 3 * 2.0 * rows * K * N
     return {"workload": "MoE expert layer: 64 experts, hidden 2048, FFN 1024, 16384 tokens, "
