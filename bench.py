@@ -35,8 +35,8 @@ FLOPS_PER_STEP = 3 * FLOPS_PER_GEMM
 KERNELS_PER_STEP = 9  # 2 amax + 2 quantize (fprop), 1 + 1 (dgrad), 3 GEMMs
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
 # DRAM bytes (read + write) of one launch of each GEMM of the step, from one-pass ncu
-# captures (profiles/gemm_nvf4_pair_mlp12b_traffic.md); reported only while the GEMM
-# source is the one that was captured.
+# captures of that launch; reported only while the GEMM source is the one that was
+# captured.
 GEMM_TRAFFIC = {"gemm_cu_sha256_16": "7ca9e5b2a0a54209", "bytes": {
     "fprop": 86695168 + 296710656, "dgrad": 406735104 + 71220224, "wgrad": 118866944 + 178942720}}
 

@@ -11,7 +11,7 @@
  * so that every `float` operation below is one IEEE-754 binary32 operation with
  * round-to-nearest-even and gradual underflow (no FMA contraction, no FTZ).
  *
- * Readings of points the pages leave open (each one also listed in the design doc):
+ * Readings of points the pages leave open (each one is the oracle's frozen spec):
  *  R1  E2M1 code = sign(bit 3) | exponent(bits 2:1, bias 1) | mantissa(bit 0);
  *      magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}.  ([NVX] "What NVFP4 actually is"
  *      fixes the 1-2-1 bit split; the value set follows from it.)

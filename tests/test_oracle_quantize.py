@@ -268,6 +268,26 @@ def test_row_rht_equals_column_rht_of_transpose(ora):
         assert np.array_equal(p0, p1) and np.array_equal(sf0, sf1)
 
 
+def test_row_rht_dense_product(ora):
+    """The standalone transform along the contiguous axis is the dense product
+    x_chunk . diag(s) . H16 of every 16-chunk of every row, rounded once to fp32: a
+    mistake that moves outputs to other columns, drops the signs or uses the wrong
+    chunk fails here, not only in the maximum."""
+    x = syn.normal_bf16((40, 96), 23, outlier_prob=0.02)
+    s = syn.rht_signs(7)
+    y = ora.rht(x, 1, s)
+    H = scipy.linalg.hadamard(16).astype(np.float64)
+    xf = syn.bf16_bits_to_f32(x).astype(np.float64)
+    ref = np.einsum("rji,i,ik->rjk", xf.reshape(40, 6, 16), s.astype(np.float64), H)
+    assert np.array_equal(y.reshape(40, 6, 16), ref.astype(np.float32))
+    # one nonzero input picks out one signed row of H in its own chunk, nothing else
+    e = np.zeros((2, 32), dtype=np.uint16)
+    e[1, 16 + 5] = 0x3F80  # 1.0
+    ye = ora.rht(e, 1, s)
+    assert (ye[0] == 0).all() and (ye[1, :16] == 0).all()
+    assert np.array_equal(ye[1, 16:], (s[5] * H[5]).astype(np.float32))
+
+
 def test_row_rht_amax_is_max_of_standalone_rht(ora):
     x = syn.normal_bf16((32, 96), 22)
     s = syn.rht_signs(4)
