@@ -57,7 +57,8 @@ typedef enum nvfp4_status {
     NVFP4_ERR_NONFINITE = -5, /* device status: the input held Inf or NaN           */
     NVFP4_ERR_TIMEOUT = -6,   /* device status: a bounded wait in a kernel ran out  */
     NVFP4_ERR_WORKSPACE = -7, /* workspace pointer null or smaller than required    */
-    NVFP4_ERR_DEVICE = -8     /* the current device is not sm_100 (B200 class)      */
+    NVFP4_ERR_DEVICE = -8,    /* the current device is not sm_100 (B200 class)      */
+    NVFP4_ERR_INDEX = -9      /* a row index lies outside its source tensor (device) */
 } nvfp4_status;
 
 enum { NVFP4_BLOCK_1X16 = 0, NVFP4_BLOCK_16X16 = 1 };
@@ -154,6 +155,21 @@ int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uin
                int64_t K, void* D_bf16, float* D_f32, int* status, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gemm_wait_limit -- nvfp4_gemm with the pipeline waits' bound set by the
+ * caller instead of the default 2^31 clock cycles (about a second): a testing hook
+ * for the failure path, not a computation of the pages.  With a bound of a few
+ * cycles the waits run out in normal operation; the kernel then records
+ * NVFP4_ERR_TIMEOUT in *status, stops issuing work, waits (with the default bound)
+ * for the copies and MMAs it already issued, frees its tensor memory and returns,
+ * and D is incomplete.  wait_cycles >= 0 (0 selects the default); other arguments
+ * as nvfp4_gemm.
+ */
+int nvfp4_gemm_wait_limit(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                          const float* scale_a, const float* scale_b, float alpha, int64_t M,
+                          int64_t N, int64_t K, void* D_bf16, float* D_f32, int* status,
+                          long long wait_cycles, nvfp4_stream_t stream);
+
+/*
  * Linear layer Y = X W^T in NVFP4 (artiverse.ca: forward, backward and weight-gradient
  * GEMMs in 4 bits; 16x16 weight blocks; RHT on the weight-gradient inputs; stochastic
  * rounding on gradients only).
@@ -231,6 +247,15 @@ int nvfp4_moe_grouped_operand(void* ws, const int64_t* group_rows, int E, int64_
 int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, const int64_t* group_rows,
                             int E, int64_t K, int64_t N, const int8_t* rht_signs, void* ws,
                             size_t ws_bytes, nvfp4_stream_t stream);
+/* nvfp4_moe_grouped_fprop with the routing gather fused into the quantization of X:
+ * row r of the permuted X is row row_src[r] of X_tok [tokens][K] (row_src: device
+ * int32 [R]; -1 reads as a zero row, the padding).  The permuted bf16 copy is never
+ * written.  Results equal nvfp4_moe_gather followed by nvfp4_moe_grouped_fprop.  An
+ * entry >= tokens is read as a zero row and recorded as NVFP4_ERR_INDEX in the status
+ * word.                                                                              */
+int nvfp4_moe_grouped_fprop_gather(const void* X_tok, const int32_t* row_src, int64_t tokens, const void* W,
+                                   void* Y_perm, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                                   const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
                             int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
                             size_t ws_bytes, nvfp4_stream_t stream);
@@ -318,8 +343,10 @@ int nvfp4_linear_operand(void* ws, int64_t M, int64_t K, int64_t N, int which,
  * of NVFP4_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
  * until exit; a call needing more than that would be refused with
  * NVFP4_ERR_WORKSPACE.  The first call on a device looks the array's address up
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  All calls share the array and each clears it on its stream
+ * (cudaGetSymbolAddress) with that device current and caches it for that device;
+ * make that first call before any stream capture.  The cached address belongs to
+ * the device's current context: after cudaDeviceReset the next call sees a new
+ * context and looks the address up again (make that call outside a capture too).  All calls share the array and each clears it on its stream
  * before use: calls that overlap on the GPU (other streams, other threads) race.
  * There is no status word to read back: an Inf/NaN input shows as a NaN
  * tensor_scale.  It calls no allocator.

@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libnvfp4.so")
 
 OK, ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_WORKSPACE, \
-    ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6, -7, -8
+    ERR_DEVICE, ERR_INDEX = 0, -1, -2, -3, -4, -5, -6, -7, -8, -9
 BLOCK_1X16, BLOCK_16X16 = 0, 1
 ROUND_RNE, ROUND_SR = 0, 1
 LIN_X_ROW, LIN_X_COL, LIN_W_ROW, LIN_W_COL, LIN_DY_ROW, LIN_DY_COL = range(6)
@@ -32,7 +32,8 @@ EXPORTS = (
     "nvfp4_linear_fprop_ex", "nvfp4_linear_dgrad_ex",
     "nvfp4_mx_scale_bytes", "nvfp4_mx_quantize", "nvfp4_mx_gemm",
     "nvfp4_moe_grouped_workspace_bytes", "nvfp4_moe_grouped_operand", "nvfp4_moe_grouped_fprop",
-    "nvfp4_moe_grouped_dgrad", "nvfp4_moe_grouped_wgrad",
+    "nvfp4_moe_grouped_dgrad", "nvfp4_moe_grouped_wgrad", "nvfp4_gemm_wait_limit",
+    "nvfp4_moe_grouped_fprop_gather",
 )
 
 
@@ -80,6 +81,8 @@ def load(path: str = LIB_PATH):
                                    C.POINTER(Tensor), vp, vp]),
         "nvfp4_rht": (ci, [vp, i64, i64, ci, vp, ci, vp, vp]),
         "nvfp4_gemm": (ci, [vp, vp, vp, vp, vp, vp, f32, i64, i64, i64, vp, vp, vp, vp]),
+        "nvfp4_gemm_wait_limit": (ci, [vp, vp, vp, vp, vp, vp, f32, i64, i64, i64, vp, vp, vp,
+                                       C.c_longlong, vp]),
         "nvfp4_linear_workspace_bytes": (sz, [i64, i64, i64]),
         "nvfp4_linear_fprop": (ci, [vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
         "nvfp4_linear_dgrad": (ci, [vp, vp, i64, i64, i64, u64, vp, vp, sz, vp]),
@@ -105,6 +108,7 @@ def load(path: str = LIB_PATH):
         "nvfp4_moe_grouped_workspace_bytes": (sz, [vp, ci, i64, i64]),
         "nvfp4_moe_grouped_operand": (ci, [vp, vp, ci, i64, i64, ci, C.POINTER(Tensor)]),
         "nvfp4_moe_grouped_fprop": (ci, [vp, vp, vp, vp, ci, i64, i64, vp, vp, sz, vp]),
+        "nvfp4_moe_grouped_fprop_gather": (ci, [vp, vp, i64, vp, vp, vp, ci, i64, i64, vp, vp, sz, vp]),
         "nvfp4_moe_grouped_dgrad": (ci, [vp, vp, vp, ci, i64, i64, u64, vp, vp, sz, vp]),
         "nvfp4_moe_grouped_wgrad": (ci, [vp, vp, ci, i64, i64, vp, sz, vp]),
     }
@@ -212,6 +216,15 @@ def nvfp4_gemm(A, sfA, B, sfB, alpha, M, N, K, D_bf16=None, D_f32=None, scale_a=
     _check("nvfp4_gemm", load().nvfp4_gemm(
         _ptr(A), _ptr(sfA), _ptr(B), _ptr(sfB), _ptr(scale_a), _ptr(scale_b), float(alpha), M, N,
         K, _ptr(D_bf16), _ptr(D_f32), _ptr(status), _stream(stream)))
+
+
+def nvfp4_gemm_wait_limit(A, sfA, B, sfB, alpha, M, N, K, wait_cycles, D_bf16=None, D_f32=None,
+                          scale_a=None, scale_b=None, status=None, stream=None):
+    """nvfp4_gemm with the pipeline waits bounded by `wait_cycles` clock cycles (a
+    testing hook of the timeout path; 0 selects the default bound)."""
+    _check("nvfp4_gemm_wait_limit", load().nvfp4_gemm_wait_limit(
+        _ptr(A), _ptr(sfA), _ptr(B), _ptr(sfB), _ptr(scale_a), _ptr(scale_b), float(alpha), M, N,
+        K, _ptr(D_bf16), _ptr(D_f32), _ptr(status), int(wait_cycles), _stream(stream)))
 
 
 def nvfp4_linear_fprop(X, W, Y, rht_signs, ws, stream=None):
@@ -359,6 +372,17 @@ def nvfp4_moe_grouped_fprop(X_perm, W, Y_perm, group_rows, rht_signs, ws, stream
     keep, sp = _signs(rht_signs)
     _check("nvfp4_moe_grouped_fprop", load().nvfp4_moe_grouped_fprop(
         _ptr(X_perm), _ptr(W), _ptr(Y_perm), gp, E, K, N, sp, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    del keep, g
+
+
+def nvfp4_moe_grouped_fprop_gather(X_tok, row_src, W, Y_perm, group_rows, rht_signs, ws, stream=None):
+    """Grouped fprop reading X's rows through row_src (the gather fused in)."""
+    g, gp = _rows(group_rows)
+    E, N, K = W.shape
+    keep, sp = _signs(rht_signs)
+    _check("nvfp4_moe_grouped_fprop_gather", load().nvfp4_moe_grouped_fprop_gather(
+        _ptr(X_tok), _ptr(row_src), X_tok.shape[0], _ptr(W), _ptr(Y_perm), gp, E, K, N, sp, _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
     del keep, g
 

@@ -126,8 +126,9 @@ int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_
 
 int gemm_call(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
               const float* sa, const float* sb, float alpha, int64_t M, int64_t N, int64_t K,
-              void* Dbf, float* Df, int* status, int sms, cudaStream_t st) {
+              void* Dbf, float* Df, int* status, int sms, cudaStream_t st, long long wait_cycles = 0) {
     GemmParams g{};
+    g.wait_cycles = wait_cycles;
     g.A = A;
     g.sfA = sfA;
     g.B = B;
@@ -197,6 +198,7 @@ const char* nvfp4_status_string(int s) {
         case NVFP4_ERR_TIMEOUT: return "a bounded wait in a kernel ran out";
         case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
         case NVFP4_ERR_DEVICE: return "device is not sm_100";
+        case NVFP4_ERR_INDEX: return "a row index lies outside its source tensor";
         default: return "unknown status";
     }
 }
@@ -300,7 +302,16 @@ int nvfp4_rht(const void* x, int64_t rows, int64_t cols, int axis, const int8_t*
 int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                const float* scale_a, const float* scale_b, float alpha, int64_t M, int64_t N,
                int64_t K, void* D_bf16, float* D_f32, int* status, nvfp4_stream_t stream) {
+    return nvfp4_gemm_wait_limit(A, sfA, B, sfB, scale_a, scale_b, alpha, M, N, K, D_bf16, D_f32,
+                                 status, 0, stream);
+}
+
+int nvfp4_gemm_wait_limit(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
+                          const float* scale_a, const float* scale_b, float alpha, int64_t M,
+                          int64_t N, int64_t K, void* D_bf16, float* D_f32, int* status,
+                          long long wait_cycles, nvfp4_stream_t stream) {
     if (!A || !sfA || !B || !sfB || (!D_bf16 && !D_f32)) return NVFP4_ERR_ARG;
+    if (wait_cycles < 0) return NVFP4_ERR_ARG;
     if (M < 1 || N < 8 || K < 64 || K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_SHAPE;
     if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K / 2 > (1ll << 31)) return NVFP4_ERR_SHAPE;
     if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sfA, 16) || !aligned(sfB, 16) ||
@@ -310,7 +321,7 @@ int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uin
     int rc = device_check(&sms);
     if (rc) return rc;
     return gemm_call(A, sfA, B, sfB, scale_a, scale_b, alpha, M, N, K, D_bf16, D_f32, status, sms,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<cudaStream_t>(stream), wait_cycles);
 }
 
 size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -568,14 +579,20 @@ struct MoeLayout {
     int64_t words_x, words_w, words_dy;          // 2E words each
     int64_t gx_row, gx_col, gw_row, gw_col, gdy_row, gdy_col;  // E floats each
     int64_t mtile_group, group_row0, group_nrows;
+    int64_t pair_row0, pair_group, pair_rows;  // 256-row tiles of the groups
     int64_t x_row, x_row_sf, x_col, x_col_sf, w_row, w_row_sf, w_col, w_col_sf;
     int64_t dy_row, dy_row_sf, dy_col, dy_col_sf, total;
     int64_t R;
+    int64_t pair_tiles;  // sum over groups of ceil(rows / 256)
 };
 MoeLayout moe_layout(const int64_t* group_rows, int E, int64_t K, int64_t N) {
     MoeLayout L;
     L.R = 0;
-    for (int e = 0; e < E; ++e) L.R += group_rows[e];
+    L.pair_tiles = 0;
+    for (int e = 0; e < E; ++e) {
+        L.R += group_rows[e];
+        L.pair_tiles += (group_rows[e] + 255) / 256;
+    }
     int64_t off = 256;  // header: status word
     auto take = [&](int64_t bytes) {
         const int64_t o = off;
@@ -594,6 +611,9 @@ MoeLayout moe_layout(const int64_t* group_rows, int E, int64_t K, int64_t N) {
     L.mtile_group = take(4 * (L.R / 128));
     L.group_row0 = take(8 * E);
     L.group_nrows = take(8 * E);
+    L.pair_row0 = take(8 * L.pair_tiles);
+    L.pair_group = take(4 * L.pair_tiles);
+    L.pair_rows = take(4 * L.pair_tiles);
     const int64_t R = L.R, EN = (int64_t)E * N;
     L.x_row = take(R * K / 2);
     L.x_row_sf = take((int64_t)nvfp4_scale_bytes(R, K));
@@ -637,7 +657,10 @@ int moe_grouped_begin(const int64_t* group_rows, int E, int64_t K, int64_t N, vo
     uint8_t* b = static_cast<uint8_t*>(ws);
     if (launch_group_tables(group_rows, E, reinterpret_cast<int32_t*>(b + L->mtile_group),
                             reinterpret_cast<int64_t*>(b + L->group_row0),
-                            reinterpret_cast<int64_t*>(b + L->group_nrows), st) != cudaSuccess)
+                            reinterpret_cast<int64_t*>(b + L->group_nrows), st,
+                            reinterpret_cast<int64_t*>(b + L->pair_row0),
+                            reinterpret_cast<int32_t*>(b + L->pair_group),
+                            reinterpret_cast<int32_t*>(b + L->pair_rows)) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
@@ -647,7 +670,8 @@ int run_quantize_grouped(const void* x, int64_t rows, int64_t cols, bool two_d, 
                          uint64_t seed, int col_rht, uint32_t mask, uint8_t* rd, uint8_t* rsf, float* rg,
                          uint8_t* cd, uint8_t* csf, float* cg, uint32_t* words, int* status,
                          const int32_t* row_group, const int64_t* row0, const int64_t* nrows,
-                         int64_t uniform, int sms, cudaStream_t st) {
+                         int64_t uniform, int sms, cudaStream_t st, const int32_t* row_src = nullptr,
+                         int64_t src_rows = 0) {
     QuantParams p;
     memset(&p, 0, sizeof p);
     p.x = static_cast<const uint16_t*>(x);
@@ -670,6 +694,8 @@ int run_quantize_grouped(const void* x, int64_t rows, int64_t cols, bool two_d, 
     p.group_row0 = row0;
     p.group_nrows = nrows;
     p.group_rows_uniform = uniform;
+    p.row_src = row_src;
+    p.src_rows = src_rows;
     cudaError_t e = launch_amax_grouped(p, sms, st);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     e = launch_quant_tile(p, two_d, st);
@@ -679,8 +705,15 @@ int run_quantize_grouped(const void* x, int64_t rows, int64_t cols, bool two_d, 
 int moe_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, const float* sa,
              const float* sb, float alpha, int64_t M, int64_t N, int64_t K, void* D, int* status, int mode,
              const int32_t* mtile_group, int64_t b_group_rows, int64_t b_group_k, int64_t Kb,
-             const int64_t* k_start, const int64_t* k_len, int groups, int sms, cudaStream_t st) {
+             const int64_t* k_start, const int64_t* k_len, int groups, int sms, cudaStream_t st,
+             const MoeLayout* L = nullptr, const uint8_t* ws = nullptr) {
     GemmParams g{};
+    if (mode == 1 && L && ws) {  // the 256-row group tiles of the two-SM kernel
+        g.pair_row0 = reinterpret_cast<const int64_t*>(ws + L->pair_row0);
+        g.pair_group = reinterpret_cast<const int32_t*>(ws + L->pair_group);
+        g.pair_rows = reinterpret_cast<const int32_t*>(ws + L->pair_rows);
+        g.num_pair_tiles = L->pair_tiles;
+    }
     g.A = A;
     g.sfA = sfA;
     g.B = B;
@@ -778,11 +811,17 @@ int nvfp4_moe_grouped_operand(void* ws, const int64_t* group_rows, int E, int64_
     return NVFP4_OK;
 }
 
-int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, const int64_t* group_rows,
-                            int E, int64_t K, int64_t N, const int8_t* rht_signs, void* ws,
-                            size_t ws_bytes, nvfp4_stream_t stream) {
-    if (!X_perm || !W || !Y_perm) return NVFP4_ERR_ARG;
-    if (!aligned(X_perm, 16) || !aligned(W, 16) || !aligned(Y_perm, 16)) return NVFP4_ERR_ALIGN;
+}  // extern "C"
+
+namespace {
+// Grouped fprop; X rows come from X_perm directly (row_src null) or from the token
+// rows row_src[r] of X (tokens rows).
+int moe_grouped_fprop(const void* X, const int32_t* row_src, int64_t tokens, const void* W, void* Y_perm,
+                      const int64_t* group_rows, int E, int64_t K, int64_t N, const int8_t* rht_signs,
+                      void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!X || !W || !Y_perm) return NVFP4_ERR_ARG;
+    if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y_perm, 16)) return NVFP4_ERR_ALIGN;
+    const void* X_perm = X;
     uint32_t mask = 0;
     if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -802,7 +841,7 @@ int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, con
     // X: rows (1x16 RNE) for fprop, RHT columns (1x16 RNE) for wgrad, per expert
     rc = run_quantize_grouped(X_perm, L.R, K, false, 0, 0, 0, 1, mask, b + L.x_row, b + L.x_row_sf,
                               (float*)(b + L.gx_row), b + L.x_col, b + L.x_col_sf, (float*)(b + L.gx_col),
-                              (uint32_t*)(b + L.words_x), status, mt, r0, nr, 0, sms, st);
+                              (uint32_t*)(b + L.words_x), status, mt, r0, nr, 0, sms, st, row_src, tokens);
     if (rc) return rc;
     // W [E][N][K] as [E*N][K]: 16x16 RNE, both orientations, per expert
     rc = run_quantize_grouped(W, (int64_t)E * N, K, true, 0, 0, 0, 0, 0, b + L.w_row, b + L.w_row_sf,
@@ -812,7 +851,27 @@ int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, con
     // Y rows of expert e = X rows of e times W_e^T
     return moe_gemm(b + L.x_row, b + L.x_row_sf, b + L.w_row, b + L.w_row_sf, (float*)(b + L.gx_row),
                     (float*)(b + L.gw_row), 1.0f, L.R, N, K, Y_perm, status, 1, mt, N, 0, 0, nullptr,
-                    nullptr, E, sms, st);
+                    nullptr, E, sms, st, &L, b);
+}
+}  // namespace
+
+extern "C" {
+
+int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, const int64_t* group_rows,
+                            int E, int64_t K, int64_t N, const int8_t* rht_signs, void* ws,
+                            size_t ws_bytes, nvfp4_stream_t stream) {
+    return moe_grouped_fprop(X_perm, nullptr, 0, W, Y_perm, group_rows, E, K, N, rht_signs, ws, ws_bytes,
+                             stream);
+}
+
+int nvfp4_moe_grouped_fprop_gather(const void* X_tok, const int32_t* row_src, int64_t tokens, const void* W,
+                                   void* Y_perm, const int64_t* group_rows, int E, int64_t K, int64_t N,
+                                   const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!row_src) return NVFP4_ERR_ARG;
+    if (tokens < 1 || tokens > (1ll << 31) - 1) return NVFP4_ERR_SHAPE;
+    if (!aligned(row_src, 4)) return NVFP4_ERR_ALIGN;
+    return moe_grouped_fprop(X_tok, row_src, tokens, W, Y_perm, group_rows, E, K, N, rht_signs, ws, ws_bytes,
+                             stream);
 }
 
 int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
@@ -844,7 +903,7 @@ int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* g
     // dX rows of expert e = dY rows of e times W_e (B = W^T [K][E*N], columns of e)
     return moe_gemm(b + L.dy_row, b + L.dy_row_sf, b + L.w_col, b + L.w_col_sf, (float*)(b + L.gdy_row),
                     (float*)(b + L.gw_col), 1.0f, L.R, K, N, dX_perm, status, 1, mt, 0, N, (int64_t)E * N,
-                    nullptr, nullptr, E, sms, st);
+                    nullptr, nullptr, E, sms, st, &L, b);
 }
 
 int nvfp4_moe_grouped_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,

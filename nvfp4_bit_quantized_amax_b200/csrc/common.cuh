@@ -20,6 +20,7 @@ namespace nvfp4 {
 // ---------------------------------------------------------------- status codes
 constexpr int kStatusNonFinite = -5;
 constexpr int kStatusTimeout = -6;
+constexpr int kStatusIndex = -9;
 
 // Record the first device-side error in a status word (0 = ok).
 __device__ __forceinline__ void set_status(int* status, int code) {
@@ -92,16 +93,6 @@ __device__ __forceinline__ TensorScale tensor_scale_from_amax(float amax) {
     return s;
 }
 
-// Block scale: code s = E4M3((amax_b / 6) * enc) and element multiplier
-// inv = 1 / (dec(s) * g) (0 when that product is 0, clamped to FLT_MAX).
-__device__ __forceinline__ void block_scale(float amax_b, const TensorScale& ts, uint32_t& s,
-                                            float& inv) {
-    float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), ts.enc);
-    s = e4m3_rn_satfinite(t);
-    float d = __fmul_rn(e4m3_to_f32(s), ts.g);
-    inv = (d == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, d), 3.402823466e38f);
-}
-
 // ---------------------------------------------------------------- Philox4x32-10
 // Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11): four
 // 32-bit counter words, two key words, 10 rounds of two 32x32->64 multiplies.
@@ -139,38 +130,6 @@ __device__ __forceinline__ Philox4 sr_draws8(const uint32_t (&rk)[20], uint32_t 
 __device__ __forceinline__ uint32_t draw16(const Philox4& p, int j) {
     const uint32_t w = (j >> 1) == 0 ? p.x : (j >> 1) == 1 ? p.y : (j >> 1) == 2 ? p.z : p.w;
     return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
-}
-
-// Stochastic rounding of eight values straight to packed E2M1 codes (element i
-// in bits [4i, 4i+4), sign bit of v kept, zero included).  Let a = min(|v|, 6)
-// and lo <= a <= hi the adjacent grid points; the rule rounds up iff
-// r < p * 2^16 with p = (a - lo) / (hi - lo) and r the 16-bit draw.  The map
-// c(a) = min(2a, a + 2, a / 2 + 4, 7) is affine between grid points and sends the
-// grid {0, .5, 1, 1.5, 2, 3, 4, 6} to the codes 0..7, so floor(c(a)) is the code
-// of lo and frac(c(a)) is p; hence code = floor(c) + [r < p * 2^16] =
-// (ceil(c * 2^16) + 65535 - r) >> 16, and grid points (p = 0) never move.  Each
-// line is one fp32 FMA rounded upward with 2^23 + offset * 2^16 + 65535 as its
-// addend (integers below 2^24, so the only rounding is the ceiling, and the
-// ceiling commutes with the minimum); the float's bits minus r then carry the
-// code in byte 2.  Byte permutes gather the codes and the sign bits.
-__device__ __forceinline__ uint32_t sr_e2m1x8(const float (&v)[8], const Philox4& rnd) {
-    uint32_t e[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float a = fabsf(v[i]);
-        const float t = fminf(fminf(__fmaf_ru(a, 131072.0f, 8454143.0f), __fmaf_ru(a, 65536.0f, 8585215.0f)),
-                              fminf(__fmaf_ru(a, 32768.0f, 8716287.0f), 8912895.0f));
-        e[i] = __float_as_uint(t) - draw16(rnd, i);
-    }
-    const uint32_t ce = __byte_perm(__byte_perm(e[0], e[2], 0x0062), __byte_perm(e[4], e[6], 0x0062), 0x5410);
-    const uint32_t co = __byte_perm(__byte_perm(e[1], e[3], 0x0062), __byte_perm(e[5], e[7], 0x0062), 0x5410);
-    const uint32_t se = __byte_perm(__byte_perm(__float_as_uint(v[0]), __float_as_uint(v[2]), 0x0073),
-                                    __byte_perm(__float_as_uint(v[4]), __float_as_uint(v[6]), 0x0073), 0x5410);
-    const uint32_t so = __byte_perm(__byte_perm(__float_as_uint(v[1]), __float_as_uint(v[3]), 0x0073),
-                                    __byte_perm(__float_as_uint(v[5]), __float_as_uint(v[7]), 0x0073), 0x5410);
-    const uint32_t even = ce | ((se >> 4) & 0x08080808u);  // element 2k in byte k, sign in bit 3
-    const uint32_t odd = co | ((so >> 4) & 0x08080808u);
-    return even + (odd << 4);
 }
 
 // ---------------------------------------------------------------- scale layout

@@ -65,13 +65,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity to complete: false once
+// `budget` clock cycles have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitCycles) return false;
+        if (clock64() - t0 > budget) return false;
     return true;
+}
+// Wait, at exit after a timeout, for this CTA's own asynchronous work (copies it
+// issued, MMAs it committed) to finish.  That work always completes, so the bound
+// is the long default, never the (possibly short) budget of the pipeline waits.
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+    (void)mbar_wait(bar, parity, kWaitCycles);
+}
+// After a timeout: spin ~`cycles` so that mbarrier arrivals already on their way
+// between the two CTAs of a pair land before either CTA can leave.
+__device__ __forceinline__ void settle(long long cycles) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < cycles) {
+    }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
@@ -231,6 +245,7 @@ struct __align__(1024) GemmSmem {
     uint64_t sf_full[4];   // scale region r written (4 scale-writer warps arrive)
     uint64_t acc_full;   // accumulator of the current tile complete (MMA commit)
     uint64_t acc_empty;  // accumulator drained by the 8 epilogue warps
+    uint64_t drain;      // after a timeout: every MMA issued so far complete
     uint32_t tmem_base;
 };
 
@@ -408,6 +423,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(smem_addr(&S.acc_full), 1);
         mbar_init(smem_addr(&S.acc_empty), 8);
+        mbar_init(smem_addr(&S.drain), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -423,18 +439,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    const long long budget = p.wait_cycles > 0 ? p.wait_cycles : kWaitCycles;
+    int64_t it = 0;  // producer thread: k-tiles whose copies it issued (all tiles)
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
-            int64_t it = 0;  // k-tiles issued by this CTA so far (all tiles)
             for (int64_t tile = blockIdx.x; tile < tiles && !*(volatile int*)&timed_out; tile += gridDim.x) {
                 const TileJob jb = tile_job<BN>(p, tile, tiles_n, tiles_per_group);
                 const int KTt = (int)((jb.k_len + 255) / 256);
                 for (int kt = 0; kt < KTt; ++kt, ++it) {
                     const int s = (int)(it % STAGES);
                     const uint32_t use = (uint32_t)(it / STAGES);
-                    if (it >= STAGES && !mbar_wait(smem_addr(&S.empty[s]), (use & 1u) ^ 1u)) {
+                    if (it >= STAGES && !mbar_wait(smem_addr(&S.empty[s]), (use & 1u) ^ 1u, budget)) {
                         timed_out = 1;
                         break;
                     }
@@ -457,11 +474,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                       p.sfB + ((jb.b_row / 128 + g) * katoms_b + jb.bk0 / kAtomK + katom) * 512,
                                       sf_bytes, fb);
                 }
-            }
-            if (*(volatile int*)&timed_out) {
-                // let copies already issued land before the CTA can exit
-                for (int64_t k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
-                    mbar_wait(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
             }
         }
         __syncwarp();
@@ -486,14 +498,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int KT = (int)((jb.k_len + 255) / 256);
                 const int KT_full = (int)(jb.k_len / 256);  // k-tiles with all four K = 64 steps
                 // the epilogue has drained the accumulator of the previous tile
-                if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u)) {
+                if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u, budget)) {
                     timed_out = 1;
                     break;
                 }
                 tc_fence_after();
                 bool bad = false;
                 for (int kt = 0; kt < KT; ++kt) {
-                    if (!mbar_wait(sf_full0 + 8u * s, ph)) {
+                    if (!mbar_wait(sf_full0 + 8u * s, ph, budget)) {
                         bad = true;
                         break;
                     }
@@ -546,7 +558,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // those MMAs completed before the producer could refill stage s (it
             // waited for their commit), so the arrival of k-tile it in stage s
             // also means that region r is free.
-            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u)) {
+            if (!mbar_wait(smem_addr(&S.full[s]), (uint32_t)(it / STAGES) & 1u, budget)) {
                 timed_out = 1;
                 stop = true;
                 break;
@@ -591,21 +603,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int gs = jb.group < 0 ? 0 : jb.group;
             if (p.scale_a) alpha = __fmul_rn(alpha, p.scale_a[gs]);
             if (p.scale_b) alpha = __fmul_rn(alpha, p.scale_b[gs]);
-            const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u);
+            const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u, budget);
             tc_fence_after();
             __syncwarp();
             if (!acc_ok) timed_out = 1;
+            // after a timeout the accumulator is neither read nor stored
             const bool bad = *(volatile int*)&timed_out != 0;
             const int64_t m_in = (jb.d_row - (jb.group >= 0 && p.group_mode == 2 ? (int64_t)jb.group * p.M : 0)) + 32 * q;
             epilogue_tile<BN>(lane_base, jb.d_row + 32 * q, jb.n0 + half * HC, p, alpha,
-                              !bad && m_in < p.M, jb.k_len == 0, smem_addr(&S.acc_empty), 0u,
+                              !bad && m_in < p.M, bad || jb.k_len == 0, smem_addr(&S.acc_empty), 0u,
                               smem_addr(S.dstage[warp - 6]), &tmD);
         }
         if (lane == 0) bulk_wait_all();  // every store of this warp has landed
         __syncwarp();
     }
     __syncthreads();
-    if (threadIdx.x == 0 && *(volatile int*)&timed_out) set_status(p.status, kStatusTimeout);
+    // Every role has left its loop.  After a timeout some consumers stopped early,
+    // so work this CTA issued may still be in flight: the producer waits for the
+    // copies of its last STAGES k-tiles (earlier ones were waited for before their
+    // stage was refilled), the MMA issuer commits once more and waits for that
+    // commit (it arrives when every MMA issued so far has completed).  Only then
+    // is TMEM freed and the CTA allowed to exit.
+    if (*(volatile int*)&timed_out) {
+        if (warp == 0 && lane == 0)
+            for (int64_t k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
+                mbar_wait_drain(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
+        if (warp == 1 && lane == 0) {
+            tc_commit(smem_addr(&S.drain));
+            mbar_wait_drain(smem_addr(&S.drain), 0u);
+        }
+        if (threadIdx.x == 0) set_status(p.status, kStatusTimeout);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -645,16 +673,6 @@ __device__ __forceinline__ void cluster_sync_all() {
 // tcgen05.wait::st, which has already completed the TMEM writes it announces.
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// Tile load into this CTA's shared memory whose bytes complete on a barrier of
-// either CTA of the pair (cluster address).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                                 uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(map), "r"(x), "r"(y), "r"(bar_cluster)
-        : "memory");
 }
 // Arrive (once the pair's MMAs issued so far complete) on the barrier at this
 // shared-memory offset in both CTAs.
@@ -710,18 +728,47 @@ struct __align__(1024) PairSmem {
     uint8_t dstage[8][32 * 32];              // per epilogue warp: 32 rows x 16 bf16, 32B-swizzled
     uint8_t sfa[STAGES][4 * 512];            // scales of this CTA's A rows
     uint8_t sfb[STAGES][2][4 * 512];         // scales of all 256 B rows of the tile
-    uint64_t full[STAGES];       // leader: A/B bytes of both CTAs landed
+    uint64_t full[STAGES];       // this CTA's A/B boxes landed
     uint64_t sf_loaded[STAGES];  // this CTA's scale atoms landed
     uint64_t empty[STAGES];      // stage free (leader's commit, both CTAs)
-    uint64_t sf_full[STAGES];    // leader: TMEM scales of both CTAs written (8 warps)
+    uint64_t sf_full[STAGES];    // leader: operands landed and TMEM scales written in both CTAs (8 warps)
     uint64_t acc_full;           // accumulator ready (leader's commit, both CTAs)
     uint64_t acc_empty;          // leader: accumulators of both CTAs drained (16 warps)
+    uint64_t drain;              // leader, after a timeout: every MMA issued so far complete
     uint32_t tmem_base;
 };
 
 constexpr int kPairThreads = 480;  // the warps of the one-SM kernel + a scale-copy producer
 
-template <int STAGES>
+// Operands and result of one 256 x 256 output tile of the pair kernel (the group
+// modes of GemmParams; mode 1 walks the 256-row tiles of every group, whose second
+// half may lie past the group's rows).
+struct PairJob {
+    int64_t m0;     // first A row of the tile (CTA rank r owns rows m0 + 128 r ..)
+    int64_t b_row;  // first B row of the tile (rank r loads rows b_row + 128 r ..)
+    int64_t n0;     // first D column
+    int64_t d_row;  // first D row
+    int64_t k0;     // first reduction element of A (B adds bk0)
+    int64_t bk0;    // extra reduction offset into B
+    int64_t k_len;  // reduction length
+    int64_t rows;   // rows from m0 that belong to the tile's problem (up to 256)
+    int group;      // -1 when not grouped
+};
+
+// MXFP4 (kMx): one pair MMA K step with UE8M0 scales over 32-element blocks.
+__device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X"
+        " [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+template <int STAGES, bool kMx>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
@@ -731,43 +778,78 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     constexpr int kUsed = BN + STAGES * kRegion;
     static_assert(kUsed <= 512, "TMEM holds 512 columns");
     constexpr uint32_t kAlloc = 512;
+    constexpr uint32_t kIdesc = kIdescPair | ((kMx ? 1u : 0u) << 23);  // UE8M0 scales for MX
+    constexpr int64_t kAtomK = kMx ? 128 : 64;  // reduction elements per scale atom
     extern __shared__ uint8_t smem_raw[];
     Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
-    const int64_t katoms = p.K / 64;
-    const int KT = (int)((p.K + 255) / 256);
-    const int64_t na_groups = (p.M + 127) / 128, nb_groups = (p.N + 127) / 128;
+    const int64_t katoms = (p.K + kAtomK - 1) / kAtomK;                       // per 128-row group of A
+    const int64_t katoms_b = ((p.Kb ? p.Kb : p.K) + kAtomK - 1) / kAtomK;     // ... of B
+    const int64_t b_rows_total = p.group_mode == 1 && p.b_group_rows ? p.b_group_rows * p.num_groups : p.N;
+    const int64_t na_groups = (p.M + 127) / 128, nb_groups = (b_rows_total + 127) / 128;
     const int64_t tiles_n = (p.N + BN - 1) / BN, tiles_m = (p.M + 255) / 256;
-    const int64_t tiles = tiles_m * tiles_n;
+    const int64_t tiles = p.group_mode == 1 ? p.num_pair_tiles * tiles_n
+                        : p.group_mode == 2 ? tiles_m * tiles_n * p.num_groups
+                                            : tiles_m * tiles_n;
     const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
-    // Tile order, for reuse of the operands in L2 (measured on the DRAM counters):
-    // if the smaller operand (codes + scales) fits in a quarter of L2 the clusters
-    // sweep along its dimension first, so it is re-read from L2 while the larger one
-    // streams from DRAM once; otherwise neither stays resident across waves and
-    // the tiles go in bands of kBand 256-row tile rows (M fastest inside a band),
-    // so each wave reads about as many A bands as B bands.
-    constexpr int64_t kBand = 8;
-    const int64_t small_bytes = (p.M < p.N ? p.M : p.N) * (p.K / 2 + p.K / 16);
-    const int order = small_bytes <= (int64_t(32) << 20) ? (p.M < p.N ? 1 : 0) : 2;
-    auto tile_origin = [&](int64_t pt, int64_t& m0, int64_t& n0) {
-        int64_t tm, tn;
-        if (order == 0) {  // N fastest
-            tm = pt / tiles_n;
-            tn = pt % tiles_n;
-        } else if (order == 1) {  // M fastest
-            tm = pt % tiles_m;
-            tn = pt / tiles_m;
-        } else {
-            const int64_t band = pt / (kBand * tiles_n), w = pt % (kBand * tiles_n);
-            const int64_t rows = tiles_m - band * kBand < kBand ? tiles_m - band * kBand : kBand;
-            tm = band * kBand + w % rows;
-            tn = w / rows;
+    // Tile order of the ungrouped problem (chosen on the host, pair_tile_order): 0 N
+    // fastest, 1 M fastest, 2 bands of tile_band 256-row tile rows with M fastest
+    // inside a band, 3 bands of tile_band tile columns with N fastest inside.
+    // Grouped problems go N fastest inside each 256-row tile of a group: the
+    // group's B and the tile's A rows are reused from L2.
+    const int order = p.tile_order;
+    const int64_t band_len = p.tile_band > 0 ? p.tile_band : 1;
+    auto job_of = [&](int64_t pt) {
+        PairJob j;
+        j.k0 = 0;
+        j.bk0 = 0;
+        j.k_len = p.K;
+        j.group = -1;
+        if (p.group_mode == 1) {
+            const int64_t t = pt / tiles_n;
+            j.n0 = (pt % tiles_n) * BN;
+            j.m0 = p.pair_row0[t];
+            j.group = p.pair_group[t];
+            j.rows = p.pair_rows[t];
+            j.b_row = (int64_t)j.group * p.b_group_rows + j.n0;
+            j.bk0 = (int64_t)j.group * p.b_group_k;
+            j.d_row = j.m0;
+            return j;
         }
-        m0 = tm * 256;
-        n0 = tn * BN;
+        int64_t tm, tn, t = pt;
+        if (p.group_mode == 2) {
+            j.group = (int)(pt / (tiles_m * tiles_n));
+            t = pt % (tiles_m * tiles_n);
+            tm = t / tiles_n;
+            tn = t % tiles_n;
+            j.k0 = p.k_start[j.group];
+            j.k_len = p.k_len[j.group];
+        } else if (order == 0) {  // N fastest
+            tm = t / tiles_n;
+            tn = t % tiles_n;
+        } else if (order == 1) {  // M fastest
+            tm = t % tiles_m;
+            tn = t / tiles_m;
+        } else if (order == 2) {  // bands of tile rows, M fastest inside a band
+            const int64_t band = t / (band_len * tiles_n), w = t % (band_len * tiles_n);
+            const int64_t rows = tiles_m - band * band_len < band_len ? tiles_m - band * band_len : band_len;
+            tm = band * band_len + w % rows;
+            tn = w / rows;
+        } else {  // bands of tile columns, N fastest inside a band
+            const int64_t band = t / (band_len * tiles_m), w = t % (band_len * tiles_m);
+            const int64_t cols = tiles_n - band * band_len < band_len ? tiles_n - band * band_len : band_len;
+            tn = band * band_len + w % cols;
+            tm = w / cols;
+        }
+        j.m0 = tm * 256;
+        j.n0 = tn * BN;
+        j.b_row = j.n0;
+        j.rows = p.M - j.m0 < 256 ? p.M - j.m0 : 256;
+        j.d_row = (j.group > 0 ? (int64_t)j.group * p.M : 0) + j.m0;
+        return j;
     };
 
     if (threadIdx.x == 0) {
@@ -779,6 +861,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         mbar_init(smem_addr(&S.acc_full), 1);
         mbar_init(smem_addr(&S.acc_empty), 16);
+        mbar_init(smem_addr(&S.drain), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -794,38 +877,35 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    const long long budget = p.wait_cycles > 0 ? p.wait_cycles : kWaitCycles;
+    int64_t issued_ab = 0;  // A/B producer thread: k-tiles whose boxes it issued
+    int64_t issued_sf = 0;  // scale producer thread: k-tiles whose atoms it issued
 
     if (warp == 0) {
         if (lane == 0) {
-            // ------------------------------------------------ A/B producer (both CTAs)
-            const uint32_t full_l0 = mapa_shared(smem_addr(&S.full[0]), 0);
+            // ------------------------------------------------ A/B producer (each CTA its own)
             const uint32_t empty0 = smem_addr(&S.empty[0]);
             uint32_t s = 0, ph = 0;
-            int64_t issued = 0;
             for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
-                int64_t m0, n0;
-            tile_origin(pt, m0, n0);
-                for (int kt = 0; kt < KT; ++kt, ++issued) {
-                    if (issued >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u)) {
+                const PairJob jb = job_of(pt);
+                const int KT = (int)((jb.k_len + 255) / 256);
+                for (int kt = 0; kt < KT; ++kt, ++issued_ab) {
+                    if (issued_ab >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u, budget)) {
                         timed_out = 1;
                         break;
                     }
-                    // A and B boxes of both CTAs (rows past M / N are zero-filled and count)
-                    if (leader) mbar_expect_tx(smem_addr(&S.full[s]), 4u * 128u * kBKBytes);
-                    tma_load_2d_pair(smem_addr(S.a[s]), &tmA, kt * kBKBytes, (int)(m0 + 128 * rank),
-                                     full_l0 + 8u * s);
-                    tma_load_2d_pair(smem_addr(S.b[s]), &tmB, kt * kBKBytes, (int)(n0 + 128 * rank),
-                                     full_l0 + 8u * s);
+                    // this CTA's A and B boxes (rows past the tensors are zero-filled and count)
+                    const uint32_t fb = smem_addr(&S.full[s]);
+                    mbar_expect_tx(fb, 2u * 128u * kBKBytes);
+                    tma_load_2d(smem_addr(S.a[s]), &tmA, (int)(jb.k0 / 2 + kt * kBKBytes),
+                                (int)(jb.m0 + 128 * rank), fb);
+                    tma_load_2d(smem_addr(S.b[s]), &tmB, (int)((jb.bk0 + jb.k0) / 2 + kt * kBKBytes),
+                                (int)(jb.b_row + 128 * rank), fb);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
-            }
-            if (*(volatile int*)&timed_out && leader) {
-                // let copies already issued land before the CTA can exit
-                for (int64_t k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k)
-                    mbar_wait(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
             }
         }
         __syncwarp();
@@ -836,39 +916,36 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             // the scale atoms have their own thread and barrier.
             const uint32_t sfl0 = smem_addr(&S.sf_loaded[0]), empty0 = smem_addr(&S.empty[0]);
             uint32_t s = 0, ph = 0;
-            int64_t issued = 0;
             for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
-                int64_t m0, n0;
-            tile_origin(pt, m0, n0);
-                const int64_t a_group = (m0 + 128 * rank) / 128;
-                for (int kt = 0; kt < KT; ++kt, ++issued) {
-                    if (issued >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u)) {
+                const PairJob jb = job_of(pt);
+                const int KT = (int)((jb.k_len + 255) / 256);
+                const int64_t a_group = (jb.m0 + 128 * rank) / 128;
+                for (int kt = 0; kt < KT; ++kt, ++issued_sf) {
+                    if (issued_sf >= STAGES && !mbar_wait(empty0 + 8u * s, ph ^ 1u, budget)) {
                         timed_out = 1;
                         break;
                     }
-                    const int64_t rem = (p.K - (int64_t)kt * 256) / kKStep;
-                    const uint32_t sf_bytes = (uint32_t)(rem < 4 ? rem : 4) * 512u;
+                    const int64_t rem = (jb.k_len - (int64_t)kt * 256) / kKStep;
+                    const int nks = rem < 4 ? (int)rem : 4;
+                    const uint32_t sf_bytes = (uint32_t)(kMx ? (nks + 1) / 2 : nks) * 512u;
+                    const int64_t katom = (jb.k0 + (int64_t)kt * 256) / kAtomK;  // first atom of the k-tile
                     uint32_t bytes = a_group < na_groups ? sf_bytes : 0u;
                     for (int g = 0; g < G; ++g)
-                        if (n0 / 128 + g < nb_groups) bytes += sf_bytes;
+                        if (jb.b_row / 128 + g < nb_groups) bytes += sf_bytes;
                     const uint32_t sb = sfl0 + 8u * s;
                     mbar_expect_tx(sb, bytes);
                     if (a_group < na_groups)
-                        bulk_load(smem_addr(S.sfa[s]), p.sfA + (a_group * katoms + (int64_t)kt * 4) * 512,
-                                  sf_bytes, sb);
+                        bulk_load(smem_addr(S.sfa[s]), p.sfA + (a_group * katoms + katom) * 512, sf_bytes, sb);
                     for (int g = 0; g < G; ++g)
-                        if (n0 / 128 + g < nb_groups)
+                        if (jb.b_row / 128 + g < nb_groups)
                             bulk_load(smem_addr(S.sfb[s][g]),
-                                      p.sfB + ((n0 / 128 + g) * katoms + (int64_t)kt * 4) * 512, sf_bytes, sb);
+                                      p.sfB + ((jb.b_row / 128 + g) * katoms_b + jb.bk0 / kAtomK + katom) * 512,
+                                      sf_bytes, sb);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
-            }
-            if (*(volatile int*)&timed_out) {
-                for (int64_t k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k)
-                    mbar_wait(sfl0 + 8u * (uint32_t)(k % STAGES), (uint32_t)(k / STAGES) & 1u);
             }
         }
         __syncwarp();
@@ -880,18 +957,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const uint64_t bdesc0 = operand_desc(smem_addr(S.b[0]));
             const uint32_t tsf0 = tmem + (uint32_t)BN;
             const uint32_t sf_full0 = smem_addr(&S.sf_full[0]), empty0 = smem_addr(&S.empty[0]);
-            const int KT_full = (int)(p.K / 256);
             uint32_t s = 0, ph = 0;
             uint32_t local = 0;
             for (int64_t pt = cid; pt < tiles; pt += ncl, ++local) {
-                if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u)) {
+                const PairJob jb = job_of(pt);
+                const int KT = (int)((jb.k_len + 255) / 256);
+                const int KT_full = (int)(jb.k_len / 256);  // k-tiles with all four K = 64 steps
+                if (local > 0 && !mbar_wait(smem_addr(&S.acc_empty), (local - 1) & 1u, budget)) {
                     timed_out = 1;
                     break;
                 }
                 tc_fence_after();
                 bool bad = false;
                 for (int kt = 0; kt < KT; ++kt) {
-                    if (!mbar_wait(sf_full0 + 8u * s, ph)) {
+                    if (!mbar_wait(sf_full0 + 8u * s, ph, budget)) {
                         bad = true;
                         break;
                     }
@@ -899,12 +978,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint64_t ad = adesc0 + kStep * s, bd = bdesc0 + kStep * s;
                     const uint32_t t_sfa = tsf0 + (uint32_t)kRegion * s;
                     const uint32_t t_sfb = t_sfa + kSfaCols;
-                    if (kt < KT_full) {
-                        tc_mma_nvf4_pair_x4(tmem, ad, bd, kIdescPair, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
-                    } else {  // K tail: 1 to 3 steps of 64
-                        const int nks = (int)((p.K - (int64_t)kt * 256) / kKStep);
+                    if (kMx) {
+                        // an atom serves two K = 64 steps: steps 0, 1 read atom 0 (scale
+                        // ids 0, 2), steps 2, 3 atom 1
+                        const int nks = kt < KT_full ? 4 : (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
                         for (int j = 0; j < nks; ++j)
-                            tc_mma_nvf4_pair(tmem, ad + 2u * j, bd + 2u * j, kIdescPair, t_sfa + 4 * j,
+                            tc_mma_mx_pair(tmem, ad + 2u * j, bd + 2u * j, mx_sf_id(kIdesc, 2u * (j & 1)),
+                                           t_sfa + 4 * (j >> 1), t_sfb + 4 * G * (j >> 1),
+                                           (kt > 0 || j > 0) ? 1u : 0u);
+                    } else if (kt < KT_full) {
+                        tc_mma_nvf4_pair_x4(tmem, ad, bd, kIdesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
+                    } else {  // K tail: 1 to 3 steps of 64
+                        const int nks = (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
+                        for (int j = 0; j < nks; ++j)
+                            tc_mma_nvf4_pair(tmem, ad + 2u * j, bd + 2u * j, kIdesc, t_sfa + 4 * j,
                                              t_sfb + 4 * G * j, (kt > 0 || j > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(empty0 + 8u * s);
@@ -925,21 +1012,23 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // ---------------------------------------------------- scale writers (warps 2-5, both CTAs)
         // Into this CTA's TMEM: the A scales of its own 128 rows and the B scales
         // of all 256 rows of the tile, in the layout of the one-SM kernel.  The
-        // leader's writers also wait for the A/B bytes of both CTAs, so the
-        // issuer needs only the sf_full barrier.  Region s was last read by the
+        // writers of each CTA also wait for that CTA's A/B boxes, so the leader's
+        // sf_full (all eight writer warps) means both CTAs' operands have landed and
+        // the issuer needs no other barrier.  Region s was last read by the
         // previous use of stage s, whose commit the producer waited for before
         // refilling the stage's scale atoms.
         const int q = warp & 3;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        const int64_t my_tiles = cid < tiles ? (tiles - cid + ncl - 1) / ncl : 0;
-        const int64_t total = my_tiles * KT;
         const uint32_t sfl0 = smem_addr(&S.sf_loaded[0]), full0 = smem_addr(&S.full[0]);
         const uint32_t sf_full_local0 = smem_addr(&S.sf_full[0]);
         const uint32_t sf_full_l0 = mapa_shared(sf_full_local0, 0);
         uint32_t s = 0, ph = 0;
-        for (int64_t it = 0; it < total; ++it) {
-            if (!mbar_wait(sfl0 + 8u * s, ph) || (leader && !mbar_wait(full0 + 8u * s, ph))) {
+        bool stop = false;
+        for (int64_t pt = cid; pt < tiles && !stop; pt += ncl)
+        for (int kt = (int)((job_of(pt).k_len + 255) / 256); kt > 0; --kt) {
+            if (!mbar_wait(sfl0 + 8u * s, ph, budget) || !mbar_wait(full0 + 8u * s, ph, budget)) {
                 timed_out = 1;
+                stop = true;
                 break;
             }
             tc_fence_after();
@@ -983,30 +1072,58 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const int half = (warp - 6) >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
         const uint32_t acc_empty_l = leader ? smem_addr(&S.acc_empty) : mapa_shared(smem_addr(&S.acc_empty), 0);
-        float alpha = p.alpha;
-        if (p.scale_a) alpha = __fmul_rn(alpha, *p.scale_a);
-        if (p.scale_b) alpha = __fmul_rn(alpha, *p.scale_b);
         uint32_t local = 0;
         for (int64_t pt = cid; pt < tiles; pt += ncl, ++local) {
             if (*(volatile int*)&timed_out) break;
-            int64_t m0, n0;
-            tile_origin(pt, m0, n0);
-            const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u);
+            const PairJob jb = job_of(pt);
+            float alpha = p.alpha;
+            const int gs = jb.group < 0 ? 0 : jb.group;
+            if (p.scale_a) alpha = __fmul_rn(alpha, p.scale_a[gs]);
+            if (p.scale_b) alpha = __fmul_rn(alpha, p.scale_b[gs]);
+            const bool acc_ok = mbar_wait(smem_addr(&S.acc_full), local & 1u, budget);
             tc_fence_after();
             __syncwarp();
             if (!acc_ok) timed_out = 1;
+            // after a timeout the accumulator is neither read nor stored
             const bool bad = *(volatile int*)&timed_out != 0;
-            epilogue_tile<BN>(lane_base, m0 + 128 * rank + 32 * q, n0 + half * HC, p, alpha,
-                              !bad && m0 + 128 * rank + 32 * q < p.M, false, acc_empty_l, leader ? 0u : 1u,
+            const int64_t r_in = 128 * rank + 32 * q;  // this warp's first row inside the tile
+            epilogue_tile<BN>(lane_base, jb.d_row + r_in, jb.n0 + half * HC, p, alpha, !bad && r_in < jb.rows,
+                              bad || jb.k_len == 0, acc_empty_l, leader ? 0u : 1u,
                               smem_addr(S.dstage[warp - 6]), &tmD);
         }
         if (lane == 0) bulk_wait_all();
         __syncwarp();
     }
     __syncthreads();
-    if (threadIdx.x == 0 && *(volatile int*)&timed_out) set_status(p.status, kStatusTimeout);
+    // Every role of this CTA has left its loop.  A CTA that saw no timeout has
+    // consumed every copy it issued (its scale writers waited for each stage) and,
+    // on the leader, its epilogue waited for the last MMA commit.  After a timeout
+    // each producer waits for the copies of its last STAGES k-tiles (they complete
+    // on this CTA's own barriers), the leader's issuer commits once more and waits
+    // for that commit (every MMA issued so far complete), and the CTA spins a few
+    // microseconds so that arrivals already sent to the other CTA land.  Only then
+    // do the two CTAs meet, free TMEM and exit.
+    if (*(volatile int*)&timed_out) {
+        if (warp == 0 && lane == 0)
+            for (int64_t k = (issued_ab > STAGES ? issued_ab - STAGES : 0); k < issued_ab; ++k)
+                mbar_wait_drain(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
+        if (warp == 14 && lane == 0)
+            for (int64_t k = (issued_sf > STAGES ? issued_sf - STAGES : 0); k < issued_sf; ++k)
+                mbar_wait_drain(smem_addr(&S.sf_loaded[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
+        if (warp == 1 && lane == 0 && leader) {
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             smem_addr(&S.drain))
+                         : "memory");
+            mbar_wait_drain(smem_addr(&S.drain), 0u);
+        }
+        if (threadIdx.x == 0) {
+            set_status(p.status, kStatusTimeout);
+            settle(20000);
+        }
+    }
+    __syncthreads();
     tc_fence_before();
-    cluster_sync_all();  // both CTAs done: no MMA, commit or remote arrive pending
+    cluster_sync_all();  // both CTAs done: no copy, MMA, commit or remote arrive pending
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAlloc)
@@ -1082,22 +1199,64 @@ static cudaError_t launch_gemm_cfg(const GemmParams& p, int sm_count, cudaStream
     return cudaGetLastError();
 }
 
-template <int STAGES>
-static cudaError_t launch_gemm_pair(const GemmParams& p, int sm_count, cudaStream_t st) {
+// Tile order of an ungrouped pair GEMM, for reuse of the operands in L2 (measured
+// on the DRAM counters).  If the smaller operand (codes + scales) fits in a quarter
+// of L2, the clusters sweep along its dimension first: it is re-read from L2 and
+// the larger one streams from DRAM once.  Otherwise the tiles go in bands: a band
+// of one operand (up to 40% of L2) stays resident while the other operand streams
+// past it once per band; the banded operand and the band width are the ones with
+// the fewer bytes read in total.
+static void pair_tile_order(GemmParams& g, int64_t l2_bytes) {
+    const int64_t row_bytes = g.K / 2 + g.K / 16 * (g.mx ? 1 : 2) / 2;
+    const int64_t a = g.M * row_bytes, b = g.N * row_bytes;
+    const int64_t tiles_m = (g.M + 255) / 256, tiles_n = (g.N + 255) / 256;
+    if ((a < b ? a : b) <= l2_bytes / 4) {
+        g.tile_order = g.M < g.N ? 1 : 0;
+        g.tile_band = 0;
+        return;
+    }
+    int64_t band = (l2_bytes * 2 / 5) / (256 * row_bytes);
+    if (band < 1) band = 1;
+    const int64_t bm = band < tiles_m ? band : tiles_m, bn = band < tiles_n ? band : tiles_n;
+    const int64_t reads_m = a + (tiles_m + bm - 1) / bm * b;  // A bands resident, B streamed per band
+    const int64_t reads_n = b + (tiles_n + bn - 1) / bn * a;
+    g.tile_order = reads_m <= reads_n ? 2 : 3;
+    g.tile_band = reads_m <= reads_n ? bm : bn;
+}
+
+template <int STAGES, bool kMx>
+static cudaError_t launch_gemm_pair(const GemmParams& params, int sm_count, cudaStream_t st) {
+    GemmParams p = params;
+    if (p.group_mode == 0) {
+        static int64_t l2 = 0;
+        if (l2 == 0) {
+            int dev = 0, v = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess || v <= 0)
+                v = 126 << 20;
+            l2 = v;
+        }
+        pair_tile_order(p, l2);
+    }
     CUtensorMap ma, mb, md;
-    if (!make_operand_map(&ma, p.A, p.M, p.K / 2, 128) || !make_operand_map(&mb, p.B, p.N, p.K / 2, 128))
+    const int64_t b_rows = p.group_mode == 1 && p.b_group_rows ? p.b_group_rows * p.num_groups : p.N;
+    const int64_t kb = p.Kb ? p.Kb : p.K;
+    if (!make_operand_map(&ma, p.A, p.M, p.K / 2, 128) || !make_operand_map(&mb, p.B, b_rows, kb / 2, 128))
         return cudaErrorInvalidValue;
     memset(&md, 0, sizeof(md));
-    if (p.D_bf16 && !make_output_map(&md, p.D_bf16, p.M, p.N)) return cudaErrorInvalidValue;
+    const int64_t d_rows = p.group_mode == 2 ? p.M * p.num_groups : p.M;
+    if (p.D_bf16 && !make_output_map(&md, p.D_bf16, d_rows, p.N)) return cudaErrorInvalidValue;
     const size_t smem = sizeof(PairSmem<STAGES>) + 1024;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<STAGES>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<STAGES, kMx>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const int64_t tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
+    const int64_t tiles_n = (p.N + 255) / 256, tiles_m = (p.M + 255) / 256;
+    const int64_t tiles = p.group_mode == 1 ? p.num_pair_tiles * tiles_n
+                        : p.group_mode == 2 ? tiles_m * tiles_n * p.num_groups
+                                            : tiles_m * tiles_n;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kPairThreads);
     cfg.dynamicSmemBytes = smem;
@@ -1114,16 +1273,21 @@ static cudaError_t launch_gemm_pair(const GemmParams& p, int sm_count, cudaStrea
     static int resident = 0;
     if (resident == 0) {
         cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
-        if (cudaOccupancyMaxActiveClusters(&resident, gemm_nvf4_pair_kernel<STAGES>, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&resident, gemm_nvf4_pair_kernel<STAGES, kMx>, &cfg) != cudaSuccess ||
             resident < 1)
             resident = sm_count / 2;
     }
-    cfg.gridDim = dim3((unsigned)(2 * (tiles < resident ? tiles : resident)));
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<STAGES>, ma, mb, md, p);
+    const int64_t clusters = tiles < resident ? (tiles > 0 ? tiles : 1) : resident;
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<STAGES, kMx>, ma, mb, md, p);
 }
 
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
-    if (!p.mx && p.group_mode == 0 && p.M > 128 && sm_count >= 2) return launch_gemm_pair<5>(p, sm_count, st);
+    // two-SM pairs for every problem taller than one 128-row tile, and for the grouped
+    // problems (mode 1 needs its table of 256-row group tiles)
+    const bool pair = sm_count >= 2 && (p.group_mode == 0 ? p.M > 128
+                                        : p.group_mode == 2 || p.pair_row0 != nullptr);
+    if (pair) return p.mx ? launch_gemm_pair<5, true>(p, sm_count, st) : launch_gemm_pair<5, false>(p, sm_count, st);
     if (p.mx) return launch_gemm_cfg<256, 4, true>(p, sm_count, st);
     return launch_gemm_cfg<256, 4, false>(p, sm_count, st);
 }

@@ -6,6 +6,21 @@
 
 namespace nvfp4 {
 
+// Sign flips of the 16 rotation inputs, as constants the kernels read from their
+// parameters: pair[i] flips both bf16 of a packed word (0x80008000 or 0), lo[i] is
+// the same flip for the low value once shifted into an fp32 (0x80000000 or 0).
+struct RhtFlips {
+    uint32_t pair[16];
+    uint32_t lo[16];
+};
+inline void rht_flips(uint32_t sign_mask, RhtFlips& f) {
+    for (int i = 0; i < 16; ++i) {
+        const bool neg = (sign_mask >> i) & 1u;
+        f.pair[i] = neg ? 0x80008000u : 0u;
+        f.lo[i] = neg ? 0x80000000u : 0u;
+    }
+}
+
 // One quantize pass.  Outputs with a null data pointer are not written.
 struct QuantParams {
     const uint16_t* x;  // bf16 [rows][cols]
@@ -22,6 +37,7 @@ struct QuantParams {
     int row_sr, col_sr, col_rht;
     int row_rht;         // rotate the row orientation too (tile kernel, ungrouped, 1x16)
     uint32_t sign_mask;  // bit i set: rotation sign i is -1
+    RhtFlips flips;      // the same signs as flip constants (filled by the launchers)
     uint32_t rk[20];     // Philox4x32-10 round keys of `seed` (filled by the launchers)
     // Grouped tensors (mixture of experts): row r belongs to group
     // row_group[r / 128] (table) or r / group_rows_uniform; group g owns rows
@@ -32,6 +48,11 @@ struct QuantParams {
     const int64_t* group_row0;
     const int64_t* group_nrows;
     int64_t group_rows_uniform;
+    // Gathered input (nullable): row r of the quantized tensor is row row_src[r] of
+    // x, which has src_rows rows; a negative entry reads as a zero row, one past the
+    // source records kStatusIndex and also reads as zeros.
+    const int32_t* row_src;
+    int64_t src_rows;
 };
 
 // Rows one launch of the quantize tile kernel covers: 64-row tiles along the
@@ -43,10 +64,12 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
 
 // Group tables of a grouped tensor from its group sizes (host array of E <=
 // kMaxGroups entries, multiples of 128): group of every 128-row block, first row
-// and rows of every group, written on `st`.
+// and rows of every group, and (when pair_row0 is not null) the 256-row tiles of
+// every group in order (first row, group, rows inside the group), written on `st`.
 constexpr int kMaxGroups = 1024;
 cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block_group, int64_t* row0,
-                                int64_t* nrows, cudaStream_t st);
+                                int64_t* nrows, cudaStream_t st, int64_t* pair_row0 = nullptr,
+                                int32_t* pair_group = nullptr, int32_t* pair_rows = nullptr);
 
 // Philox4x32-10 key schedule of a 64-bit seed: round r uses
 // (lo(seed) + r * 0x9E3779B9, hi(seed) + r * 0xBB67AE85), mod 2^32.
@@ -104,7 +127,19 @@ struct GemmParams {
     const int64_t* k_start;
     const int64_t* k_len;
     int num_groups;
+    // Mode 1 on the two-SM kernel: the 256-row tiles of every group (first row,
+    // group, rows that belong to the group: 128 or 256), num_pair_tiles entries.
+    const int64_t* pair_row0;
+    const int32_t* pair_group;
+    const int32_t* pair_rows;
+    int64_t num_pair_tiles;
     int mx;  // MXFP4 operands: UE8M0 scales over 32-element blocks, no tensor scales
+    // Ungrouped two-SM problems: tile order and band width (filled by the launcher).
+    int tile_order;
+    int64_t tile_band;
+    // Clock cycles a pipeline wait may last before the kernel gives up and records
+    // NVFP4_ERR_TIMEOUT (0: the default, 2^31, about a second).
+    long long wait_cycles;
 };
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st);
 

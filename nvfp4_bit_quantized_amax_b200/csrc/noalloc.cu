@@ -13,6 +13,7 @@
 // loads this library until the process exits.  All calls share it: the call
 // clears the words that must start at zero on its stream before using them, and
 // calls that overlap on the GPU (other streams, other host threads) race on it.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,13 +38,48 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 uint32_t* g_scratch_ptr[kMaxDevices] = {};
 int g_sm_count[kMaxDevices] = {};
+unsigned long long g_ctx_id[kMaxDevices] = {};  // context the cached address belongs to
 
-// Once per device, with that device current: resolve the array's device address.
+// Unique id of the calling thread's current context (0 when it cannot be read).
+// A device's primary context gets a new id when it is re-created, e.g. after
+// cudaDeviceReset, and a module's symbol address is only valid in the context it
+// was resolved in.
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrent)(CUcontext*);
+    typedef CUresult (*GetId)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrent>(a);
+            get_id = reinterpret_cast<GetId>(b);
+        }
+        looked_up = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Once per device (and again if that device's context was re-created), with the
+// device current: resolve the array's device address.
 int scratch_for_current_device(uint32_t** ptr, int* sms) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
+    // 0 when no context is current on this thread yet (the runtime binds the
+    // primary context at its first call that needs one, cudaGetSymbolAddress below)
+    const unsigned long long ctx = current_context_id();
+    if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_ctx_id[dev]) {
         int major = 0, count = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -54,6 +90,7 @@ int scratch_for_current_device(uint32_t** ptr, int* sms) {
             return NVFP4_ERR_CUDA;
         g_sm_count[dev] = count;
         g_scratch_ptr[dev] = static_cast<uint32_t*>(p);
+        g_ctx_id[dev] = current_context_id();
     }
     *ptr = g_scratch_ptr[dev];
     *sms = g_sm_count[dev];

@@ -18,11 +18,97 @@
 namespace nvfp4 {
 
 // ============================================================================
-// 16-point Hadamard butterfly in fp64.  The Sylvester H16 is symmetric, so
-// x . diag(s) . H16 == H16 . (s * x); four radix-2 stages compute it.  Inputs
-// are bf16 values (8 significant bits), so every partial sum is exact while the
-// chunk's exponents span at most 41 binades; the fp32 rounding of the result is
-// then the correctly rounded value of the exact sum.
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): element 0 in the low word.  Every
+// operation rounds to nearest even and keeps subnormals, like its scalar form.
+// ============================================================================
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pk(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ f32x2 pk_bits(uint32_t lo, uint32_t hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpk(f32x2 v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// a * b + c rounded once, upward (toward +inf)
+__device__ __forceinline__ f32x2 fma2_ru(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rp.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// Two 16-bit lanes: signed minimum, unsigned maximum.
+__device__ __forceinline__ uint32_t vmin_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// 32-byte streaming load (16 bf16) of data read once; `p` 32-byte aligned.
+__device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&r)[8]) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+// Sixteen bf16 at p (16-byte aligned): one 32-byte load when p is 32-byte aligned,
+// else two 16-byte loads.
+__device__ __forceinline__ void ld_block16(const uint16_t* p, bool al32, uint32_t (&r)[8]) {
+    if (al32) {
+        ld_stream_v8(p, r);
+    } else {
+        const uint4 a = ld_stream_v4(p), b = ld_stream_v4(p + 8);
+        r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+        r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
+    }
+}
+
+// ============================================================================
+// 16-point random Hadamard transform of bf16 inputs, exactly rounded.
+//
+// The quantizer sees y_j = RN32(sum_i s_i x_i H16[i][j]): the fp32 rounding of the
+// exact sum (Sylvester H16, unnormalised; x . diag(s) . H16 == H16 . (s * x) since
+// H16 is symmetric).  Four radix-2 butterfly stages compute it; after three stages
+// every value is a signed sum of at most 8 inputs, the fourth adds two of those.
+// A bf16 input with biased exponent E has 8 significant bits, so it is a multiple
+// of 2^(max(E,1) - 134) below 2^(E - 126).  When the chunk's nonzero inputs satisfy
+// E_max - max(E_min, 1) <= 13 (and E_max <= 251, no overflow), a sum of up to 8 of
+// them is a multiple of 2^(max(E_min,1) - 134) below 8 * 2^(E_max - 126), i.e. below
+// 2^24 such units: exactly representable in fp32.  The first three fp32 stages are
+// then exact and the last is one correctly rounded addition of two exact values,
+// which is RN32 of the exact sum.  Other chunks (rare: a tiny value beside a large
+// one, or Inf / NaN) take an fp64 butterfly, exact while the span is at most 41
+// binades; its fp32 rounding is the same RN32 of the exact sum.
 // ============================================================================
 __device__ __forceinline__ void fwht16(double (&y)[16]) {
 #pragma unroll
@@ -38,10 +124,156 @@ __device__ __forceinline__ void fwht16(double (&y)[16]) {
     }
 }
 
+// bf16 bit pattern with its sign flipped where the rotation sign is -1.
+__device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t flip) {
+    return (double)__uint_as_float((bits16 ^ (flip << 15)) << 16);
+}
+
+// The exponent-span test above for one 16-bit lane of the chunk statistics: with
+// v = |x| + 0x7FFF per bf16 (0x7FFF for a zero, >= 0x8000 otherwise), vmx is the
+// unsigned maximum of v and vmn its signed minimum (the smallest nonzero |x|).
+__device__ __forceinline__ bool span_ok(uint32_t vmx, uint32_t vmn) {
+    if (vmx == 0x7FFFu) return true;  // all inputs zero
+    const int emax = (int)((vmx - 0x7FFFu) >> 7);
+    const int emin = (int)((vmn - 0x7FFFu) >> 7);
+    return emax <= 251 && emax - max(emin, 1) <= 13;
+}
+
+// Chunk statistics of packed bf16 words (two independent lanes): per 16-bit lane,
+// the unsigned maximum and signed minimum of v = |x| + 0x7FFF (no carry between the
+// lanes: |x| <= 0x7FFF).
+template <int N>
+__device__ __forceinline__ void chunk_stats(const uint32_t (&w)[N], uint32_t& vmx, uint32_t& vmn) {
+    vmx = 0u;
+    vmn = 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const uint32_t v = (w[i] & 0x7FFF7FFFu) + 0x7FFF7FFFu;
+        vmx = vmax_u16x2(vmx, v);
+        vmn = vmin_s16x2(vmn, v);
+    }
+}
+
+// fp64 transform of one column of a column pair (half 0: low values, 1: high).
+__device__ __forceinline__ void rht16_col_f64(const uint32_t (&w)[16], int half, uint32_t sign_mask,
+                                              float (&y)[16]) {
+    double d[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        d[i] = bf16_signed_to_f64(half ? (w[i] >> 16) : (w[i] & 0xFFFFu), (sign_mask >> i) & 1u);
+    fwht16(d);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __double2float_rn(d[i]);
+}
+
+// Rotation of a column pair: w[i] holds row i of two adjacent columns (the first in
+// the low half).  y0 / y1 receive the transforms of the two columns.
+__device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFlips& f, uint32_t sign_mask,
+                                           float (&y0)[16], float (&y1)[16]) {
+    uint32_t vmx, vmn;
+    chunk_stats<16>(w, vmx, vmn);
+    if (span_ok(vmx & 0xFFFFu, vmn & 0xFFFFu) && span_ok(vmx >> 16, vmn >> 16)) {
+        f32x2 x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = pk_bits(w[i] * 65536u + f.lo[i], (w[i] ^ f.pair[i]) & 0xFFFF0000u);
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if ((i & h) == 0) {
+                    const f32x2 a = x[i], b = x[i + h];
+                    x[i] = add2(a, b);
+                    x[i + h] = sub2(a, b);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) unpk(x[i], y0[i], y1[i]);
+    } else {
+        rht16_col_f64(w, 0, sign_mask, y0);
+        rht16_col_f64(w, 1, sign_mask, y1);
+    }
+}
+
+// max_j |y_j| over both columns of a column pair.  On the fp32 path the last stage
+// is not formed: max(|RN(a+b)|, |RN(a-b)|) = RN(|a| + |b|) exactly (RN is monotone
+// and odd, and max(|a+b|, |a-b|) = |a| + |b|).
+__device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], const RhtFlips& f,
+                                                   uint32_t sign_mask, uint32_t vmx, uint32_t vmn) {
+    float m = 0.0f;
+    if (span_ok(vmx & 0xFFFFu, vmn & 0xFFFFu) && span_ok(vmx >> 16, vmn >> 16)) {
+        f32x2 x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = pk_bits(w[i] * 65536u + f.lo[i], (w[i] ^ f.pair[i]) & 0xFFFF0000u);
+#pragma unroll
+        for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if ((i & h) == 0) {
+                    const f32x2 a = x[i], b = x[i + h];
+                    x[i] = add2(a, b);
+                    x[i + h] = sub2(a, b);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a0, a1, b0, b1;
+            unpk(x[j], a0, a1);
+            unpk(x[j + 8], b0, b1);
+            m = fmaxf(m, fmaxf(fabsf(a0) + fabsf(b0), fabsf(a1) + fabsf(b1)));
+        }
+    } else {
+        float y[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            rht16_col_f64(w, half, sign_mask, y);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(y[i]));
+        }
+    }
+    return m;
+}
+
+// Rotation of one row block held by one thread: w[k] holds elements 2k, 2k+1 of the
+// block (16 values).  Scalar fp32 butterfly under the same span test, else fp64.
+__device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_mask, float (&y)[16]) {
+    uint32_t vmx, vmn;
+    chunk_stats<8>(w, vmx, vmn);
+    const uint32_t mx = max(vmx & 0xFFFFu, vmx >> 16);
+    const uint32_t mn = (uint32_t)(uint16_t)min((int16_t)(vmn & 0xFFFFu), (int16_t)(vmn >> 16));
+    if (span_ok(mx, mn)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t b = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
+            y[i] = __uint_as_float((b ^ (((sign_mask >> i) & 1u) << 15)) << 16);
+        }
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if ((i & h) == 0) {
+                    const float a = y[i], b = y[i + h];
+                    y[i] = __fadd_rn(a, b);
+                    y[i + h] = __fsub_rn(a, b);
+                }
+            }
+        }
+    } else {
+        double d[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            d[i] = bf16_signed_to_f64((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu), (sign_mask >> i) & 1u);
+        fwht16(d);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __double2float_rn(d[i]);
+    }
+}
+
 // 16-point rotation of a row chunk held by a lane pair (even lane: elements 0-7,
 // odd lane: 8-15; both lanes of every pair call this together): three butterfly
-// stages inside the lane, the last across the pair.  In fp64, exact like fwht16;
-// y receives the lane's eight outputs.
+// stages inside the lane, the last across the pair, in fp64 (exact like fwht16).
+// Used by the amax pass of the rotated row orientation.
 __device__ __forceinline__ void rht16_lane_pair(const uint4& w, uint32_t sign_mask, int lane,
                                                 double (&y)[8]) {
     const int base = (lane & 1) * 8;
@@ -69,11 +301,6 @@ __device__ __forceinline__ void rht16_lane_pair(const uint4& w, uint32_t sign_ma
     }
 }
 
-// bf16 bit pattern with its sign flipped where the rotation sign is -1.
-__device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t flip) {
-    return (double)__uint_as_float((bits16 ^ (flip << 15)) << 16);
-}
-
 // ============================================================================
 // amax prepass.  One warp handles a 16-row x 256-column unit, each lane 16 rows
 // x 8 columns (sixteen 16-byte loads).  Word 0 receives max |x| (fp32 bits of a
@@ -84,31 +311,48 @@ __device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t f
 // words[2g] and words[2g+1]; each unit is folded into them by the warp.
 // kRowRht: word 0 (or 2g) is max |RHT16 along the rows| instead of max |x| (the
 // row orientation is rotated); a non-finite input still makes it non-finite.
-template <bool kColRht, bool kGrouped, bool kRowRht>
-__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                   int64_t cols, uint32_t sign_mask,
+// row_src (nullable): row r of the tensor is row row_src[r] of x (see QuantParams).
+template <bool kColRht, bool kRowRht>
+constexpr int amax_min_blocks() {
+    return (kColRht && kRowRht) ? 1 : 2;  // both rotations: registers for one CTA per SM
+}
+template <bool kColRht, bool kGrouped, bool kRowRht, bool kGather>
+__global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                   int64_t cols, uint32_t sign_mask, const RhtFlips flips,
                                                    uint32_t* __restrict__ words,
                                                    const int32_t* __restrict__ row_group,
-                                                   int64_t group_rows_uniform) {
+                                                   int64_t group_rows_uniform,
+                                                   const int32_t* __restrict__ row_src, int64_t src_rows,
+                                                   int* status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t col_units = (cols + 255) >> 8;
     const int64_t units = ((rows + 15) >> 4) * col_units;
     uint32_t m_row = 0;   // two packed 16-bit magnitudes
-    double m_col = 0.0;
+    float m_col = 0.0f;
     double m_rrht = 0.0;  // kRowRht: max |rotated row|
     for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += (int64_t)gridDim.x * 8) {
         const int64_t r0 = (u / col_units) * 16;
         const int64_t c0 = (u % col_units) * 256 + lane * 8;
         if (kGrouped) {
             m_row = 0;
-            m_col = 0.0;
+            m_col = 0.0f;
         }
         if (kRowRht || c0 < cols) {
         uint4 v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            v[i] = (c0 < cols && r0 + i < rows) ? ld_stream_v4(x + (r0 + i) * cols + c0)
-                                                : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 16; ++i) {
+            bool in = c0 < cols && r0 + i < rows;
+            int64_t sr = r0 + i;
+            if (kGather && in) {
+                sr = __ldg(row_src + r0 + i);
+                if (sr >= src_rows) {
+                    if (lane == 0) set_status(status, kStatusIndex);
+                    in = false;
+                }
+                in = in && sr >= 0;
+            }
+            v[i] = in ? ld_stream_v4(x + sr * cols + c0) : make_uint4(0, 0, 0, 0);
+        }
         if (kRowRht) {  // every lane takes part (zeros past the columns)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -118,34 +362,33 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
                 for (int k = 0; k < 8; ++k) m_rrht = fmax(m_rrht, fabs(y[k]));
             }
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            m_row = __vmaxu2(m_row, v[i].x & 0x7FFF7FFFu);
-            m_row = __vmaxu2(m_row, v[i].y & 0x7FFF7FFFu);
-            m_row = __vmaxu2(m_row, v[i].z & 0x7FFF7FFFu);
-            m_row = __vmaxu2(m_row, v[i].w & 0x7FFF7FFFu);
-        }
         if (kColRht) {
+            // column pairs (2c, 2c+1) of the lane's 8 columns: the chunk statistics
+            // give max |x| too
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                double y[16];
+            for (int c = 0; c < 4; ++c) {
+                uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = (c >> 1) == 0 ? v[i].x : (c >> 1) == 1 ? v[i].y
-                                     : (c >> 1) == 2 ? v[i].z : v[i].w;
-                    const uint32_t b = (c & 1) ? (w >> 16) : (w & 0xFFFFu);
-                    y[i] = bf16_signed_to_f64(b, (sign_mask >> i) & 1u);
-                }
-                fwht16(y);
+                for (int i = 0; i < 16; ++i) w[i] = c == 0 ? v[i].x : c == 1 ? v[i].y : c == 2 ? v[i].z : v[i].w;
+                uint32_t vmx, vmn;
+                chunk_stats<16>(w, vmx, vmn);
+                m_row = vmax_u16x2(m_row, vmx - 0x7FFF7FFFu);
+                m_col = fmaxf(m_col, rht16_pair_absmax(w, flips, sign_mask, vmx, vmn));
+            }
+        } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) m_col = fmax(m_col, fabs(y[i]));
+            for (int i = 0; i < 16; ++i) {
+                m_row = __vmaxu2(m_row, v[i].x & 0x7FFF7FFFu);
+                m_row = __vmaxu2(m_row, v[i].y & 0x7FFF7FFFu);
+                m_row = __vmaxu2(m_row, v[i].z & 0x7FFF7FFFu);
+                m_row = __vmaxu2(m_row, v[i].w & 0x7FFF7FFFu);
             }
         }
         }
         if (kGrouped) {
             const int64_t g = row_group ? (int64_t)row_group[r0 >> 7] : r0 / group_rows_uniform;
             uint32_t ur = max(m_row & 0xFFFFu, m_row >> 16) << 16;
-            uint32_t uc = kColRht ? __float_as_uint(__double2float_rn(m_col)) : 0u;
+            uint32_t uc = kColRht ? __float_as_uint(m_col) : 0u;
             ur = __reduce_max_sync(0xFFFFFFFFu, ur);
             uc = __reduce_max_sync(0xFFFFFFFFu, uc);
             if (lane == 0) {
@@ -157,7 +400,7 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     if (kGrouped) return;
     uint32_t a_row = max(m_row & 0xFFFFu, m_row >> 16) << 16;
     if (kRowRht && a_row < 0x7F800000u) a_row = __float_as_uint(__double2float_rn(m_rrht));
-    uint32_t a_col = kColRht ? __float_as_uint(__double2float_rn(m_col)) : 0u;
+    uint32_t a_col = kColRht ? __float_as_uint(m_col) : 0u;
     a_row = __reduce_max_sync(0xFFFFFFFFu, a_row);
     a_col = __reduce_max_sync(0xFFFFFFFFu, a_col);
     __shared__ uint32_t red[2][8];
@@ -183,21 +426,78 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
 // ============================================================================
 __device__ __forceinline__ bool finite_bits(uint32_t b) { return (b & 0x7FFFFFFFu) < 0x7F800000u; }
 
-// Eight values -> packed codes with RNE or SR (element index e0 .. e0+7 of the
-// quantized tensor, e0 % 8 == 0); element i lands in bits [4i, 4i+4).
-__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float inv, bool sr,
-                                            const uint32_t (&rk)[20], uint32_t stream,
-                                            uint64_t e0) {
-    if (!sr) {
-        float q[8];
+// Element multiplier of E4M3 block-scale code s: 1 / (dec(s) * g), 0 when that
+// product is 0, clamped to FLT_MAX (the op order of block_scale).  A CTA fills a
+// 256-entry table once per tensor scale and looks the multiplier up per block.
+__device__ __forceinline__ float block_inv_of_code(uint32_t s, float g) {
+    const float d = __fmul_rn(e4m3_to_f32(s), g);
+    return (d == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, d), 3.402823466e38f);
+}
+// E4M3 code of a block with amax_b: RNE_satfinite((amax_b / 6) * enc).
+__device__ __forceinline__ uint32_t block_code(float amax_b, const TensorScale& ts) {
+    return e4m3_rn_satfinite(__fmul_rn(__fdiv_rn(amax_b, 6.0f), ts.enc));
+}
+
+// Stochastic rounding of eight values straight to packed E2M1 codes (element i in
+// bits [4i, 4i+4), the sign bit of y kept, zero included), the magnitude being
+// a = min(|y| * inv, 6).  With lo <= a <= hi the adjacent grid points the rule rounds
+// up iff r < p * 2^16, p = (a - lo) / (hi - lo), r the element's 16-bit draw.  The map
+// c(a) = min(2a, a + 2, a / 2 + 4) is affine between grid points and sends the grid
+// {0, .5, 1, 1.5, 2, 3, 4, 6} to the codes 0..7, so floor(c(a)) is the code of lo
+// and frac(c(a)) is p; hence code = floor(c) + [r < p * 2^16] =
+// (ceil(c * 2^16) + 65535 - r) >> 16, and grid points (p = 0) never move.  Each
+// line is an fp32 FMA rounded upward with 2^23 + offset * 2^16 + 65535 as its addend
+// (integers below 2^24, so the only rounding is the ceiling, which commutes with
+// the minimum), two elements per packed FMA; the float's bits minus r then carry
+// the code in byte 2.  Byte permutes gather the codes and the sign bits.
+__device__ __forceinline__ uint32_t sr_codes8(const float (&y)[8], float inv, const Philox4& rnd) {
+    const f32x2 k1 = pk(131072.0f, 131072.0f), k2 = pk(65536.0f, 65536.0f), k3 = pk(32768.0f, 32768.0f);
+    const f32x2 c1 = pk(8454143.0f, 8454143.0f), c2 = pk(8585215.0f, 8585215.0f), c3 = pk(8716287.0f, 8716287.0f);
+    uint32_t e[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
-        return e2m1x8_rn(q);
+    for (int m = 0; m < 4; ++m) {
+        const f32x2 a = pk(fminf(__fmul_rn(fabsf(y[2 * m]), inv), 6.0f),
+                           fminf(__fmul_rn(fabsf(y[2 * m + 1]), inv), 6.0f));
+        float t1l, t1h, t2l, t2h, t3l, t3h;
+        unpk(fma2_ru(a, k1, c1), t1l, t1h);
+        unpk(fma2_ru(a, k2, c2), t2l, t2h);
+        unpk(fma2_ru(a, k3, c3), t3l, t3h);
+        e[2 * m] = __float_as_uint(fmin3(t1l, t2l, t3l)) - draw16(rnd, 2 * m);
+        e[2 * m + 1] = __float_as_uint(fmin3(t1h, t2h, t3h)) - draw16(rnd, 2 * m + 1);
     }
+    const uint32_t ce = __byte_perm(__byte_perm(e[0], e[2], 0x0062), __byte_perm(e[4], e[6], 0x0062), 0x5410);
+    const uint32_t co = __byte_perm(__byte_perm(e[1], e[3], 0x0062), __byte_perm(e[5], e[7], 0x0062), 0x5410);
+    const uint32_t se = __byte_perm(__byte_perm(__float_as_uint(y[0]), __float_as_uint(y[2]), 0x0073),
+                                    __byte_perm(__float_as_uint(y[4]), __float_as_uint(y[6]), 0x0073), 0x5410);
+    const uint32_t so = __byte_perm(__byte_perm(__float_as_uint(y[1]), __float_as_uint(y[3]), 0x0073),
+                                    __byte_perm(__float_as_uint(y[5]), __float_as_uint(y[7]), 0x0073), 0x5410);
+    const uint32_t even = ce | ((se >> 4) & 0x08080808u);  // element 2k in byte k, sign in bit 3
+    const uint32_t odd = co | ((so >> 4) & 0x08080808u);
+    return even + (odd << 4);
+}
+
+// Round-to-nearest-even codes of y * inv, eight values.
+__device__ __forceinline__ uint32_t rn_codes8(const float (&y)[8], float inv) {
+    const f32x2 iv = pk(inv, inv);
     float q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
-    return sr_e2m1x8(q, sr_draws8(rk, stream, e0 >> 3));
+    for (int m = 0; m < 4; ++m) unpk(mul2(pk(y[2 * m], y[2 * m + 1]), iv), q[2 * m], q[2 * m + 1]);
+    return e2m1x8_rn(q);
+}
+
+// One 16-element block (element index e0 % 16 == 0 of the quantized tensor) ->
+// two words of packed codes, RNE or SR (stream `stream`).
+__device__ __forceinline__ uint2 encode16(const float (&y)[16], float inv, bool sr, const uint32_t (&rk)[20],
+                                          uint32_t stream, uint64_t e0) {
+    float lo[8], hi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        lo[i] = y[i];
+        hi[i] = y[8 + i];
+    }
+    if (!sr) return make_uint2(rn_codes8(lo, inv), rn_codes8(hi, inv));
+    return make_uint2(sr_codes8(lo, inv, sr_draws8(rk, stream, e0 >> 3)),
+                      sr_codes8(hi, inv, sr_draws8(rk, stream, (e0 >> 3) + 1)));
 }
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&v)[8]) {
@@ -210,6 +510,21 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&v)[8]) {
 __device__ __forceinline__ float absmax8(const uint4& w) {
     uint32_t m = __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
                           __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+    return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+}
+
+__device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float (&v)[16]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        v[2 * k] = bf16_lo(w[k]);
+        v[2 * k + 1] = bf16_hi(w[k]);
+    }
+}
+
+__device__ __forceinline__ float absmax16(const uint32_t (&w)[8]) {
+    uint32_t m = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = vmax_u16x2(m, w[k] & 0x7FFF7FFFu);
     return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
 }
 
@@ -238,68 +553,60 @@ __device__ __forceinline__ bool load_tensor_scales(const QuantParams& p, TensorS
 }
 
 // ============================================================================
-// Row orientation only, 1x16 blocks: every lane owns 8 consecutive elements
-// (one 16-byte load); a block is a lane pair.  Grid-stride over 8-chunks.
+// Row orientation only, 1x16 blocks: every thread owns whole 16-element blocks
+// (one 32-byte load each).  Grid-stride over blocks.
 // ============================================================================
 __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
     TensorScale tr, tc;
     if (!load_tensor_scales(p, tr, tc)) return;
-    const int64_t cpr = p.cols >> 3;  // 8-chunks per row (even)
-    const int64_t nchunks = p.rows * cpr;
-    const int64_t katoms = (p.cols / 16 + 3) >> 2;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    // warp-uniform trip count: every lane takes part in the pair shuffle
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < nchunks;
-         base += stride) {
-        const int64_t q = base + (threadIdx.x & 31);
-        const bool valid = q < nchunks;
-        const uint4 w = valid ? ld_stream_v4(p.x + q * 8) : make_uint4(0, 0, 0, 0);
-        float amax = absmax8(w);
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-        uint32_t s;
-        float inv;
-        block_scale(amax, tr, s, inv);
-        float v[8];
-        unpack8(w, v);
-        const uint32_t codes = encode8(v, inv, p.row_sr, p.rk, 0u, (uint64_t)q * 8);
-        if (valid) {
-            reinterpret_cast<uint32_t*>(p.row_data)[q] = codes;
-            if ((q & 1) == 0) {
-                const int64_t r = q / cpr, kb = (q % cpr) >> 1;
-                p.row_sf[sf_offset(r, kb, katoms)] = (uint8_t)s;
-            }
-        }
+    __shared__ float inv_tab[256];
+    inv_tab[threadIdx.x] = block_inv_of_code(threadIdx.x, tr.g);
+    __syncthreads();
+    const int64_t bpr = p.cols >> 4;  // 16-blocks per row
+    const int64_t nblocks = p.rows * bpr;
+    const int64_t katoms = (bpr + 3) >> 2;
+    const bool al32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        uint32_t w[8];
+        ld_block16(p.x + b * 16, al32, w);
+        const uint32_t s = block_code(absmax16(w), tr);
+        const float inv = inv_tab[s];
+        float v[16];
+        unpack16(w, v);
+        const uint2 codes = encode16(v, inv, p.row_sr, p.rk, 0u, (uint64_t)b * 16);
+        reinterpret_cast<uint2*>(p.row_data)[b] = codes;
+        p.row_sf[sf_offset(b / bpr, b % bpr, katoms)] = (uint8_t)s;
     }
 }
 
 // ============================================================================
-// Tile kernel: a CTA loads a 64 x 128 bf16 tile once (registers + shared
-// memory) and writes the row orientation (from registers, lane pairs) and/or
-// the column orientation (from shared memory, one lane per column, two
-// 16-row chunks per lane).  k2D: 16x16 blocks, the tile scale is found by the
-// column pass and shared by both orientations.  kRht: 16-point RHT in fp64
-// down each column chunk before the column orientation is quantized.
+// Tile kernel: a CTA loads a 64 x 128 bf16 tile once (registers + shared memory)
+// and writes the row orientation (from registers, one thread per 16-element row
+// block) and/or the column orientation (from shared memory, one thread per column
+// pair and 16-row chunk).  k2D: 16x16 blocks, the tile scale is found by the
+// column pass and shared by both orientations.  kRht: the 16-point RHT down each
+// column chunk before the column orientation is quantized.  Tiles run bottom-up,
+// so the first ones re-read the rows the amax pass read last (still in L2).
 // ============================================================================
 constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;
 
 // Grouped (kGrouped): the tile's rows lie in one group g (see QuantParams), which
 // supplies the tensor scales, the Philox key seed + g and the origin of the
 // element indices.
-// kRowRht: the row orientation is rotated too (16-point RHT along each row block,
-// the block's lane pair exchanging halves), e.g. dgrad operands under the Mosaic
-// recipe.
-// Resident CTAs per SM that the register budget is sized for.  A CTA loads its
-// tile once and then only computes and stores, so more resident CTAs keep more
-// loads in flight; the grouped RHT variant keeps three (at four it spills).
+// kRowRht: the row orientation is rotated too (16-point RHT along each row block),
+// e.g. dgrad operands under the Mosaic recipe.
+// Resident CTAs per SM that the register budget is sized for.
 template <bool k2D, bool kRht, bool kGrouped>
 constexpr int quant_tile_min_blocks() {
-    return (kGrouped && kRht) ? 3 : 4;
+    return (kRht || k2D) ? 3 : 4;
 }
 
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
 __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGrouped>()))
     quant_tile_kernel(QuantParams p) {
     __shared__ __align__(16) uint16_t tile[kTR][kPitch];
+    __shared__ float inv_tab[2][256];  // element multipliers of every scale code: rows, columns
     __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
     __shared__ float tile_inv[kTR / 16][kTC / 16];
     // The tile's scales, staged so that they leave in wide stores instead of one
@@ -310,7 +617,7 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t r0 = (int64_t)blockIdx.y * kTR, c0 = (int64_t)blockIdx.x * kTC;
+    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
     TensorScale tr, tc;
     int64_t g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
     uint32_t rkg[20];                     // the group's Philox round keys
@@ -350,126 +657,149 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     const bool want_row = p.row_data != nullptr;
     const bool want_col = p.col_data != nullptr;
     const bool use_smem = want_col || k2D;
+    {
+        const float dec = e4m3_to_f32((uint32_t)tid);
+        const float gr = __fmul_rn(dec, tr.g), gc = __fmul_rn(dec, tc.g);
+        inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gr), 3.402823466e38f);
+        inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gc), 3.402823466e38f);
+    }
 
-    // ---- load: chunk q = k*256 + tid covers row q/16, columns (q%16)*8 .. +7
-    uint4 reg[4];
+    // ---- load: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
+    const bool al32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0;
+    uint32_t rb[2][8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int q = k * 256 + tid;
-        const int lr = q >> 4, lc = (q & 15) * 8;
+    for (int k = 0; k < 2; ++k) {
+        const int lr = (k * 256 + tid) >> 3, lc = (tid & 7) * 16;
         const int64_t r = r0 + lr, c = c0 + lc;
-        reg[k] = (r < p.rows && c < p.cols) ? ld_stream_v4(p.x + r * p.cols + c)
-                                            : make_uint4(0, 0, 0, 0);
-        if (use_smem) *reinterpret_cast<uint4*>(&tile[lr][lc]) = reg[k];
+        bool in = r < p.rows && c < p.cols;
+        int64_t sr = r;
+        if (p.row_src != nullptr && in) {  // gathered rows
+            sr = __ldg(p.row_src + r);
+            if (sr >= p.src_rows) {
+                set_status(p.status, kStatusIndex);
+                in = false;
+            }
+            in = in && sr >= 0;
+        }
+        if (in) {
+            ld_block16(p.x + sr * p.cols + c, al32, rb[k]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rb[k][i] = 0u;
+        }
     }
-    if (use_smem) __syncthreads();
-
-    // ---- column pass: lane -> column lc, chunks j0, j0+1 (16 rows each)
-    if (use_smem) {
-        const int lc = 32 * (warp & 3) + lane;
-        const int j0 = 2 * (warp >> 2);
-        const int64_t c = c0 + lc;
-        uint32_t out[4];
+    __syncthreads();  // multiplier tables filled (the loads are still in flight)
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-            const int j = j0 + jj;
-            float y[16];
-            if (kRht) {
-                double d[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    d[i] = bf16_signed_to_f64(tile[16 * j + i][lc], (p.sign_mask >> i) & 1u);
-                fwht16(d);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) y[i] = __double2float_rn(d[i]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) y[i] = __uint_as_float((uint32_t)tile[16 * j + i][lc] << 16);
-            }
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
-            uint32_t s;
-            float inv;
-            if (k2D) {
-                // 16x16 tile: 16 lanes hold its 16 columns
-#pragma unroll
-                for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-                block_scale(amax, tc, s, inv);
-                if ((lane & 15) == 0) {
-                    tile_s[j][lc >> 4] = s;
-                    tile_inv[j][lc >> 4] = inv;
-                }
-            } else {
-                block_scale(amax, tc, s, inv);
-            }
-            if (want_col) {
-                const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
-                float lo8[8], hi8[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    lo8[i] = y[i];
-                    hi8[i] = y[8 + i];
-                }
-                out[2 * jj] = encode8(lo8, inv, p.col_sr, rk, 1u, e0);
-                out[2 * jj + 1] = encode8(hi8, inv, p.col_sr, rk, 1u, e0 + 8);
-                // atom byte of (column lc, block j): line lc % 32, group lc / 32
-                col_atom[lane * 16 + (warp & 3) * 4 + j] =
-                    (c < p.cols && r0 + 16 * j < p.rows) ? (uint8_t)s : (uint8_t)0;
-            }
+    for (int k = 0; k < 2; ++k) {
+        const int lr = (k * 256 + tid) >> 3, lc = (tid & 7) * 16;
+        if (use_smem) {
+            // two 16-byte stores, the lane quads of a row taking the halves in opposite
+            // order so that eight lanes cover all 32 banks
+            const int h = (lane >> 2) & 1;
+            uint4* dst = reinterpret_cast<uint4*>(&tile[lr][lc]);
+            dst[h] = h ? make_uint4(rb[k][4], rb[k][5], rb[k][6], rb[k][7])
+                       : make_uint4(rb[k][0], rb[k][1], rb[k][2], rb[k][3]);
+            dst[h ^ 1] = h ? make_uint4(rb[k][0], rb[k][1], rb[k][2], rb[k][3])
+                           : make_uint4(rb[k][4], rb[k][5], rb[k][6], rb[k][7]);
         }
-        if (want_col && c < p.cols) {
-            uint8_t* base = p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j0) >> 1);
-            const bool both = r0 + 16 * (j0 + 1) < p.rows;
-            if (both && (reinterpret_cast<uintptr_t>(base) & 15u) == 0) {
-                *reinterpret_cast<uint4*>(base) = make_uint4(out[0], out[1], out[2], out[3]);
-            } else {
-                if (r0 + 16 * j0 < p.rows) *reinterpret_cast<uint2*>(base) = make_uint2(out[0], out[1]);
-                if (both) *reinterpret_cast<uint2*>(base + 8) = make_uint2(out[2], out[3]);
-            }
-        }
-        if (k2D) __syncthreads();
     }
 
-    // ---- row pass from registers: a 16-block is a lane pair
-    if (want_row) {
+    // ---- row pass from registers: one thread per 16-element block
+    auto row_pass = [&]() {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int q = k * 256 + tid;
-            const int lr = q >> 4, lc = (q & 15) * 8;
+        for (int k = 0; k < 2; ++k) {
+            const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
             const int64_t r = r0 + lr, c = c0 + lc;
             uint32_t s;
             float inv;
-            float v[8];
+            float v[16];
             if (kRowRht) {
-                double y[8];
-                rht16_lane_pair(reg[k], p.sign_mask, lane, y);
+                rht16_row(rb[k], p.sign_mask, v);
                 float amax = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    v[i] = __double2float_rn(y[i]);
-                    amax = fmaxf(amax, fabsf(v[i]));
-                }
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-                block_scale(amax, tr, s, inv);
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                s = block_code(amax, tr);
+                inv = inv_tab[0][s];
             } else if (k2D) {
-                s = tile_s[lr >> 4][lc >> 4];
-                inv = tile_inv[lr >> 4][lc >> 4];
-                unpack8(reg[k], v);
+                s = tile_s[lr >> 4][bc];
+                inv = tile_inv[lr >> 4][bc];
+                unpack16(rb[k], v);
             } else {
-                float amax = absmax8(reg[k]);
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-                block_scale(amax, tr, s, inv);
-                unpack8(reg[k], v);
+                s = block_code(absmax16(rb[k]), tr);
+                inv = inv_tab[0][s];
+                unpack16(rb[k], v);
             }
-            const uint32_t codes =
-                encode8(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
+            const uint2 codes =
+                encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
             const bool inside = r < p.rows && c < p.cols;
-            if (inside) *reinterpret_cast<uint32_t*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
-            // (row lr, block lc / 16): half-atom lc / 64, line lr % 32, byte 4 * (lr / 32) + block % 4
-            if ((lc & 15) == 0)
-                row_half_atoms[lc >> 6][lr & 31][(lr >> 5) * 4 + ((lc >> 4) & 3)] = inside ? (uint8_t)s : (uint8_t)0;
+            if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
+            // (row lr, block bc): half-atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
+            row_half_atoms[bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)s : (uint8_t)0;
         }
+    };
+    if (want_row && !k2D) row_pass();
+    __syncthreads();  // tile in shared memory
+
+    // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunk j
+    if (use_smem) {
+        const int cp = tid & 63, j = tid >> 6;
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = *reinterpret_cast<const uint32_t*>(&tile[16 * j + i][2 * cp]);
+        float y0[16], y1[16];
+        if (kRht) {
+            rht16_pair(w, p.flips, p.sign_mask, y0, y1);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                y0[i] = bf16_lo(w[i]);
+                y1[i] = bf16_hi(w[i]);
+            }
+        }
+        float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            a0 = fmaxf(a0, fabsf(y0[i]));
+            a1 = fmaxf(a1, fabsf(y1[i]));
+        }
+        uint32_t s0, s1;
+        float inv0, inv1;
+        if (k2D) {
+            // the 16x16 tile: 8 consecutive lanes hold its 16 columns
+            float a = fmaxf(a0, a1);
+#pragma unroll
+            for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+            s0 = s1 = block_code(a, tc);
+            inv0 = inv1 = inv_tab[1][s0];
+            if ((cp & 7) == 0) {
+                tile_s[j][cp >> 3] = s0;
+                tile_inv[j][cp >> 3] = inv0;
+            }
+        } else {
+            s0 = block_code(a0, tc);
+            s1 = block_code(a1, tc);
+            inv0 = inv_tab[1][s0];
+            inv1 = inv_tab[1][s1];
+        }
+        if (want_col) {
+            const bool rin = r0 + 16 * j < p.rows;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int lc = 2 * cp + h;
+                const int64_t c = c0 + lc;
+                const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
+                const uint2 codes = encode16(h ? y1 : y0, h ? inv1 : inv0, p.col_sr, rk, 1u, e0);
+                const bool inside = c < p.cols && rin;
+                if (inside)
+                    *reinterpret_cast<uint2*>(p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j) >> 1)) = codes;
+                // atom byte of (column lc, block j): line lc % 32, group lc / 32
+                col_atom[(lc & 31) * 16 + (lc >> 5) * 4 + j] = inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
+            }
+        }
+    }
+    if (want_row && k2D) {
+        __syncthreads();  // tile scales written
+        row_pass();
     }
 
     // ---- scale stores.  Every entry written lies inside the scale buffer: the
@@ -569,61 +899,41 @@ __global__ void sf_pad_kernel(uint8_t* __restrict__ sf, int64_t rows, int64_t nb
 }
 
 // ============================================================================
-// Standalone RHT.  axis 1: a thread transforms 16 contiguous elements.
-// axis 0: a thread transforms 8 columns x 16 rows (like the amax unit).
+// Standalone RHT, through the same exactly rounded transforms as the quantizer.
+// axis 1: a thread transforms one 16-element chunk of a row (rht16_row).
+// axis 0: a thread transforms a column pair x 16 rows (rht16_pair); consecutive
+// lanes take consecutive column pairs, so loads and stores are coalesced.
 // ============================================================================
 __global__ void __launch_bounds__(256) rht_axis1_kernel(const uint16_t* __restrict__ x, float* __restrict__ y,
                                                        int64_t nchunks, uint32_t sign_mask) {
+    const bool al32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0;
     for (int64_t ch = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ch < nchunks;
          ch += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 a = ld_stream_v4(x + ch * 16), b = ld_stream_v4(x + ch * 16 + 8);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        double d[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            d[i] = bf16_signed_to_f64((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu),
-                                      (sign_mask >> i) & 1u);
-        fwht16(d);
+        uint32_t w[8];
+        ld_block16(x + ch * 16, al32, w);
+        float v[16];
+        rht16_row(w, sign_mask, v);
         float4* out = reinterpret_cast<float4*>(y + ch * 16);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            out[i] = make_float4(__double2float_rn(d[4 * i]), __double2float_rn(d[4 * i + 1]),
-                                 __double2float_rn(d[4 * i + 2]), __double2float_rn(d[4 * i + 3]));
+        for (int i = 0; i < 4; ++i) out[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
 }
 
 __global__ void __launch_bounds__(256) rht_axis0_kernel(const uint16_t* __restrict__ x, float* __restrict__ y,
-                                                       int64_t rows, int64_t cols, uint32_t sign_mask) {
-    const int64_t cunits = cols / 8;
-    const int64_t units = (rows / 16) * cunits;
+                                                       int64_t rows, int64_t cols, uint32_t sign_mask,
+                                                       const RhtFlips flips) {
+    const int64_t cpairs = cols / 2;
+    const int64_t units = (rows / 16) * cpairs;
     for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units;
          u += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r0 = (u / cunits) * 16, c0 = (u % cunits) * 8;
-        uint4 v[16];
+        const int64_t r0 = (u / cpairs) * 16, c = (u % cpairs) * 2;
+        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = ld_stream_v4(x + (r0 + i) * cols + c0);
+        for (int i = 0; i < 16; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(x + (r0 + i) * cols + c));
+        float y0[16], y1[16];
+        rht16_pair(w, flips, sign_mask, y0, y1);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {  // columns 4*half .. 4*half+3
-            float o[16][4];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const int c = 4 * half + cc;
-                double d[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = (c >> 1) == 0 ? v[i].x : (c >> 1) == 1 ? v[i].y
-                                     : (c >> 1) == 2 ? v[i].z : v[i].w;
-                    d[i] = bf16_signed_to_f64((c & 1) ? (w >> 16) : (w & 0xFFFFu), (sign_mask >> i) & 1u);
-                }
-                fwht16(d);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[i][cc] = __double2float_rn(d[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                *reinterpret_cast<float4*>(y + (r0 + i) * cols + c0 + 4 * half) =
-                    make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
-        }
+        for (int i = 0; i < 16; ++i) *reinterpret_cast<float2*>(y + (r0 + i) * cols + c) = make_float2(y0[i], y1[i]);
     }
 }
 
@@ -643,14 +953,16 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
                         bool row_rht) {
     const int64_t units = ((rows + 15) / 16) * ((cols + 255) / 256);
     const int grid = grid_for(units, 8, sm_count, 8);
+    RhtFlips f;
+    rht_flips(sign_mask, f);
     if (row_rht && col_rht)
-        amax_kernel<true, false, true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+        amax_kernel<true, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
     else if (row_rht)
-        amax_kernel<false, false, true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+        amax_kernel<false, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
     else if (col_rht)
-        amax_kernel<true, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+        amax_kernel<true, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
     else
-        amax_kernel<false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, words, nullptr, 0);
+        amax_kernel<false, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
     return cudaGetLastError();
 }
 
@@ -658,12 +970,20 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
     const int64_t units = ((p.rows + 15) >> 4) * ((p.cols + 255) >> 8);
     const int grid = grid_for(units, 8, sm_count, 8);
     uint32_t* words = const_cast<uint32_t*>(p.amax_words);
-    if (p.col_rht)
-        amax_kernel<true, true, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
-                                                     p.group_rows_uniform);
+    RhtFlips f;
+    rht_flips(p.sign_mask, f);
+    if (p.col_rht && p.row_src)
+        amax_kernel<true, true, false, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
+                                                                   p.row_group, p.group_rows_uniform, p.row_src,
+                                                                   p.src_rows, p.status);
+    else if (p.col_rht)
+        amax_kernel<true, true, false, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
+                                                                    p.row_group, p.group_rows_uniform, nullptr, 0,
+                                                                    p.status);
     else
-        amax_kernel<false, true, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, words, p.row_group,
-                                                      p.group_rows_uniform);
+        amax_kernel<false, true, false, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
+                                                                     p.row_group, p.group_rows_uniform, nullptr,
+                                                                     0, p.status);
     return cudaGetLastError();
 }
 
@@ -676,13 +996,19 @@ struct GroupSizes {
     int64_t rows[kMaxGroups];
 };
 __global__ void group_tables_kernel(GroupSizes gs, int E, int32_t* __restrict__ block_group,
-                                    int64_t* __restrict__ row0, int64_t* __restrict__ nrows) {
+                                    int64_t* __restrict__ row0, int64_t* __restrict__ nrows,
+                                    int64_t* __restrict__ pair_row0, int32_t* __restrict__ pair_group,
+                                    int32_t* __restrict__ pair_rows) {
     __shared__ int64_t start[kMaxGroups + 1];
+    __shared__ int32_t tstart[kMaxGroups];  // first 256-row tile of every group
     if (threadIdx.x == 0) {
         int64_t r = 0;
+        int32_t t = 0;
         for (int e = 0; e < E; ++e) {
             start[e] = r;
+            tstart[e] = t;
             r += gs.rows[e];
+            t += (int32_t)((gs.rows[e] + 255) / 256);
         }
         start[E] = r;
     }
@@ -690,6 +1016,18 @@ __global__ void group_tables_kernel(GroupSizes gs, int E, int32_t* __restrict__ 
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         row0[e] = start[e];
         nrows[e] = gs.rows[e];
+    }
+    // the 256-row tiles of every group (block 0 writes them): a group of 128 * odd
+    // rows ends with a tile whose second half lies past the group
+    if (pair_row0 && blockIdx.x == 0) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const int32_t n = (int32_t)((gs.rows[e] + 255) / 256);
+            for (int32_t t = 0; t < n; ++t) {
+                pair_row0[tstart[e] + t] = start[e] + 256 * (int64_t)t;
+                pair_group[tstart[e] + t] = e;
+                pair_rows[tstart[e] + t] = (int32_t)(gs.rows[e] - 256 * (int64_t)t < 256 ? gs.rows[e] - 256 * (int64_t)t : 256);
+            }
+        }
     }
     const int64_t blocks = start[E] / 128;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < blocks;
@@ -705,7 +1043,8 @@ __global__ void group_tables_kernel(GroupSizes gs, int E, int32_t* __restrict__ 
 }
 
 cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block_group, int64_t* row0,
-                                int64_t* nrows, cudaStream_t st) {
+                                int64_t* nrows, cudaStream_t st, int64_t* pair_row0, int32_t* pair_group,
+                                int32_t* pair_rows) {
     if (E < 1 || E > kMaxGroups) return cudaErrorInvalidValue;
     GroupSizes gs;
     memset(&gs, 0, sizeof gs);
@@ -716,15 +1055,16 @@ cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block
     }
     const int64_t blocks = total / 128;
     const int grid = (int)((blocks + 255) / 256 < 64 ? (blocks + 255) / 256 : 64);
-    group_tables_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(gs, E, block_group, row0, nrows);
+    group_tables_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(gs, E, block_group, row0, nrows, pair_row0,
+                                                               pair_group, pair_rows);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStream_t st) {
     QuantParams p = params;
     philox_round_keys(p.seed, p.rk);
-    const int64_t nchunks = p.rows * (p.cols / 8);
-    const int grid = grid_for(nchunks, 256, sm_count, 8);
+    const int64_t nblocks = p.rows * (p.cols / 16);
+    const int grid = grid_for(nblocks, 256, sm_count, 8);
     quant_rows_kernel<<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
@@ -732,6 +1072,7 @@ cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStrea
 cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, cudaStream_t st) {
     QuantParams p = params;
     philox_round_keys(p.seed, p.rk);
+    rht_flips(p.sign_mask, p.flips);
     const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
     const bool grouped = p.row_group != nullptr || p.group_rows_uniform > 0;
     if (p.row_rht && (grouped || two_d)) return cudaErrorInvalidValue;
@@ -769,8 +1110,10 @@ cudaError_t launch_rht(const uint16_t* x, float* y, int64_t rows, int64_t cols, 
         const int64_t n = rows * cols / 16;
         rht_axis1_kernel<<<grid_for(n, 256, sm_count, 8), 256, 0, st>>>(x, y, n, sign_mask);
     } else {
-        const int64_t n = (rows / 16) * (cols / 8);
-        rht_axis0_kernel<<<grid_for(n, 256, sm_count, 4), 256, 0, st>>>(x, y, rows, cols, sign_mask);
+        const int64_t n = (rows / 16) * (cols / 2);
+        RhtFlips f;
+        rht_flips(sign_mask, f);
+        rht_axis0_kernel<<<grid_for(n, 256, sm_count, 4), 256, 0, st>>>(x, y, rows, cols, sign_mask, f);
     }
     return cudaGetLastError();
 }

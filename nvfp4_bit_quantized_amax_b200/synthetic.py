@@ -138,3 +138,33 @@ def linear_small_inputs(seed=0):
     W = normal_bf16((s["N"], s["K"]), seed + 1, outlier_prob=0.01)
     dY = normal_bf16((s["M"], s["N"]), seed + 2, outlier_prob=0.01)
     return X, W, dY
+
+
+def device_bf16(kind, shape, seed, device, std=1.0):
+    """Benchmark-scale inputs drawn on the GPU with torch's seeded generator (same
+    distributions as the host recipes above, not the same values): kind "normal"
+    N(0, std^2), "student_t" with nu = 3 (Z0 / sqrt((Z1^2 + Z2^2 + Z3^2) / 3)),
+    "laplace" Laplace(0, 1) (the difference of two unit exponentials).  Drawn in
+    fp32, rounded to bf16 (nearest, ties to even).  Parity tests use the host
+    recipes; these only feed throughput measurements."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    if kind == "normal":
+        z = torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std
+    elif kind == "student_t":
+        z0 = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        v = torch.zeros(shape, device=device, dtype=torch.float32)
+        for _ in range(3):
+            v += torch.randn(shape, generator=g, device=device, dtype=torch.float32) ** 2
+        z = z0 / torch.sqrt(v / 3.0)
+        del z0, v
+    elif kind == "laplace":
+        e1 = -torch.log1p(-torch.rand(shape, generator=g, device=device, dtype=torch.float32))
+        e2 = -torch.log1p(-torch.rand(shape, generator=g, device=device, dtype=torch.float32))
+        z = e1 - e2
+        del e1, e2
+    else:
+        raise ValueError(kind)
+    return z.to(torch.bfloat16)

@@ -124,3 +124,112 @@ def test_grouped_rejects_unaligned_groups():
     g = np.array([128, 64], dtype=np.int64)
     assert capi.moe_grouped_workspace_bytes(g, 128, 128) == 0
     assert capi.moe_grouped_workspace_bytes(np.array([128], dtype=np.int64), 192, 128) == 0
+
+
+def test_grouped_config_vs_oracle(ora):
+    """The grouped expert layer as the MoE benchmark runs it (64 experts, hidden 2048,
+    expert FFN 1024, 16384 tokens, top-4 of Zipf(1.1), segments padded to 128 rows),
+    checked against the oracle directly: for the largest, the smallest and a middle
+    expert every grouped operand byte (codes and swizzled scales) and every tensor
+    scale, and a 32 x 32 grid of sampled outputs of Y, dX and dW[e] within the bound.
+    The largest expert's wgrad reduces over its whole row range (45+ k-tiles)."""
+    s = syn.MOE
+    E, K, N = s["experts"], s["hidden"], s["ffn"]
+    d = syn.moe_inputs(s["tokens"], E, K, N, s["topk"], s["zipf_s"], seed=0, pad=128)
+    g = d["group_rows"]
+    R = int(g.sum())
+    offs = np.concatenate([[0], np.cumsum(g)]).astype(np.int64)
+    signs = syn.rht_signs(0)
+    seed = 4242
+
+    x_tok = to_dev_bf16(d["X"])
+    W = to_dev_bf16(d["W"].reshape(E * N, K)).view(E, N, K)
+    dY = to_dev_bf16(d["dY"])
+    row_src = torch.from_numpy(d["row_src"]).to(DEV)
+    Y, dX, dW = nan_bf16(R, N), nan_bf16(R, K), nan_bf16(E, N, K)
+    ws = torch.empty(capi.moe_grouped_workspace_bytes(g, K, N), dtype=torch.uint8, device=DEV)
+    # as the benchmark runs it: the gather fused into the quantization of X
+    capi.nvfp4_moe_grouped_fprop_gather(x_tok, row_src, W, Y, g, signs, ws)
+    capi.nvfp4_moe_grouped_dgrad(dY, dX, g, seed, signs, ws)
+    capi.nvfp4_moe_grouped_wgrad(dW, g, ws)
+    torch.cuda.synchronize()
+    assert capi.nvfp4_read_status(ws) == 0
+
+    # the routed tokens' rows in expert order (padding rows zero), gathered on the host
+    rs = d["row_src"]
+    xp = np.zeros((R, K), np.uint16)
+    xp[rs >= 0] = d["X"][rs[rs >= 0]]
+
+    views = {w: grouped_view(ws, g, K, N, w) for w in range(6)}
+    kinds = {capi.LIN_X_ROW: "rows", capi.LIN_X_COL: "cols", capi.LIN_W_ROW: "wrows",
+             capi.LIN_W_COL: "wcols", capi.LIN_DY_ROW: "rows", capi.LIN_DY_COL: "cols"}
+    order = np.argsort(g)
+    for e in (int(order[-1]), int(order[0]), int(order[len(order) // 2])):
+        off, m = int(offs[e]), int(g[e])
+        Xe, We, dYe = xp[off:off + m], d["W"][e], d["dY"][off:off + m]
+        specs = {capi.LIN_X_ROW: (Xe, 0, False, 0, 0, 0), capi.LIN_X_COL: (Xe, 1, True, 0, 0, 0),
+                 capi.LIN_W_ROW: (We, 0, False, 1, 0, 0), capi.LIN_W_COL: (We, 1, False, 1, 0, 0),
+                 capi.LIN_DY_ROW: (dYe, 0, False, 0, 1, seed + e),
+                 capi.LIN_DY_COL: (dYe, 1, True, 0, 1, seed + e)}
+        ref = {}
+        for which, (src, orient, rht, bm, rnd, sd) in specs.items():
+            p, sf, gg, _ = ora.quantize(src, orient, rht, signs, bm, rnd, sd)
+            gv, gdata, gsf, gscale = views[which]
+            dd, ss = expert_slice(kinds[which], gv, gdata, gsf, e, off, m, N)
+            assert np.array_equal(dd, p), (e, which)
+            assert np.array_equal(ss, ora.sf_swizzle(sf, p.shape[1] * 2)), (e, which)
+            assert gscale[e].view(np.uint32) == np.float32(gg).view(np.uint32), (e, which)
+            ref[which] = (p, sf, float(gg))
+        rng = np.random.default_rng(e)
+        for out, a, b, alpha in ((Y[off:off + m], capi.LIN_X_ROW, capi.LIN_W_ROW, 1.0),
+                                 (dX[off:off + m], capi.LIN_DY_ROW, capi.LIN_W_COL, 1.0),
+                                 (dW[e], capi.LIN_DY_COL, capi.LIN_X_COL, 1.0 / 16)):
+            pa, sa, ga = ref[a]
+            pb, sb, gb = ref[b]
+            mi = np.repeat(rng.choice(pa.shape[0], 32, replace=pa.shape[0] < 32), 32)
+            ni = np.tile(rng.choice(pb.shape[0], 32, replace=False), 32)
+            r, bound = ora.gemm_pairs(pa, sa, pb, sb, alpha * ga * gb, mi, ni)
+            got = out.float()[torch.from_numpy(mi).to(DEV), torch.from_numpy(ni).to(DEV)]
+            got = got.cpu().numpy().astype(np.float64)
+            # fp32 within 1e-4 * bound of the exact value, then one bf16 rounding
+            # (half an ulp, 2^-9 relative)
+            lim = 1e-4 * bound * (1 + 2.0 ** -9) + 2.0 ** -9 * np.abs(r) + 1e-30
+            assert (np.abs(got - r) <= lim).all(), (e, a)
+
+
+def test_fused_gather_equals_gather_then_grouped():
+    """nvfp4_moe_grouped_fprop_gather (X's rows read through row_src inside the
+    quantizer) leaves the same X and W operands, tensor scales and Y as the gather
+    kernel followed by nvfp4_moe_grouped_fprop; an index past the token rows is
+    reported as NVFP4_ERR_INDEX and read as a zero row."""
+    E, K, N, T, k = 6, 256, 384, 300, 2
+    d = syn.moe_inputs(T, E, K, N, k, 1.1, seed=5, pad=128)
+    g = d["group_rows"]
+    R = int(g.sum())
+    signs = syn.rht_signs(1)
+    x_tok = to_dev_bf16(d["X"])
+    W = to_dev_bf16(d["W"].reshape(E * N, K)).view(E, N, K)
+    row_src = torch.from_numpy(d["row_src"]).to(DEV)
+
+    ws_a = torch.empty(capi.moe_grouped_workspace_bytes(g, K, N), dtype=torch.uint8, device=DEV)
+    ws_b = torch.empty_like(ws_a)
+    X_perm = torch.empty((R, K), dtype=torch.bfloat16, device=DEV)
+    Ya, Yb = nan_bf16(R, N), nan_bf16(R, N)
+    capi.nvfp4_moe_gather(x_tok, row_src, X_perm)
+    capi.nvfp4_moe_grouped_fprop(X_perm, W, Ya, g, signs, ws_a)
+    capi.nvfp4_moe_grouped_fprop_gather(x_tok, row_src, W, Yb, g, signs, ws_b)
+    torch.cuda.synchronize()
+    assert capi.nvfp4_read_status(ws_a) == 0 and capi.nvfp4_read_status(ws_b) == 0
+    assert torch.equal(bits(Ya), bits(Yb))
+    for which in (capi.LIN_X_ROW, capi.LIN_X_COL, capi.LIN_W_ROW, capi.LIN_W_COL):
+        _, da, sa, ga = grouped_view(ws_a, g, K, N, which)
+        _, db, sb, gb = grouped_view(ws_b, g, K, N, which)
+        assert np.array_equal(da, db) and np.array_equal(sa, sb), which
+        assert np.array_equal(ga.view(np.uint32), gb.view(np.uint32)), which
+
+    bad = d["row_src"].copy()
+    first_real = int(np.nonzero(bad >= 0)[0][0])
+    bad[first_real] = T + 7  # past the token rows
+    capi.nvfp4_moe_grouped_fprop_gather(x_tok, torch.from_numpy(bad).to(DEV), W, Yb, g, signs, ws_b)
+    torch.cuda.synchronize()
+    assert capi.nvfp4_read_status(ws_b) == capi.ERR_INDEX

@@ -45,7 +45,7 @@ def test_mx_quantize_parity(ora, rows, cols, kind):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (256, 512, 1024), (200, 136, 384),
-                                   (128, 256, 2048)])
+                                   (128, 256, 2048), (640, 520, 1152)])
 def test_mx_gemm_parity(ora, M, N, K):
     rng = np.random.default_rng(M + N + K)
     A = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)

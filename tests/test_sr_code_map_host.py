@@ -1,16 +1,17 @@
 """The stochastic-rounding arithmetic of the quantize kernels, emulated exactly on
 the host and compared with the oracle's rounding rule (CPU only).
 
-The kernels do not select grid neighbours per element.  They map a = min(|v|, 6)
-through the concave code-space map c(a) = min(2a, a + 2, a/2 + 4, 7), which is
-affine between grid points and sends the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6} to
-the codes 0..7.  So floor(c) is the code of the lower neighbour and frac(c) is
+The kernels do not select grid neighbours per element.  They clamp a = min(|v|, 6)
+and map it through the concave code-space map c(a) = min(2a, a + 2, a/2 + 4), which
+is affine between grid points and sends the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6} to
+the codes 0..7 (c(6) = 7, so no further cap is needed).  So floor(c) is the code of the lower neighbour and frac(c) is
 the round-up probability p, and the code is floor(c) + [r < p * 2^16] =
 (ceil(c * 2^16) + 65535 - r) >> 16 for the 16-bit draw r.  Each branch of the
 minimum is one fp32 FMA rounded upward, with addend 2^23 + offset * 2^16 + 65535.
 The sums are integers below 2^24, so the only rounding is the ceiling, and the
-minimum commutes with it.  The float's bits minus r then hold the code in bits
-16-18.
+minimum commutes with it (the kernels evaluate two elements per packed fp32x2 FMA
+and take the minimum of the three branches in one three-input min).  The float's
+bits minus r then hold the code in bits 16-18.
 
 This test repeats those steps with exact rational arithmetic for the upward
 rounding and compares the code with the oracle's rule ("round up iff r < p * 2^16",
@@ -29,7 +30,6 @@ from oracle import oracle as ora
 
 SLOPES = (131072.0, 65536.0, 32768.0)  # 2^16 * (2, 1, 1/2)
 ADDENDS = (8388608 + 65535, 8388608 + 2 * 65536 + 65535, 8388608 + 4 * 65536 + 65535)
-CLAMP = np.float32(8388608 + 7 * 65536 + 65535)  # code 7 (magnitude 6) and above
 
 
 def fma_round_up(a, b, c):
@@ -47,8 +47,8 @@ def fma_round_up(a, b, c):
 
 def kernel_code(v, r):
     v = np.float32(v)
-    a = np.float32(abs(float(v)))
-    t = min(min(fma_round_up(a, s, c) for s, c in zip(SLOPES, ADDENDS)), CLAMP)
+    a = np.float32(min(abs(float(v)), 6.0))
+    t = min(fma_round_up(a, s, c) for s, c in zip(SLOPES, ADDENDS))
     bits = int(np.float32(t).view(np.uint32))
     assert bits >> 23 == 0x96  # the value lies in [2^23, 2^24): the code is in bits 16-18
     code = ((bits - r) >> 16) & 7
