@@ -58,7 +58,11 @@ typedef enum nvfp4_status {
     NVFP4_ERR_TIMEOUT = -6,   /* device status: a bounded wait in a kernel ran out  */
     NVFP4_ERR_WORKSPACE = -7, /* workspace pointer null or smaller than required    */
     NVFP4_ERR_DEVICE = -8,    /* the current device is not sm_100 (B200 class)      */
-    NVFP4_ERR_INDEX = -9      /* a row index lies outside its source tensor (device) */
+    NVFP4_ERR_INDEX = -9,     /* a row index lies outside its source tensor (device) */
+    NVFP4_ERR_RHT_RANGE = -10 /* a rotated 16-chunk's inputs span more than 41 binades
+                                 (device): the outputs were still written, but that
+                                 chunk's transform is the fp64 rounding of its sum,
+                                 not the correctly rounded exact sum                  */
 } nvfp4_status;
 
 enum { NVFP4_BLOCK_1X16 = 0, NVFP4_BLOCK_16X16 = 1 };

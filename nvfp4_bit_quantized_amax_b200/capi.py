@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libnvfp4.so")
 
 OK, ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_WORKSPACE, \
-    ERR_DEVICE, ERR_INDEX = 0, -1, -2, -3, -4, -5, -6, -7, -8, -9
+    ERR_DEVICE, ERR_INDEX, ERR_RHT_RANGE = 0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10
 BLOCK_1X16, BLOCK_16X16 = 0, 1
 ROUND_RNE, ROUND_SR = 0, 1
 LIN_X_ROW, LIN_X_COL, LIN_W_ROW, LIN_W_COL, LIN_DY_ROW, LIN_DY_COL = range(6)

@@ -96,7 +96,7 @@ int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_
                  uint8_t* cd, uint8_t* csf, float* cg, uint32_t* words, int* status, int sms,
                  cudaStream_t st, bool rows_only_kernel, int row_rht = 0) {
     cudaError_t e = launch_amax(static_cast<const uint16_t*>(x), rows, cols, col_rht && cd, mask,
-                                words, sms, st, row_rht != 0);
+                                words, sms, st, row_rht != 0, status);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     QuantParams p;
     memset(&p, 0, sizeof p);
@@ -199,6 +199,7 @@ const char* nvfp4_status_string(int s) {
         case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
         case NVFP4_ERR_DEVICE: return "device is not sm_100";
         case NVFP4_ERR_INDEX: return "a row index lies outside its source tensor";
+        case NVFP4_ERR_RHT_RANGE: return "a rotated 16-chunk spans more than 41 binades";
         default: return "unknown status";
     }
 }

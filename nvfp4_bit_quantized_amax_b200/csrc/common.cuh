@@ -21,6 +21,7 @@ namespace nvfp4 {
 constexpr int kStatusNonFinite = -5;
 constexpr int kStatusTimeout = -6;
 constexpr int kStatusIndex = -9;
+constexpr int kStatusRhtRange = -10;
 
 // Record the first device-side error in a status word (0 = ok).
 __device__ __forceinline__ void set_status(int* status, int code) {

@@ -85,7 +85,7 @@ inline void philox_round_keys(uint64_t seed, uint32_t (&rk)[20]) {
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
                         uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st,
-                        bool row_rht = false);
+                        bool row_rht = false, int* status = nullptr);
 cudaError_t launch_quant_rows(const QuantParams& p, int sm_count, cudaStream_t st);
 cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, cudaStream_t st);
 cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st);

@@ -139,6 +139,16 @@ __device__ __forceinline__ bool span_ok(uint32_t vmx, uint32_t vmn) {
     return emax <= 251 && emax - max(emin, 1) <= 13;
 }
 
+// Outside the fp64 butterfly's exact domain (span above 41 binades, or Inf / NaN):
+// the transform is then the fp64 rounding, not the exact sum's.  Recorded in the
+// status word (nullable) when a chunk of the quantizer's input lies there.
+__device__ __forceinline__ void note_f64_domain(uint32_t vmx, uint32_t vmn, int* status) {
+    if (status == nullptr || vmx == 0x7FFFu) return;
+    const int emax = (int)((vmx - 0x7FFFu) >> 7);
+    const int emin = (int)((vmn - 0x7FFFu) >> 7);
+    if (emax <= 254 && emax - max(emin, 1) > 41) set_status(status, kStatusRhtRange);
+}
+
 // Chunk statistics of packed bf16 words (two independent lanes): per 16-bit lane,
 // the unsigned maximum and signed minimum of v = |x| + 0x7FFF (no carry between the
 // lanes: |x| <= 0x7FFF).
@@ -169,7 +179,7 @@ __device__ __forceinline__ void rht16_col_f64(const uint32_t (&w)[16], int half,
 // Rotation of a column pair: w[i] holds row i of two adjacent columns (the first in
 // the low half).  y0 / y1 receive the transforms of the two columns.
 __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFlips& f, uint32_t sign_mask,
-                                           float (&y0)[16], float (&y1)[16]) {
+                                           float (&y0)[16], float (&y1)[16], int* status = nullptr) {
     uint32_t vmx, vmn;
     chunk_stats<16>(w, vmx, vmn);
     if (span_ok(vmx & 0xFFFFu, vmn & 0xFFFFu) && span_ok(vmx >> 16, vmn >> 16)) {
@@ -190,6 +200,8 @@ __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFli
 #pragma unroll
         for (int i = 0; i < 16; ++i) unpk(x[i], y0[i], y1[i]);
     } else {
+        note_f64_domain(vmx & 0xFFFFu, vmn & 0xFFFFu, status);
+        note_f64_domain(vmx >> 16, vmn >> 16, status);
         rht16_col_f64(w, 0, sign_mask, y0);
         rht16_col_f64(w, 1, sign_mask, y1);
     }
@@ -199,7 +211,8 @@ __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFli
 // is not formed: max(|RN(a+b)|, |RN(a-b)|) = RN(|a| + |b|) exactly (RN is monotone
 // and odd, and max(|a+b|, |a-b|) = |a| + |b|).
 __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], const RhtFlips& f,
-                                                   uint32_t sign_mask, uint32_t vmx, uint32_t vmn) {
+                                                   uint32_t sign_mask, uint32_t vmx, uint32_t vmn,
+                                                   int* status) {
     float m = 0.0f;
     if (span_ok(vmx & 0xFFFFu, vmn & 0xFFFFu) && span_ok(vmx >> 16, vmn >> 16)) {
         f32x2 x[16];
@@ -224,6 +237,8 @@ __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], cons
             m = fmaxf(m, fmaxf(fabsf(a0) + fabsf(b0), fabsf(a1) + fabsf(b1)));
         }
     } else {
+        note_f64_domain(vmx & 0xFFFFu, vmn & 0xFFFFu, status);
+        note_f64_domain(vmx >> 16, vmn >> 16, status);
         float y[16];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -237,7 +252,8 @@ __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], cons
 
 // Rotation of one row block held by one thread: w[k] holds elements 2k, 2k+1 of the
 // block (16 values).  Scalar fp32 butterfly under the same span test, else fp64.
-__device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_mask, float (&y)[16]) {
+__device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_mask, float (&y)[16],
+                                          int* status = nullptr) {
     uint32_t vmx, vmn;
     chunk_stats<8>(w, vmx, vmn);
     const uint32_t mx = max(vmx & 0xFFFFu, vmx >> 16);
@@ -260,6 +276,7 @@ __device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_
             }
         }
     } else {
+        note_f64_domain(mx, mn, status);
         double d[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -373,7 +390,7 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
                 uint32_t vmx, vmn;
                 chunk_stats<16>(w, vmx, vmn);
                 m_row = vmax_u16x2(m_row, vmx - 0x7FFF7FFFu);
-                m_col = fmaxf(m_col, rht16_pair_absmax(w, flips, sign_mask, vmx, vmn));
+                m_col = fmaxf(m_col, rht16_pair_absmax(w, flips, sign_mask, vmx, vmn, status));
             }
         } else {
 #pragma unroll
@@ -714,7 +731,7 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
             float inv;
             float v[16];
             if (kRowRht) {
-                rht16_row(rb[k], p.sign_mask, v);
+                rht16_row(rb[k], p.sign_mask, v, p.status);
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
@@ -748,7 +765,7 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
         for (int i = 0; i < 16; ++i) w[i] = *reinterpret_cast<const uint32_t*>(&tile[16 * j + i][2 * cp]);
         float y0[16], y1[16];
         if (kRht) {
-            rht16_pair(w, p.flips, p.sign_mask, y0, y1);
+            rht16_pair(w, p.flips, p.sign_mask, y0, y1, p.status);
         } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -950,19 +967,19 @@ static int grid_for(int64_t work_items, int per_block, int sm_count, int blocks_
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
                         uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st,
-                        bool row_rht) {
+                        bool row_rht, int* status) {
     const int64_t units = ((rows + 15) / 16) * ((cols + 255) / 256);
     const int grid = grid_for(units, 8, sm_count, 8);
     RhtFlips f;
     rht_flips(sign_mask, f);
     if (row_rht && col_rht)
-        amax_kernel<true, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
+        amax_kernel<true, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
     else if (row_rht)
-        amax_kernel<false, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
+        amax_kernel<false, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
     else if (col_rht)
-        amax_kernel<true, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
+        amax_kernel<true, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
     else
-        amax_kernel<false, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, nullptr);
+        amax_kernel<false, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
     return cudaGetLastError();
 }
 

@@ -191,9 +191,9 @@ def test_grouped_config_vs_oracle(ora):
             r, bound = ora.gemm_pairs(pa, sa, pb, sb, alpha * ga * gb, mi, ni)
             got = out.float()[torch.from_numpy(mi).to(DEV), torch.from_numpy(ni).to(DEV)]
             got = got.cpu().numpy().astype(np.float64)
-            # fp32 within 1e-4 * bound of the exact value, then one bf16 rounding
-            # (half an ulp, 2^-9 relative)
-            lim = 1e-4 * bound * (1 + 2.0 ** -9) + 2.0 ** -9 * np.abs(r) + 1e-30
+            # fp32 value v within 1e-4 * bound of the exact r, then one bf16 rounding:
+            # half an ulp of v, at most 2^-8 |v| (8 significant bits)
+            lim = 1e-4 * bound * (1 + 2.0 ** -8) + 2.0 ** -8 * np.abs(r) + 1e-30
             assert (np.abs(got - r) <= lim).all(), (e, a)
 
 
