@@ -117,7 +117,7 @@ int run_quantize(const void* x, int64_t rows, int64_t cols, bool two_d, int row_
     p.col_rht = (col_rht && cd) ? 1 : 0;
     p.row_rht = row_rht;
     p.sign_mask = mask;
-    e = rows_only_kernel && !row_rht ? launch_quant_rows(p, sms, st) : launch_quant_tile(p, two_d, st);
+    e = rows_only_kernel && !row_rht ? launch_quant_rows(p, sms, st) : launch_quant_tile(p, two_d, sms, st);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     if (rsf && (e = launch_sf_pad(rsf, rows, cols / 16, sms, st)) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (csf && (e = launch_sf_pad(csf, cols, rows / 16, sms, st)) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -699,7 +699,7 @@ int run_quantize_grouped(const void* x, int64_t rows, int64_t cols, bool two_d, 
     p.src_rows = src_rows;
     cudaError_t e = launch_amax_grouped(p, sms, st);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-    e = launch_quant_tile(p, two_d, st);
+    e = launch_quant_tile(p, two_d, sms, st);
     return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

@@ -87,7 +87,7 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
                         uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st,
                         bool row_rht = false, int* status = nullptr);
 cudaError_t launch_quant_rows(const QuantParams& p, int sm_count, cudaStream_t st);
-cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, cudaStream_t st);
+cudaError_t launch_quant_tile(const QuantParams& p, bool two_d, int sm_count, cudaStream_t st);
 cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st);
 cudaError_t launch_mx_quant_rows(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* packed,
                                  uint8_t* sf, int sm_count, cudaStream_t st);

@@ -141,7 +141,7 @@ extern "C" int nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols,
     p.seed = seed;
     p.row_sr = rounding == NVFP4_ROUND_SR;
     cudaError_t e = (block_mode == NVFP4_BLOCK_1X16) ? launch_quant_rows(p, sms, st)
-                                                     : launch_quant_tile(p, true, st);
+                                                     : launch_quant_tile(p, true, sms, st);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     if (launch_sf_pad(scales, rows, cols / 16, sms, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     return NVFP4_OK;

@@ -110,9 +110,15 @@ __device__ __forceinline__ void ld_block16(const uint16_t* p, bool al32, uint32_
 // one, or Inf / NaN) take an fp64 butterfly, exact while the span is at most 41
 // binades; its fp32 rounding is the same RN32 of the exact sum.
 // ============================================================================
+// An exact zero sum is +0 (the real number 0): adding +0 to the first operand of the
+// last stage turns a -0 partial sum into +0, and then a +- b is -0 for no inputs.
 __device__ __forceinline__ void fwht16(double (&y)[16]) {
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {
+        if (h == 8) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = __dadd_rn(y[i], 0.0);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             if ((i & h) == 0) {
@@ -186,8 +192,13 @@ __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFli
         f32x2 x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = pk_bits(w[i] * 65536u + f.lo[i], (w[i] ^ f.pair[i]) & 0xFFFF0000u);
+        const f32x2 zero2 = pk_bits(0u, 0u);
 #pragma unroll
         for (int h = 1; h < 16; h <<= 1) {
+            if (h == 8) {  // exact zero sums are +0 (see fwht16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = add2(x[i], zero2);
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 if ((i & h) == 0) {
@@ -266,6 +277,10 @@ __device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_
         }
 #pragma unroll
         for (int h = 1; h < 16; h <<= 1) {
+            if (h == 8) {  // exact zero sums are +0 (see fwht16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __fadd_rn(y[i], 0.0f);
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 if ((i & h) == 0) {
@@ -598,246 +613,319 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 }
 
 // ============================================================================
-// Tile kernel: a CTA loads a 64 x 128 bf16 tile once (registers + shared memory)
-// and writes the row orientation (from registers, one thread per 16-element row
-// block) and/or the column orientation (from shared memory, one thread per column
-// pair and 16-row chunk).  k2D: 16x16 blocks, the tile scale is found by the
+// Tile kernel (persistent).  A CTA walks 64 x 128 bf16 tiles -- tiles c, c + G,
+// c + 2G, ... of the G CTAs -- bottom row of tiles first, so the first tiles re-read
+// the rows the amax pass read last (still in L2).  A tile lands in one of
+// kTileStages shared-memory stages by 64 row copies (cp.async.bulk, one per row and
+// thread; a gathered row comes from its source row, a padding row is zero-filled),
+// issued kTileStages - 1 tiles ahead so that the loads of later tiles overlap the
+// arithmetic of this one.  From the stage the CTA writes the row orientation (one
+// thread per 16-element row block) and/or the column orientation (one thread per
+// column pair and 16-row chunk).  k2D: 16x16 blocks, the tile scale is found by the
 // column pass and shared by both orientations.  kRht: the 16-point RHT down each
-// column chunk before the column orientation is quantized.  Tiles run bottom-up,
-// so the first ones re-read the rows the amax pass read last (still in L2).
+// column chunk before the column orientation is quantized.  kRowRht: the row
+// orientation is rotated along each row block (the Mosaic recipe's dgrad operands).
+// kGrouped: the tile's rows lie in one group g (see QuantParams), which supplies the
+// tensor scales, the Philox key seed + g and the origin of the element indices.
 // ============================================================================
-constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;
+constexpr int kTR = 64, kTC = 128, kTileStages = 3;
 
-// Grouped (kGrouped): the tile's rows lie in one group g (see QuantParams), which
-// supplies the tensor scales, the Philox key seed + g and the origin of the
-// element indices.
-// kRowRht: the row orientation is rotated too (16-point RHT along each row block),
-// e.g. dgrad operands under the Mosaic recipe.
-// Resident CTAs per SM that the register budget is sized for.
-template <bool k2D, bool kRht, bool kGrouped>
-constexpr int quant_tile_min_blocks() {
-    return (kRht || k2D) ? 3 : 4;
+struct __align__(16) TileSmem {
+    uint16_t tile[kTileStages][kTR][kTC];  // dense 256-byte rows
+    float inv_tab[2][256];                  // element multipliers of every scale code: rows, columns
+    uint32_t tile_s[kTR / 16][kTC / 16];
+    float tile_inv[kTR / 16][kTC / 16];
+    // The tile's scales, staged so that they leave in wide stores (two buffers, by
+    // tile parity): the column orientation's 128 columns x 4 blocks are exactly one
+    // 512-byte atom; the row orientation's 64 rows x 8 blocks are 8 bytes of each of
+    // the 32 lines of two atoms.  Entries past the tensor hold 0 (the padding).
+    uint8_t col_atom[2][512];
+    uint8_t row_half_atoms[2][2][32][8];
+    uint64_t full[kTileStages];  // the stage's 64 rows have landed (64 arrivals + bytes)
+};
+
+__device__ __forceinline__ uint32_t s_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void s_mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void s_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Bounded wait for phase `parity` of a stage barrier (false after ~2^31 cycles).
+__device__ __forceinline__ bool s_mbar_wait(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred q;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > (1ll << 31)) return false;
+    }
+}
+
+// Thread t < 64 brings row t of `tile` into shared-memory stage `stage`, and arrives
+// on the stage's barrier once (expecting its bytes).  Rows past the tensor are not
+// written (their outputs are never stored); a gathered row with a negative source
+// index is written as zeros (the stores precede the arrival, which releases them);
+// columns past the tensor keep stale bytes (whole 16-column blocks, never stored).
+__device__ __forceinline__ void tile_row_fetch(const QuantParams& p, TileSmem& S, int64_t tile, int64_t ntx,
+                                               int64_t nty, int stage, int t) {
+    const int64_t r0 = (nty - 1 - tile / ntx) * kTR, c0 = (tile % ntx) * kTC;
+    const int64_t r = r0 + t;
+    uint16_t* dst = &S.tile[stage][t][0];
+    const uint32_t bar = s_addr(&S.full[stage]);
+    uint32_t bytes = 0;
+    int64_t src = r;
+    if (r < p.rows) {
+        if (p.row_src != nullptr) {
+            src = __ldg(p.row_src + r);
+            if (src >= p.src_rows) {
+                set_status(p.status, kStatusIndex);
+                src = -1;
+            }
+        }
+        if (src < 0) {
+#pragma unroll
+            for (int i = 0; i < kTC / 8; ++i) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
+        } else {
+            bytes = (uint32_t)((p.cols - c0 < kTC ? p.cols - c0 : kTC) * 2);
+        }
+    }
+    s_arrive_expect_tx(bar, bytes);
+    if (bytes)
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                s_addr(dst)),
+            "l"(p.x + src * p.cols + c0), "r"(bytes), "r"(bar)
+            : "memory");
 }
 
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
-__global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGrouped>()))
-    quant_tile_kernel(QuantParams p) {
-    __shared__ __align__(16) uint16_t tile[kTR][kPitch];
-    __shared__ float inv_tab[2][256];  // element multipliers of every scale code: rows, columns
-    __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
-    __shared__ float tile_inv[kTR / 16][kTC / 16];
-    // The tile's scales, staged so that they leave in wide stores instead of one
-    // byte each: the column orientation's 128 columns x 4 blocks are exactly one
-    // 512-byte atom; the row orientation's 64 rows x 8 blocks are 8 bytes of each
-    // of the 32 lines of two atoms.  Entries past the tensor hold 0 (the padding).
-    __shared__ __align__(16) uint8_t col_atom[512];
-    __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
-
+__global__ void __launch_bounds__(256, 2) quant_tile_kernel(const QuantParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    TileSmem& S = *reinterpret_cast<TileSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
-    TensorScale tr, tc;
-    int64_t g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
-    uint32_t rkg[20];                     // the group's Philox round keys
-    if (kGrouped) {
-        const int64_t g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
-        g_row0 = p.row_group ? p.group_row0[g] : g * p.group_rows_uniform;
-        g_rows = p.row_group ? p.group_nrows[g] : p.group_rows_uniform;
-        const uint32_t wr = p.amax_words[2 * g];
-        const uint32_t wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
-        const bool first = r0 == g_row0 && c0 == 0 && tid == 0;
-        if (!finite_bits(wr) || !finite_bits(wc)) {
-            if (first) {
-                set_status(p.status, kStatusNonFinite);
-                if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
-                if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
-            }
-            return;
-        }
-        tr = tensor_scale_from_amax(__uint_as_float(wr));
-        tc = tensor_scale_from_amax(__uint_as_float(wc));
-        if (first) {
-            if (p.row_g) p.row_g[g] = tr.g;
-            if (p.col_g) p.col_g[g] = tc.g;
-        }
-        uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
-#pragma unroll
-        for (int r = 0; r < 10; ++r) {
-            rkg[2 * r] = k0;
-            rkg[2 * r + 1] = k1;
-            k0 += 0x9E3779B9u;
-            k1 += 0xBB67AE85u;
-        }
-    } else {
-        if (!load_tensor_scales(p, tr, tc)) return;
-    }
-    const uint32_t (&rk)[20] = kGrouped ? rkg : p.rk;
+    const int64_t ntx = (p.cols + kTC - 1) / kTC, nty = (p.rows + kTR - 1) / kTR, ntiles = ntx * nty;
+    const int64_t G = gridDim.x;
     const bool want_row = p.row_data != nullptr;
     const bool want_col = p.col_data != nullptr;
-    const bool use_smem = want_col || k2D;
-    {
+
+    TensorScale tr{0.0f, 0.0f}, tc{0.0f, 0.0f};
+    auto fill_tables = [&]() {
         const float dec = e4m3_to_f32((uint32_t)tid);
         const float gr = __fmul_rn(dec, tr.g), gc = __fmul_rn(dec, tc.g);
-        inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gr), 3.402823466e38f);
-        inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gc), 3.402823466e38f);
-    }
-
-    // ---- load: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
-    const bool al32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0;
-    uint32_t rb[2][8];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int lr = (k * 256 + tid) >> 3, lc = (tid & 7) * 16;
-        const int64_t r = r0 + lr, c = c0 + lc;
-        bool in = r < p.rows && c < p.cols;
-        int64_t sr = r;
-        if (p.row_src != nullptr && in) {  // gathered rows
-            sr = __ldg(p.row_src + r);
-            if (sr >= p.src_rows) {
-                set_status(p.status, kStatusIndex);
-                in = false;
-            }
-            in = in && sr >= 0;
-        }
-        if (in) {
-            ld_block16(p.x + sr * p.cols + c, al32, rb[k]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) rb[k][i] = 0u;
-        }
-    }
-    __syncthreads();  // multiplier tables filled (the loads are still in flight)
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int lr = (k * 256 + tid) >> 3, lc = (tid & 7) * 16;
-        if (use_smem) {
-            // two 16-byte stores, the lane quads of a row taking the halves in opposite
-            // order so that eight lanes cover all 32 banks
-            const int h = (lane >> 2) & 1;
-            uint4* dst = reinterpret_cast<uint4*>(&tile[lr][lc]);
-            dst[h] = h ? make_uint4(rb[k][4], rb[k][5], rb[k][6], rb[k][7])
-                       : make_uint4(rb[k][0], rb[k][1], rb[k][2], rb[k][3]);
-            dst[h ^ 1] = h ? make_uint4(rb[k][0], rb[k][1], rb[k][2], rb[k][3])
-                           : make_uint4(rb[k][4], rb[k][5], rb[k][6], rb[k][7]);
-        }
-    }
-
-    // ---- row pass from registers: one thread per 16-element block
-    auto row_pass = [&]() {
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
-            const int64_t r = r0 + lr, c = c0 + lc;
-            uint32_t s;
-            float inv;
-            float v[16];
-            if (kRowRht) {
-                rht16_row(rb[k], p.sign_mask, v, p.status);
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                s = block_code(amax, tr);
-                inv = inv_tab[0][s];
-            } else if (k2D) {
-                s = tile_s[lr >> 4][bc];
-                inv = tile_inv[lr >> 4][bc];
-                unpack16(rb[k], v);
-            } else {
-                s = block_code(absmax16(rb[k]), tr);
-                inv = inv_tab[0][s];
-                unpack16(rb[k], v);
-            }
-            const uint2 codes =
-                encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
-            const bool inside = r < p.rows && c < p.cols;
-            if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
-            // (row lr, block bc): half-atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
-            row_half_atoms[bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)s : (uint8_t)0;
-        }
+        S.inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gr), 3.402823466e38f);
+        S.inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gc), 3.402823466e38f);
     };
-    if (want_row && !k2D) row_pass();
-    __syncthreads();  // tile in shared memory
-
-    // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunk j
-    if (use_smem) {
-        const int cp = tid & 63, j = tid >> 6;
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = *reinterpret_cast<const uint32_t*>(&tile[16 * j + i][2 * cp]);
-        float y0[16], y1[16];
-        if (kRht) {
-            rht16_pair(w, p.flips, p.sign_mask, y0, y1, p.status);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                y0[i] = bf16_lo(w[i]);
-                y1[i] = bf16_hi(w[i]);
-            }
-        }
-        float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            a0 = fmaxf(a0, fabsf(y0[i]));
-            a1 = fmaxf(a1, fabsf(y1[i]));
-        }
-        uint32_t s0, s1;
-        float inv0, inv1;
-        if (k2D) {
-            // the 16x16 tile: 8 consecutive lanes hold its 16 columns
-            float a = fmaxf(a0, a1);
-#pragma unroll
-            for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-            s0 = s1 = block_code(a, tc);
-            inv0 = inv1 = inv_tab[1][s0];
-            if ((cp & 7) == 0) {
-                tile_s[j][cp >> 3] = s0;
-                tile_inv[j][cp >> 3] = inv0;
-            }
-        } else {
-            s0 = block_code(a0, tc);
-            s1 = block_code(a1, tc);
-            inv0 = inv_tab[1][s0];
-            inv1 = inv_tab[1][s1];
-        }
-        if (want_col) {
-            const bool rin = r0 + 16 * j < p.rows;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int lc = 2 * cp + h;
-                const int64_t c = c0 + lc;
-                const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
-                const uint2 codes = encode16(h ? y1 : y0, h ? inv1 : inv0, p.col_sr, rk, 1u, e0);
-                const bool inside = c < p.cols && rin;
-                if (inside)
-                    *reinterpret_cast<uint2*>(p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j) >> 1)) = codes;
-                // atom byte of (column lc, block j): line lc % 32, group lc / 32
-                col_atom[(lc & 31) * 16 + (lc >> 5) * 4 + j] = inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
-            }
-        }
+    if (!kGrouped) {
+        if (!load_tensor_scales(p, tr, tc)) return;  // every CTA returns: nothing issued yet
+        fill_tables();
     }
-    if (want_row && k2D) {
-        __syncthreads();  // tile scales written
-        row_pass();
+    if (tid == 0) {
+        for (int s = 0; s < kTileStages; ++s) s_mbar_init(s_addr(&S.full[s]), 64);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-
-    // ---- scale stores.  Every entry written lies inside the scale buffer: the
-    // column atom is (128-column group c0 / 128, blocks r0 / 16 .. + 3) with r0 a
-    // multiple of 64 below the rows; the row half-atoms cover 64 rows below
-    // pad128(rows), and the second is skipped when its blocks start past the
-    // padded block count.
     __syncthreads();
-    if (want_col && warp == 0) {
-        const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
-        const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
-        *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) =
-            *reinterpret_cast<const uint4*>(col_atom + lane * 16);
-    }
-    if (want_row && (warp == 2 || warp == 3)) {
-        const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
-        const int a = warp - 2;
-        if ((c0 >> 6) + a < katoms_r) {
-            const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
-            *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
-                *reinterpret_cast<const uint2*>(row_half_atoms[a][lane]);
+    if (tid < 64)
+        for (int j = 0; j < kTileStages; ++j)
+            if (blockIdx.x + (int64_t)j * G < ntiles) tile_row_fetch(p, S, blockIdx.x + (int64_t)j * G, ntx, nty, j, tid);
+
+    int64_t cur_group = -1, g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
+    bool group_ok = true;
+    uint32_t rkg[20];  // the group's Philox round keys
+    for (int64_t i = 0, tile = blockIdx.x; tile < ntiles; ++i, tile += G) {
+        const int s = (int)(i % kTileStages), par = (int)((i / kTileStages) & 1), ab = (int)(i & 1);
+        const int64_t r0 = (nty - 1 - tile / ntx) * kTR, c0 = (tile % ntx) * kTC;
+        if (kGrouped) {
+            const int64_t g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
+            if (g != cur_group) {  // the same for every thread of the CTA
+                cur_group = g;
+                g_row0 = p.row_group ? p.group_row0[g] : g * p.group_rows_uniform;
+                g_rows = p.row_group ? p.group_nrows[g] : p.group_rows_uniform;
+                const uint32_t wr = p.amax_words[2 * g];
+                const uint32_t wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
+                group_ok = finite_bits(wr) && finite_bits(wc);
+                const bool first = r0 == g_row0 && c0 == 0 && tid == 0;
+                if (!group_ok) {
+                    if (first) {
+                        set_status(p.status, kStatusNonFinite);
+                        if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
+                        if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
+                    }
+                } else {
+                    tr = tensor_scale_from_amax(__uint_as_float(wr));
+                    tc = tensor_scale_from_amax(__uint_as_float(wc));
+                    if (first) {
+                        if (p.row_g) p.row_g[g] = tr.g;
+                        if (p.col_g) p.col_g[g] = tc.g;
+                    }
+                    uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
+#pragma unroll
+                    for (int r = 0; r < 10; ++r) {
+                        rkg[2 * r] = k0;
+                        rkg[2 * r + 1] = k1;
+                        k0 += 0x9E3779B9u;
+                        k1 += 0xBB67AE85u;
+                    }
+                    fill_tables();
+                }
+                __syncthreads();  // tables of the new group written (the last tile's readers are done)
+            }
+        }
+        const uint32_t (&rkc)[20] = rkg;
+        const uint32_t (&rk)[20] = kGrouped ? rkc : p.rk;
+        const bool landed = s_mbar_wait(s_addr(&S.full[s]), (uint32_t)par);
+        const bool work = !kGrouped || group_ok;
+        const uint16_t (&T)[kTR][kTC] = S.tile[s];
+
+        // ---- row pass: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
+        auto row_pass = [&]() {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
+                const int64_t r = r0 + lr, c = c0 + lc;
+                // two 16-byte reads, the lane quads of a row taking the halves in opposite
+                // order so that eight lanes cover all 32 banks
+                const int h = (lane >> 2) & 1;
+                const uint4* src = reinterpret_cast<const uint4*>(&T[lr][lc]);
+                const uint4 q0 = src[h], q1 = src[h ^ 1];
+                const uint4 lo = h ? q1 : q0, hi = h ? q0 : q1;
+                const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                uint32_t sc;
+                float inv;
+                float v[16];
+                if (kRowRht) {
+                    rht16_row(w, p.sign_mask, v, p.status);
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+                    sc = block_code(amax, tr);
+                    inv = S.inv_tab[0][sc];
+                } else if (k2D) {
+                    sc = S.tile_s[lr >> 4][bc];
+                    inv = S.tile_inv[lr >> 4][bc];
+                    unpack16(w, v);
+                } else {
+                    sc = block_code(absmax16(w), tr);
+                    inv = S.inv_tab[0][sc];
+                    unpack16(w, v);
+                }
+                const uint2 codes =
+                    encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
+                const bool inside = r < p.rows && c < p.cols;
+                if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
+                // (row lr, block bc): half-atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
+                S.row_half_atoms[ab][bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)sc : (uint8_t)0;
+            }
+        };
+
+        if (work) {
+            if (want_row && !k2D) row_pass();
+            // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunk j
+            if (want_col || k2D) {
+                const int cp = tid & 63, j = tid >> 6;
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = *reinterpret_cast<const uint32_t*>(&T[16 * j + e][2 * cp]);
+                float y0[16], y1[16];
+                if (kRht) {
+                    rht16_pair(w, p.flips, p.sign_mask, y0, y1, p.status);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        y0[e] = bf16_lo(w[e]);
+                        y1[e] = bf16_hi(w[e]);
+                    }
+                }
+                float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    a0 = fmaxf(a0, fabsf(y0[e]));
+                    a1 = fmaxf(a1, fabsf(y1[e]));
+                }
+                uint32_t s0, s1;
+                float inv0, inv1;
+                if (k2D) {
+                    // the 16x16 tile: 8 consecutive lanes hold its 16 columns
+                    float a = fmaxf(a0, a1);
+#pragma unroll
+                    for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+                    s0 = s1 = block_code(a, tc);
+                    inv0 = inv1 = S.inv_tab[1][s0];
+                    if ((cp & 7) == 0) {
+                        S.tile_s[j][cp >> 3] = s0;
+                        S.tile_inv[j][cp >> 3] = inv0;
+                    }
+                } else {
+                    s0 = block_code(a0, tc);
+                    s1 = block_code(a1, tc);
+                    inv0 = S.inv_tab[1][s0];
+                    inv1 = S.inv_tab[1][s1];
+                }
+                if (want_col) {
+                    const bool rin = r0 + 16 * j < p.rows;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int lc = 2 * cp + h;
+                        const int64_t c = c0 + lc;
+                        const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
+                        const uint2 codes = encode16(h ? y1 : y0, h ? inv1 : inv0, p.col_sr, rk, 1u, e0);
+                        const bool inside = c < p.cols && rin;
+                        if (inside)
+                            *reinterpret_cast<uint2*>(p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j) >> 1)) = codes;
+                        // atom byte of (column lc, block j): line lc % 32, group lc / 32
+                        S.col_atom[ab][(lc & 31) * 16 + (lc >> 5) * 4 + j] =
+                            inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
+                    }
+                }
+            }
+            if (want_row && k2D) {
+                __syncthreads();  // tile scales written
+                row_pass();
+            }
+        } else if (k2D && want_row) {
+            __syncthreads();  // keep the barrier count of the k2D path
+        }
+
+        // the stage has been read and the tile's scales staged
+        if (__syncthreads_or(!landed)) {
+            // a copy did not land within the bound: record it, wait (bounded) for this
+            // CTA's copies still in flight, and stop
+            for (int64_t k = 0; k < kTileStages; ++k) {
+                const int64_t ii = i + k;
+                if (tile + k * G < ntiles) s_mbar_wait(s_addr(&S.full[ii % kTileStages]), (uint32_t)((ii / kTileStages) & 1));
+            }
+            if (tid == 0) set_status(p.status, kStatusTimeout);
+            return;
+        }
+        if (tid < 64 && tile + kTileStages * G < ntiles) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the reads above precede the refill
+            tile_row_fetch(p, S, tile + kTileStages * G, ntx, nty, s, tid);
+        }
+        // ---- scale stores.  Every entry written lies inside the scale buffer: the
+        // column atom is (128-column group c0 / 128, blocks r0 / 16 .. + 3) with r0 a
+        // multiple of 64 below the rows; the row half-atoms cover 64 rows below
+        // pad128(rows), and the second is skipped when its blocks start past the
+        // padded block count.
+        if (work && want_col && warp == 0) {
+            const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
+            const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
+            *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) =
+                *reinterpret_cast<const uint4*>(S.col_atom[ab] + lane * 16);
+        }
+        if (work && want_row && (warp == 2 || warp == 3)) {
+            const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
+            const int a = warp - 2;
+            if ((c0 >> 6) + a < katoms_r) {
+                const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
+                *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
+                    *reinterpret_cast<const uint2*>(S.row_half_atoms[ab][a][lane]);
+            }
         }
     }
 }
@@ -1086,32 +1174,40 @@ cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStrea
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, cudaStream_t st) {
+template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
+static cudaError_t launch_tile(const QuantParams& p, int sm_count, cudaStream_t st) {
+    constexpr size_t smem = sizeof(TileSmem) + 128;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<k2D, kRht, kGrouped, kRowRht>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int64_t tiles = ((p.cols + kTC - 1) / kTC) * ((p.rows + kTR - 1) / kTR);
+    const int64_t cap = 2 * (int64_t)sm_count;  // persistent: two CTAs per SM
+    const unsigned grid = (unsigned)(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
+    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, int sm_count, cudaStream_t st) {
     QuantParams p = params;
     philox_round_keys(p.seed, p.rk);
     rht_flips(p.sign_mask, p.flips);
-    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
     const bool grouped = p.row_group != nullptr || p.group_rows_uniform > 0;
     if (p.row_rht && (grouped || two_d)) return cudaErrorInvalidValue;
     const bool col_rht = p.col_rht && p.col_data;
     if (grouped) {
-        if (two_d)
-            quant_tile_kernel<true, false, true, false><<<grid, 256, 0, st>>>(p);
-        else if (col_rht)
-            quant_tile_kernel<false, true, true, false><<<grid, 256, 0, st>>>(p);
-        else
-            quant_tile_kernel<false, false, true, false><<<grid, 256, 0, st>>>(p);
-    } else if (two_d)
-        quant_tile_kernel<true, false, false, false><<<grid, 256, 0, st>>>(p);
-    else if (p.row_rht && col_rht)
-        quant_tile_kernel<false, true, false, true><<<grid, 256, 0, st>>>(p);
-    else if (p.row_rht)
-        quant_tile_kernel<false, false, false, true><<<grid, 256, 0, st>>>(p);
-    else if (col_rht)
-        quant_tile_kernel<false, true, false, false><<<grid, 256, 0, st>>>(p);
-    else
-        quant_tile_kernel<false, false, false, false><<<grid, 256, 0, st>>>(p);
-    return cudaGetLastError();
+        if (two_d) return launch_tile<true, false, true, false>(p, sm_count, st);
+        if (col_rht) return launch_tile<false, true, true, false>(p, sm_count, st);
+        return launch_tile<false, false, true, false>(p, sm_count, st);
+    }
+    if (two_d) return launch_tile<true, false, false, false>(p, sm_count, st);
+    if (p.row_rht && col_rht) return launch_tile<false, true, false, true>(p, sm_count, st);
+    if (p.row_rht) return launch_tile<false, false, false, true>(p, sm_count, st);
+    if (col_rht) return launch_tile<false, true, false, false>(p, sm_count, st);
+    return launch_tile<false, false, false, false>(p, sm_count, st);
 }
 
 cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st) {

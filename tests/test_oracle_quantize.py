@@ -288,6 +288,23 @@ def test_row_rht_dense_product(ora):
     assert np.array_equal(ye[1, 16:], (s[5] * H[5]).astype(np.float32))
 
 
+def test_rht_exact_zero_is_positive_zero(ora):
+    """Reading R7: the transform is the fp32 rounding of the exact sum, and an exact
+    sum of zero is the real number 0, stored as +0 whatever the input signs (zero
+    inputs, -0 inputs, negative rotation signs, or nonzero inputs that cancel)."""
+    s = np.array([-1, 1] * 8, dtype=np.int8)
+    x = np.zeros((4, 16), np.uint16)
+    x[1, :] = 0x8000                       # -0 everywhere
+    x[2, 0], x[2, 1] = 0x3F80, 0x3F80      # 1, 1 with signs -1, +1: cancels in half the outputs
+    x[3, 8] = 0xC000                       # one -2, the rest +0
+    y = ora.rht(x, 1, s)
+    H = scipy.linalg.hadamard(16).astype(np.float64)
+    exact = (syn.bf16_bits_to_f32(x).astype(np.float64) * s) @ H
+    assert np.array_equal(y, exact.astype(np.float32))
+    zero = exact == 0
+    assert zero.any() and (y.view(np.uint32)[zero] == 0).all()   # +0, never -0
+
+
 def test_row_rht_amax_is_max_of_standalone_rht(ora):
     x = syn.normal_bf16((32, 96), 22)
     s = syn.rht_signs(4)
