@@ -73,6 +73,37 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
     asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
+__device__ __forceinline__ uint32_t vmax_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Largest and smallest magnitude of bf16 values, per 16-bit lane of packed words,
+// from four full-rate packed min/max (no masking per word).  A sign-magnitude
+// pattern compares as unsigned by (sign, magnitude) and as signed with the negative
+// magnitudes reversed, so the unsigned maximum holds the largest negative magnitude
+// (or, with no negative value, the largest positive one) and the signed maximum the
+// largest positive magnitude (or, with no nonnegative value, the largest negative
+// one): their magnitudes' maximum is the largest magnitude.  Likewise the minima.
+template <int N>
+__device__ __forceinline__ void chunk_mag_stats(const uint32_t (&w)[N], uint32_t& mx, uint32_t& mn) {
+    uint32_t umax = 0u, smax = 0x80008000u, umin = 0xFFFFFFFFu, smin = 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        umax = vmax_u16x2(umax, w[i]);
+        smax = vmax_s16x2(smax, w[i]);
+        umin = vmin_u16x2(umin, w[i]);
+        smin = vmin_s16x2(smin, w[i]);
+    }
+    mx = vmax_u16x2(umax & 0x7FFF7FFFu, smax & 0x7FFF7FFFu);
+    mn = vmin_u16x2(umin & 0x7FFF7FFFu, smin & 0x7FFF7FFFu);
+}
 
 // 32-byte streaming load (16 bf16) of data read once; `p` 32-byte aligned.
 __device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&r)[8]) {
@@ -135,6 +166,16 @@ __device__ __forceinline__ double bf16_signed_to_f64(uint32_t bits16, uint32_t f
     return (double)__uint_as_float((bits16 ^ (flip << 15)) << 16);
 }
 
+// The exponent-span test above on one lane of chunk_mag_stats: mx and mn are the
+// largest and smallest magnitude (bf16 patterns without sign).  A chunk holding a
+// zero beside nonzero values (mn == 0) takes the fp64 path, which needs no span.
+__device__ __forceinline__ bool span_ok_mag(uint32_t mx, uint32_t mn) {
+    if (mx == 0u) return true;  // all inputs zero
+    if (mn == 0u) return false;
+    const int emax = (int)(mx >> 7), emin = (int)(mn >> 7);
+    return emax <= 251 && emax - max(emin, 1) <= 13;
+}
+
 // The exponent-span test above for one 16-bit lane of the chunk statistics: with
 // v = |x| + 0x7FFF per bf16 (0x7FFF for a zero, >= 0x8000 otherwise), vmx is the
 // unsigned maximum of v and vmn its signed minimum (the smallest nonzero |x|).
@@ -186,9 +227,9 @@ __device__ __forceinline__ void rht16_col_f64(const uint32_t (&w)[16], int half,
 // the low half).  y0 / y1 receive the transforms of the two columns.
 __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFlips& f, uint32_t sign_mask,
                                            float (&y0)[16], float (&y1)[16], int* status = nullptr) {
-    uint32_t vmx, vmn;
-    chunk_stats<16>(w, vmx, vmn);
-    if (span_ok(vmx & 0xFFFFu, vmn & 0xFFFFu) && span_ok(vmx >> 16, vmn >> 16)) {
+    uint32_t mx, mn;
+    chunk_mag_stats<16>(w, mx, mn);
+    if (span_ok_mag(mx & 0xFFFFu, mn & 0xFFFFu) && span_ok_mag(mx >> 16, mn >> 16)) {
         f32x2 x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = pk_bits(w[i] * 65536u + f.lo[i], (w[i] ^ f.pair[i]) & 0xFFFF0000u);
@@ -211,6 +252,8 @@ __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFli
 #pragma unroll
         for (int i = 0; i < 16; ++i) unpk(x[i], y0[i], y1[i]);
     } else {
+        uint32_t vmx, vmn;
+        chunk_stats<16>(w, vmx, vmn);
         note_f64_domain(vmx & 0xFFFFu, vmn & 0xFFFFu, status);
         note_f64_domain(vmx >> 16, vmn >> 16, status);
         rht16_col_f64(w, 0, sign_mask, y0);
@@ -222,10 +265,10 @@ __device__ __forceinline__ void rht16_pair(const uint32_t (&w)[16], const RhtFli
 // is not formed: max(|RN(a+b)|, |RN(a-b)|) = RN(|a| + |b|) exactly (RN is monotone
 // and odd, and max(|a+b|, |a-b|) = |a| + |b|).
 __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], const RhtFlips& f,
-                                                   uint32_t sign_mask, uint32_t vmx, uint32_t vmn,
+                                                   uint32_t sign_mask, uint32_t mx, uint32_t mn,
                                                    int* status) {
     float m = 0.0f;
-    if (span_ok(vmx & 0xFFFFu, vmn & 0xFFFFu) && span_ok(vmx >> 16, vmn >> 16)) {
+    if (span_ok_mag(mx & 0xFFFFu, mn & 0xFFFFu) && span_ok_mag(mx >> 16, mn >> 16)) {
         f32x2 x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = pk_bits(w[i] * 65536u + f.lo[i], (w[i] ^ f.pair[i]) & 0xFFFF0000u);
@@ -248,6 +291,8 @@ __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], cons
             m = fmaxf(m, fmaxf(fabsf(a0) + fabsf(b0), fabsf(a1) + fabsf(b1)));
         }
     } else {
+        uint32_t vmx, vmn;
+        chunk_stats<16>(w, vmx, vmn);
         note_f64_domain(vmx & 0xFFFFu, vmn & 0xFFFFu, status);
         note_f64_domain(vmx >> 16, vmn >> 16, status);
         float y[16];
@@ -265,11 +310,9 @@ __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], cons
 // block (16 values).  Scalar fp32 butterfly under the same span test, else fp64.
 __device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_mask, float (&y)[16],
                                           int* status = nullptr) {
-    uint32_t vmx, vmn;
-    chunk_stats<8>(w, vmx, vmn);
-    const uint32_t mx = max(vmx & 0xFFFFu, vmx >> 16);
-    const uint32_t mn = (uint32_t)(uint16_t)min((int16_t)(vmn & 0xFFFFu), (int16_t)(vmn >> 16));
-    if (span_ok(mx, mn)) {
+    uint32_t mx2, mn2;
+    chunk_mag_stats<8>(w, mx2, mn2);
+    if (span_ok_mag(max(mx2 & 0xFFFFu, mx2 >> 16), min(mn2 & 0xFFFFu, mn2 >> 16))) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const uint32_t b = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
@@ -291,7 +334,10 @@ __device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_
             }
         }
     } else {
-        note_f64_domain(mx, mn, status);
+        uint32_t vmx, vmn;
+        chunk_stats<8>(w, vmx, vmn);
+        note_f64_domain(max(vmx & 0xFFFFu, vmx >> 16),
+                        (uint32_t)(uint16_t)min((int16_t)(vmn & 0xFFFFu), (int16_t)(vmn >> 16)), status);
         double d[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -402,10 +448,10 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) w[i] = c == 0 ? v[i].x : c == 1 ? v[i].y : c == 2 ? v[i].z : v[i].w;
-                uint32_t vmx, vmn;
-                chunk_stats<16>(w, vmx, vmn);
-                m_row = vmax_u16x2(m_row, vmx - 0x7FFF7FFFu);
-                m_col = fmaxf(m_col, rht16_pair_absmax(w, flips, sign_mask, vmx, vmn, status));
+                uint32_t mx, mn;
+                chunk_mag_stats<16>(w, mx, mn);
+                m_row = vmax_u16x2(m_row, mx);
+                m_col = fmaxf(m_col, rht16_pair_absmax(w, flips, sign_mask, mx, mn, status));
             }
         } else {
 #pragma unroll
@@ -553,10 +599,16 @@ __device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float (&v)[16])
     }
 }
 
+// max |x| of a 16-element block (two full-rate packed maxima per word, see
+// chunk_mag_stats); NaN patterns sort above Inf.
 __device__ __forceinline__ float absmax16(const uint32_t (&w)[8]) {
-    uint32_t m = 0u;
+    uint32_t u = 0u, sg = 0x80008000u;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) m = vmax_u16x2(m, w[k] & 0x7FFF7FFFu);
+    for (int k = 0; k < 8; ++k) {
+        u = vmax_u16x2(u, w[k]);
+        sg = vmax_s16x2(sg, w[k]);
+    }
+    const uint32_t m = vmax_u16x2(u & 0x7FFF7FFFu, sg & 0x7FFF7FFFu);
     return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
 }
 
@@ -613,319 +665,264 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 }
 
 // ============================================================================
-// Tile kernel (persistent).  A CTA walks 64 x 128 bf16 tiles -- tiles c, c + G,
-// c + 2G, ... of the G CTAs -- bottom row of tiles first, so the first tiles re-read
-// the rows the amax pass read last (still in L2).  A tile lands in one of
-// kTileStages shared-memory stages by 64 row copies (cp.async.bulk, one per row and
-// thread; a gathered row comes from its source row, a padding row is zero-filled),
-// issued kTileStages - 1 tiles ahead so that the loads of later tiles overlap the
-// arithmetic of this one.  From the stage the CTA writes the row orientation (one
-// thread per 16-element row block) and/or the column orientation (one thread per
-// column pair and 16-row chunk).  k2D: 16x16 blocks, the tile scale is found by the
+// Tile kernel: a CTA quantizes one 64 x 128 bf16 tile.  The tile goes straight
+// from global to shared memory (cp.async, 16 bytes per copy, four per thread; rows
+// and columns past the tensor and gathered padding rows are zero-filled by the copy
+// itself), so no register holds it in flight.  Then one thread per 16-element row
+// block writes the row orientation, and one thread per column pair and 16-row chunk
+// writes the column orientation.  k2D: 16x16 blocks, the tile scale is found by the
 // column pass and shared by both orientations.  kRht: the 16-point RHT down each
 // column chunk before the column orientation is quantized.  kRowRht: the row
 // orientation is rotated along each row block (the Mosaic recipe's dgrad operands).
 // kGrouped: the tile's rows lie in one group g (see QuantParams), which supplies the
 // tensor scales, the Philox key seed + g and the origin of the element indices.
+// Tiles run bottom-up (the grid's y extent reversed), so the first tiles re-read the
+// rows the amax pass read last (still in L2).
 // ============================================================================
-constexpr int kTR = 64, kTC = 128, kTileStages = 3;
+constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;  // +16 bytes per row: conflict-free column reads
 
-struct __align__(16) TileSmem {
-    uint16_t tile[kTileStages][kTR][kTC];  // dense 256-byte rows
-    float inv_tab[2][256];                  // element multipliers of every scale code: rows, columns
-    uint32_t tile_s[kTR / 16][kTC / 16];
-    float tile_inv[kTR / 16][kTC / 16];
-    // The tile's scales, staged so that they leave in wide stores (two buffers, by
-    // tile parity): the column orientation's 128 columns x 4 blocks are exactly one
-    // 512-byte atom; the row orientation's 64 rows x 8 blocks are 8 bytes of each of
-    // the 32 lines of two atoms.  Entries past the tensor hold 0 (the padding).
-    uint8_t col_atom[2][512];
-    uint8_t row_half_atoms[2][2][32][8];
-    uint64_t full[kTileStages];  // the stage's 64 rows have landed (64 arrivals + bytes)
-};
-
-__device__ __forceinline__ uint32_t s_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void s_mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void s_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-// Bounded wait for phase `parity` of a stage barrier (false after ~2^31 cycles).
-__device__ __forceinline__ bool s_mbar_wait(uint32_t bar, uint32_t parity) {
-    const long long t0 = clock64();
-    for (;;) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred q;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, q;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if (clock64() - t0 > (1ll << 31)) return false;
-    }
+// 16-byte copy global -> shared, `src_bytes` of it read (the rest zero-filled).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
 }
 
-// Thread t < 64 brings row t of `tile` into shared-memory stage `stage`, and arrives
-// on the stage's barrier once (expecting its bytes).  Rows past the tensor are not
-// written (their outputs are never stored); a gathered row with a negative source
-// index is written as zeros (the stores precede the arrival, which releases them);
-// columns past the tensor keep stale bytes (whole 16-column blocks, never stored).
-__device__ __forceinline__ void tile_row_fetch(const QuantParams& p, TileSmem& S, int64_t tile, int64_t ntx,
-                                               int64_t nty, int stage, int t) {
-    const int64_t r0 = (nty - 1 - tile / ntx) * kTR, c0 = (tile % ntx) * kTC;
-    const int64_t r = r0 + t;
-    uint16_t* dst = &S.tile[stage][t][0];
-    const uint32_t bar = s_addr(&S.full[stage]);
-    uint32_t bytes = 0;
-    int64_t src = r;
-    if (r < p.rows) {
-        if (p.row_src != nullptr) {
-            src = __ldg(p.row_src + r);
-            if (src >= p.src_rows) {
-                set_status(p.status, kStatusIndex);
-                src = -1;
-            }
-        }
-        if (src < 0) {
-#pragma unroll
-            for (int i = 0; i < kTC / 8; ++i) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
-        } else {
-            bytes = (uint32_t)((p.cols - c0 < kTC ? p.cols - c0 : kTC) * 2);
-        }
-    }
-    s_arrive_expect_tx(bar, bytes);
-    if (bytes)
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                s_addr(dst)),
-            "l"(p.x + src * p.cols + c0), "r"(bytes), "r"(bar)
-            : "memory");
+// Resident CTAs per SM the register budget is sized for (each CTA quantizes one tile,
+// so more resident CTAs keep more copies and more independent arithmetic in flight).
+template <bool k2D, bool kRht, bool kGrouped>
+constexpr int quant_tile_min_blocks() {
+    return (kRht && kGrouped) ? 3 : 4;
 }
 
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
-__global__ void __launch_bounds__(256, 2) quant_tile_kernel(const QuantParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    TileSmem& S = *reinterpret_cast<TileSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+__global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGrouped>()))
+    quant_tile_kernel(const QuantParams p) {
+    __shared__ __align__(16) uint16_t tile[kTR][kPitch];
+    __shared__ float inv_tab[2][256];  // element multipliers of every scale code: rows, columns
+    __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
+    __shared__ float tile_inv[kTR / 16][kTC / 16];
+    // The tile's scales, staged so that they leave in wide stores instead of one
+    // byte each: the column orientation's 128 columns x 4 blocks are exactly one
+    // 512-byte atom; the row orientation's 64 rows x 8 blocks are 8 bytes of each
+    // of the 32 lines of two atoms.  Entries past the tensor hold 0 (the padding).
+    __shared__ __align__(16) uint8_t col_atom[512];
+    __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
+
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t ntx = (p.cols + kTC - 1) / kTC, nty = (p.rows + kTR - 1) / kTR, ntiles = ntx * nty;
-    const int64_t G = gridDim.x;
-    const bool want_row = p.row_data != nullptr;
-    const bool want_col = p.col_data != nullptr;
+    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
+
+    // ---- copies first (they do not depend on the scales): 1024 x 16 bytes, four per
+    // thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int q = k * 256 + tid;
+        const int lr = q >> 4, lc = (q & 15) * 8;
+        const int64_t r = r0 + lr, c = c0 + lc;
+        int64_t sr = r;
+        bool in = r < p.rows && c < p.cols;
+        if (p.row_src != nullptr && in) {  // gathered rows
+            sr = __ldg(p.row_src + r);
+            if (sr >= p.src_rows) {
+                set_status(p.status, kStatusIndex);
+                in = false;
+            }
+            in = in && sr >= 0;
+        }
+        cp_async16(&tile[lr][lc], in ? (const void*)(p.x + sr * p.cols + c) : (const void*)p.x, in ? 16u : 0u);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
 
     TensorScale tr{0.0f, 0.0f}, tc{0.0f, 0.0f};
-    auto fill_tables = [&]() {
+    int64_t g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
+    uint32_t rkg[20];                     // the group's Philox round keys
+    bool ok = true;
+    if (kGrouped) {
+        const int64_t g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
+        g_row0 = p.row_group ? p.group_row0[g] : g * p.group_rows_uniform;
+        g_rows = p.row_group ? p.group_nrows[g] : p.group_rows_uniform;
+        const uint32_t wr = p.amax_words[2 * g];
+        const uint32_t wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
+        const bool first = r0 == g_row0 && c0 == 0 && tid == 0;
+        ok = finite_bits(wr) && finite_bits(wc);
+        if (!ok) {
+            if (first) {
+                set_status(p.status, kStatusNonFinite);
+                if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
+                if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
+            }
+        } else {
+            tr = tensor_scale_from_amax(__uint_as_float(wr));
+            tc = tensor_scale_from_amax(__uint_as_float(wc));
+            if (first) {
+                if (p.row_g) p.row_g[g] = tr.g;
+                if (p.col_g) p.col_g[g] = tc.g;
+            }
+            uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
+#pragma unroll
+            for (int r = 0; r < 10; ++r) {
+                rkg[2 * r] = k0;
+                rkg[2 * r + 1] = k1;
+                k0 += 0x9E3779B9u;
+                k1 += 0xBB67AE85u;
+            }
+        }
+    } else {
+        ok = load_tensor_scales(p, tr, tc);
+    }
+    if (!ok) {  // the same for the whole CTA; let the copies land before leaving
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        return;
+    }
+    const uint32_t (&rkc)[20] = rkg;
+    const uint32_t (&rk)[20] = kGrouped ? rkc : p.rk;
+    const bool want_row = p.row_data != nullptr;
+    const bool want_col = p.col_data != nullptr;
+    {
         const float dec = e4m3_to_f32((uint32_t)tid);
         const float gr = __fmul_rn(dec, tr.g), gc = __fmul_rn(dec, tc.g);
-        S.inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gr), 3.402823466e38f);
-        S.inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gc), 3.402823466e38f);
+        inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gr), 3.402823466e38f);
+        inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gc), 3.402823466e38f);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();  // tile and tables in shared memory
+
+    // ---- row pass: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
+    auto row_pass = [&]() {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
+            const int64_t r = r0 + lr, c = c0 + lc;
+            // two 16-byte reads, the lane quads of a row taking the halves in opposite
+            // order so that eight lanes cover all 32 banks
+            const int h = (lane >> 2) & 1;
+            const uint4* src = reinterpret_cast<const uint4*>(&tile[lr][lc]);
+            const uint4 q0 = src[h], q1 = src[h ^ 1];
+            const uint4 lo = h ? q1 : q0, hi = h ? q0 : q1;
+            const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            const bool inside = r < p.rows && c < p.cols;
+            uint32_t sc;
+            float inv;
+            float v[16];
+            if (kRowRht) {
+                rht16_row(w, p.sign_mask, v, inside ? p.status : nullptr);
+                float amax = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+                sc = block_code(amax, tr);
+                inv = inv_tab[0][sc];
+            } else if (k2D) {
+                sc = tile_s[lr >> 4][bc];
+                inv = tile_inv[lr >> 4][bc];
+                unpack16(w, v);
+            } else {
+                sc = block_code(absmax16(w), tr);
+                inv = inv_tab[0][sc];
+                unpack16(w, v);
+            }
+            const uint2 codes =
+                encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
+            if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
+            // (row lr, block bc): half-atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
+            row_half_atoms[bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)sc : (uint8_t)0;
+        }
     };
-    if (!kGrouped) {
-        if (!load_tensor_scales(p, tr, tc)) return;  // every CTA returns: nothing issued yet
-        fill_tables();
-    }
-    if (tid == 0) {
-        for (int s = 0; s < kTileStages; ++s) s_mbar_init(s_addr(&S.full[s]), 64);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    if (tid < 64)
-        for (int j = 0; j < kTileStages; ++j)
-            if (blockIdx.x + (int64_t)j * G < ntiles) tile_row_fetch(p, S, blockIdx.x + (int64_t)j * G, ntx, nty, j, tid);
+    if (want_row && !k2D) row_pass();
 
-    int64_t cur_group = -1, g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
-    bool group_ok = true;
-    uint32_t rkg[20];  // the group's Philox round keys
-    for (int64_t i = 0, tile = blockIdx.x; tile < ntiles; ++i, tile += G) {
-        const int s = (int)(i % kTileStages), par = (int)((i / kTileStages) & 1), ab = (int)(i & 1);
-        const int64_t r0 = (nty - 1 - tile / ntx) * kTR, c0 = (tile % ntx) * kTC;
-        if (kGrouped) {
-            const int64_t g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
-            if (g != cur_group) {  // the same for every thread of the CTA
-                cur_group = g;
-                g_row0 = p.row_group ? p.group_row0[g] : g * p.group_rows_uniform;
-                g_rows = p.row_group ? p.group_nrows[g] : p.group_rows_uniform;
-                const uint32_t wr = p.amax_words[2 * g];
-                const uint32_t wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
-                group_ok = finite_bits(wr) && finite_bits(wc);
-                const bool first = r0 == g_row0 && c0 == 0 && tid == 0;
-                if (!group_ok) {
-                    if (first) {
-                        set_status(p.status, kStatusNonFinite);
-                        if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
-                        if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
-                    }
-                } else {
-                    tr = tensor_scale_from_amax(__uint_as_float(wr));
-                    tc = tensor_scale_from_amax(__uint_as_float(wc));
-                    if (first) {
-                        if (p.row_g) p.row_g[g] = tr.g;
-                        if (p.col_g) p.col_g[g] = tc.g;
-                    }
-                    uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
+    // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunk j
+    if (want_col || k2D) {
+        const int cp = tid & 63, j = tid >> 6;
+        uint32_t w[16];
 #pragma unroll
-                    for (int r = 0; r < 10; ++r) {
-                        rkg[2 * r] = k0;
-                        rkg[2 * r + 1] = k1;
-                        k0 += 0x9E3779B9u;
-                        k1 += 0xBB67AE85u;
-                    }
-                    fill_tables();
-                }
-                __syncthreads();  // tables of the new group written (the last tile's readers are done)
+        for (int e = 0; e < 16; ++e) w[e] = *reinterpret_cast<const uint32_t*>(&tile[16 * j + e][2 * cp]);
+        const bool rin = r0 + 16 * j < p.rows;
+        const bool chunk_in = c0 + 2 * cp < p.cols && rin;
+        float a0 = 0.0f, a1 = 0.0f;
+        float y0[16], y1[16];
+        if (kRht) {
+            rht16_pair(w, p.flips, p.sign_mask, y0, y1, chunk_in ? p.status : nullptr);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                a0 = fmaxf(a0, fabsf(y0[e]));
+                a1 = fmaxf(a1, fabsf(y1[e]));
             }
+        } else {
+            uint32_t u = 0u, sg = 0x80008000u;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                u = vmax_u16x2(u, w[e]);
+                sg = vmax_s16x2(sg, w[e]);
+            }
+            const uint32_t m = vmax_u16x2(u & 0x7FFF7FFFu, sg & 0x7FFF7FFFu);
+            a0 = __uint_as_float(m << 16);
+            a1 = __uint_as_float(m & 0xFFFF0000u);
         }
-        const uint32_t (&rkc)[20] = rkg;
-        const uint32_t (&rk)[20] = kGrouped ? rkc : p.rk;
-        const bool landed = s_mbar_wait(s_addr(&S.full[s]), (uint32_t)par);
-        const bool work = !kGrouped || group_ok;
-        const uint16_t (&T)[kTR][kTC] = S.tile[s];
-
-        // ---- row pass: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
-        auto row_pass = [&]() {
+        uint32_t s0, s1;
+        float inv0, inv1;
+        if (k2D) {
+            // the 16x16 tile: 8 consecutive lanes hold its 16 columns
+            float a = fmaxf(a0, a1);
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
-                const int64_t r = r0 + lr, c = c0 + lc;
-                // two 16-byte reads, the lane quads of a row taking the halves in opposite
-                // order so that eight lanes cover all 32 banks
-                const int h = (lane >> 2) & 1;
-                const uint4* src = reinterpret_cast<const uint4*>(&T[lr][lc]);
-                const uint4 q0 = src[h], q1 = src[h ^ 1];
-                const uint4 lo = h ? q1 : q0, hi = h ? q0 : q1;
-                const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                uint32_t sc;
-                float inv;
-                float v[16];
-                if (kRowRht) {
-                    rht16_row(w, p.sign_mask, v, p.status);
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
-                    sc = block_code(amax, tr);
-                    inv = S.inv_tab[0][sc];
-                } else if (k2D) {
-                    sc = S.tile_s[lr >> 4][bc];
-                    inv = S.tile_inv[lr >> 4][bc];
-                    unpack16(w, v);
-                } else {
-                    sc = block_code(absmax16(w), tr);
-                    inv = S.inv_tab[0][sc];
-                    unpack16(w, v);
-                }
-                const uint2 codes =
-                    encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
-                const bool inside = r < p.rows && c < p.cols;
-                if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
-                // (row lr, block bc): half-atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
-                S.row_half_atoms[ab][bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)sc : (uint8_t)0;
+            for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+            s0 = s1 = block_code(a, tc);
+            inv0 = inv1 = inv_tab[1][s0];
+            if ((cp & 7) == 0) {
+                tile_s[j][cp >> 3] = s0;
+                tile_inv[j][cp >> 3] = inv0;
             }
-        };
-
-        if (work) {
-            if (want_row && !k2D) row_pass();
-            // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunk j
-            if (want_col || k2D) {
-                const int cp = tid & 63, j = tid >> 6;
-                uint32_t w[16];
+        } else {
+            s0 = block_code(a0, tc);
+            s1 = block_code(a1, tc);
+            inv0 = inv_tab[1][s0];
+            inv1 = inv_tab[1][s1];
+        }
+        if (want_col) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) w[e] = *reinterpret_cast<const uint32_t*>(&T[16 * j + e][2 * cp]);
-                float y0[16], y1[16];
+            for (int h = 0; h < 2; ++h) {
+                const int lc = 2 * cp + h;
+                const int64_t c = c0 + lc;
+                const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
+                uint2 codes;
                 if (kRht) {
-                    rht16_pair(w, p.flips, p.sign_mask, y0, y1, p.status);
+                    codes = encode16(h ? y1 : y0, h ? inv1 : inv0, p.col_sr, rk, 1u, e0);
                 } else {
+                    float y[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        y0[e] = bf16_lo(w[e]);
-                        y1[e] = bf16_hi(w[e]);
-                    }
+                    for (int e = 0; e < 16; ++e) y[e] = h ? bf16_hi(w[e]) : bf16_lo(w[e]);
+                    codes = encode16(y, h ? inv1 : inv0, p.col_sr, rk, 1u, e0);
                 }
-                float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    a0 = fmaxf(a0, fabsf(y0[e]));
-                    a1 = fmaxf(a1, fabsf(y1[e]));
-                }
-                uint32_t s0, s1;
-                float inv0, inv1;
-                if (k2D) {
-                    // the 16x16 tile: 8 consecutive lanes hold its 16 columns
-                    float a = fmaxf(a0, a1);
-#pragma unroll
-                    for (int o = 4; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-                    s0 = s1 = block_code(a, tc);
-                    inv0 = inv1 = S.inv_tab[1][s0];
-                    if ((cp & 7) == 0) {
-                        S.tile_s[j][cp >> 3] = s0;
-                        S.tile_inv[j][cp >> 3] = inv0;
-                    }
-                } else {
-                    s0 = block_code(a0, tc);
-                    s1 = block_code(a1, tc);
-                    inv0 = S.inv_tab[1][s0];
-                    inv1 = S.inv_tab[1][s1];
-                }
-                if (want_col) {
-                    const bool rin = r0 + 16 * j < p.rows;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int lc = 2 * cp + h;
-                        const int64_t c = c0 + lc;
-                        const uint64_t e0 = (uint64_t)c * (uint64_t)g_rows + (uint64_t)(r0 - g_row0 + 16 * j);
-                        const uint2 codes = encode16(h ? y1 : y0, h ? inv1 : inv0, p.col_sr, rk, 1u, e0);
-                        const bool inside = c < p.cols && rin;
-                        if (inside)
-                            *reinterpret_cast<uint2*>(p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j) >> 1)) = codes;
-                        // atom byte of (column lc, block j): line lc % 32, group lc / 32
-                        S.col_atom[ab][(lc & 31) * 16 + (lc >> 5) * 4 + j] =
-                            inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
-                    }
-                }
+                const bool inside = c < p.cols && rin;
+                if (inside)
+                    *reinterpret_cast<uint2*>(p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j) >> 1)) = codes;
+                // atom byte of (column lc, block j): line lc % 32, group lc / 32
+                col_atom[(lc & 31) * 16 + (lc >> 5) * 4 + j] = inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
             }
-            if (want_row && k2D) {
-                __syncthreads();  // tile scales written
-                row_pass();
-            }
-        } else if (k2D && want_row) {
-            __syncthreads();  // keep the barrier count of the k2D path
         }
+    }
+    if (want_row && k2D) {
+        __syncthreads();  // tile scales written
+        row_pass();
+    }
 
-        // the stage has been read and the tile's scales staged
-        if (__syncthreads_or(!landed)) {
-            // a copy did not land within the bound: record it, wait (bounded) for this
-            // CTA's copies still in flight, and stop
-            for (int64_t k = 0; k < kTileStages; ++k) {
-                const int64_t ii = i + k;
-                if (tile + k * G < ntiles) s_mbar_wait(s_addr(&S.full[ii % kTileStages]), (uint32_t)((ii / kTileStages) & 1));
-            }
-            if (tid == 0) set_status(p.status, kStatusTimeout);
-            return;
-        }
-        if (tid < 64 && tile + kTileStages * G < ntiles) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the reads above precede the refill
-            tile_row_fetch(p, S, tile + kTileStages * G, ntx, nty, s, tid);
-        }
-        // ---- scale stores.  Every entry written lies inside the scale buffer: the
-        // column atom is (128-column group c0 / 128, blocks r0 / 16 .. + 3) with r0 a
-        // multiple of 64 below the rows; the row half-atoms cover 64 rows below
-        // pad128(rows), and the second is skipped when its blocks start past the
-        // padded block count.
-        if (work && want_col && warp == 0) {
-            const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
-            const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
-            *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) =
-                *reinterpret_cast<const uint4*>(S.col_atom[ab] + lane * 16);
-        }
-        if (work && want_row && (warp == 2 || warp == 3)) {
-            const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
-            const int a = warp - 2;
-            if ((c0 >> 6) + a < katoms_r) {
-                const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
-                *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
-                    *reinterpret_cast<const uint2*>(S.row_half_atoms[ab][a][lane]);
-            }
+    // ---- scale stores.  Every entry written lies inside the scale buffer: the
+    // column atom is (128-column group c0 / 128, blocks r0 / 16 .. + 3) with r0 a
+    // multiple of 64 below the rows; the row half-atoms cover 64 rows below
+    // pad128(rows), and the second is skipped when its blocks start past the
+    // padded block count.
+    __syncthreads();
+    if (want_col && warp == 0) {
+        const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
+        const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
+        *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) =
+            *reinterpret_cast<const uint4*>(col_atom + lane * 16);
+    }
+    if (want_row && (warp == 2 || warp == 3)) {
+        const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
+        const int a = warp - 2;
+        if ((c0 >> 6) + a < katoms_r) {
+            const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
+            *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
+                *reinterpret_cast<const uint2*>(row_half_atoms[a][lane]);
         }
     }
 }
@@ -1175,19 +1172,9 @@ cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStrea
 }
 
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
-static cudaError_t launch_tile(const QuantParams& p, int sm_count, cudaStream_t st) {
-    constexpr size_t smem = sizeof(TileSmem) + 128;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<k2D, kRht, kGrouped, kRowRht>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    const int64_t tiles = ((p.cols + kTC - 1) / kTC) * ((p.rows + kTR - 1) / kTR);
-    const int64_t cap = 2 * (int64_t)sm_count;  // persistent: two CTAs per SM
-    const unsigned grid = (unsigned)(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
-    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, smem, st>>>(p);
+static cudaError_t launch_tile(const QuantParams& p, cudaStream_t st) {
+    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
+    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -1199,15 +1186,15 @@ cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, int sm_coun
     if (p.row_rht && (grouped || two_d)) return cudaErrorInvalidValue;
     const bool col_rht = p.col_rht && p.col_data;
     if (grouped) {
-        if (two_d) return launch_tile<true, false, true, false>(p, sm_count, st);
-        if (col_rht) return launch_tile<false, true, true, false>(p, sm_count, st);
-        return launch_tile<false, false, true, false>(p, sm_count, st);
+        if (two_d) return launch_tile<true, false, true, false>(p, st);
+        if (col_rht) return launch_tile<false, true, true, false>(p, st);
+        return launch_tile<false, false, true, false>(p, st);
     }
-    if (two_d) return launch_tile<true, false, false, false>(p, sm_count, st);
-    if (p.row_rht && col_rht) return launch_tile<false, true, false, true>(p, sm_count, st);
-    if (p.row_rht) return launch_tile<false, false, false, true>(p, sm_count, st);
-    if (col_rht) return launch_tile<false, true, false, false>(p, sm_count, st);
-    return launch_tile<false, false, false, false>(p, sm_count, st);
+    if (two_d) return launch_tile<true, false, false, false>(p, st);
+    if (p.row_rht && col_rht) return launch_tile<false, true, false, true>(p, st);
+    if (p.row_rht) return launch_tile<false, false, false, true>(p, st);
+    if (col_rht) return launch_tile<false, true, false, false>(p, st);
+    return launch_tile<false, false, false, false>(p, st);
 }
 
 cudaError_t launch_sf_pad(uint8_t* sf, int64_t rows, int64_t nb, int sm_count, cudaStream_t st) {
