@@ -509,11 +509,24 @@ __device__ __forceinline__ bool finite_bits(uint32_t b) { return (b & 0x7FFFFFFF
 // 256-entry table once per tensor scale and looks the multiplier up per block.
 __device__ __forceinline__ float block_inv_of_code(uint32_t s, float g) {
     const float d = __fmul_rn(e4m3_to_f32(s), g);
-    return (d == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, d), 3.402823466e38f);
+    return (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), 3.402823466e38f);  // correctly rounded 1 / d
+}
+// RN(a / 6) for finite a >= 0.  With y = RN(1/6): q = RN(a y) is within an ulp of
+// a / 6, the residual a - 6q is exact in one FMA, and RN(q + r y) is the correctly
+// rounded quotient -- the correction step for division by a constant (Markstein;
+// Brisebarre, Muller and Raina, "Accelerating correctly rounded floating-point
+// division when the divisor is known in advance", IEEE TC 2004).  An exhaustive host
+// test (tests/test_div6_host.py) shows it equal to IEEE division for every fp32
+// a >= 2^-125; smaller a (quotients near the subnormal range) take the division.
+__device__ __forceinline__ float div6_rn(float a) {
+    if (a < 0x1p-125f) return __fdiv_rn(a, 6.0f);
+    const float y = 0x1.555556p-3f;  // RN(1/6)
+    const float q = __fmul_rn(a, y);
+    return __fmaf_rn(__fmaf_rn(-q, 6.0f, a), y, q);
 }
 // E4M3 code of a block with amax_b: RNE_satfinite((amax_b / 6) * enc).
 __device__ __forceinline__ uint32_t block_code(float amax_b, const TensorScale& ts) {
-    return e4m3_rn_satfinite(__fmul_rn(__fdiv_rn(amax_b, 6.0f), ts.enc));
+    return e4m3_rn_satfinite(__fmul_rn(div6_rn(amax_b), ts.enc));
 }
 
 // Stochastic rounding of eight values straight to packed E2M1 codes (element i in
@@ -733,47 +746,55 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 
-    TensorScale tr{0.0f, 0.0f}, tc{0.0f, 0.0f};
-    int64_t g_row0 = 0, g_rows = p.rows;  // the rows the element indices count in
-    uint32_t rkg[20];                     // the group's Philox round keys
-    bool ok = true;
+    // ---- the tensor scales (one thread computes them, the CTA shares them)
+    __shared__ float sh_scales[4];  // row g, row enc, column g, column enc
+    int64_t g = 0, g_row0 = 0, g_rows = p.rows;  // the group; the rows the element indices count in
+    uint32_t wr, wc;
     if (kGrouped) {
-        const int64_t g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
+        g = p.row_group ? (int64_t)p.row_group[r0 >> 7] : r0 / p.group_rows_uniform;
         g_row0 = p.row_group ? p.group_row0[g] : g * p.group_rows_uniform;
         g_rows = p.row_group ? p.group_nrows[g] : p.group_rows_uniform;
-        const uint32_t wr = p.amax_words[2 * g];
-        const uint32_t wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
-        const bool first = r0 == g_row0 && c0 == 0 && tid == 0;
-        ok = finite_bits(wr) && finite_bits(wc);
-        if (!ok) {
-            if (first) {
-                set_status(p.status, kStatusNonFinite);
-                if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
-                if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
-            }
-        } else {
-            tr = tensor_scale_from_amax(__uint_as_float(wr));
-            tc = tensor_scale_from_amax(__uint_as_float(wc));
-            if (first) {
-                if (p.row_g) p.row_g[g] = tr.g;
-                if (p.col_g) p.col_g[g] = tc.g;
-            }
-            uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
-#pragma unroll
-            for (int r = 0; r < 10; ++r) {
-                rkg[2 * r] = k0;
-                rkg[2 * r + 1] = k1;
-                k0 += 0x9E3779B9u;
-                k1 += 0xBB67AE85u;
-            }
-        }
+        wr = p.amax_words[2 * g];
+        wc = p.col_rht ? p.amax_words[2 * g + 1] : wr;
     } else {
-        ok = load_tensor_scales(p, tr, tc);
+        wr = p.amax_words[0];
+        wc = p.col_rht ? p.amax_words[1] : wr;
     }
-    if (!ok) {  // the same for the whole CTA; let the copies land before leaving
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
+    const bool first = tid == 0 && (kGrouped ? (r0 == g_row0 && c0 == 0) : (blockIdx.x == 0 && blockIdx.y == 0));
+    if (!finite_bits(wr) || !finite_bits(wc)) {  // the same for the whole CTA
+        if (first) {
+            set_status(p.status, kStatusNonFinite);
+            if (p.row_g) p.row_g[g] = __uint_as_float(0x7FC00000u);
+            if (p.col_g) p.col_g[g] = __uint_as_float(0x7FC00000u);
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");  // let the copies land before leaving
         return;
     }
+    if (tid == 0) {
+        const TensorScale a = tensor_scale_from_amax(__uint_as_float(wr));
+        const TensorScale b = tensor_scale_from_amax(__uint_as_float(wc));
+        sh_scales[0] = a.g;
+        sh_scales[1] = a.enc;
+        sh_scales[2] = b.g;
+        sh_scales[3] = b.enc;
+        if (first) {
+            if (p.row_g) p.row_g[g] = a.g;
+            if (p.col_g) p.col_g[g] = b.g;
+        }
+    }
+    uint32_t rkg[20];  // the group's Philox round keys
+    if (kGrouped) {
+        uint32_t k0 = (uint32_t)(p.seed + (uint64_t)g), k1 = (uint32_t)((p.seed + (uint64_t)g) >> 32);
+#pragma unroll
+        for (int r = 0; r < 10; ++r) {
+            rkg[2 * r] = k0;
+            rkg[2 * r + 1] = k1;
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+    }
+    __syncthreads();
+    const TensorScale tr{sh_scales[0], sh_scales[1]}, tc{sh_scales[2], sh_scales[3]};
     const uint32_t (&rkc)[20] = rkg;
     const uint32_t (&rk)[20] = kGrouped ? rkc : p.rk;
     const bool want_row = p.row_data != nullptr;
@@ -781,8 +802,8 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     {
         const float dec = e4m3_to_f32((uint32_t)tid);
         const float gr = __fmul_rn(dec, tr.g), gc = __fmul_rn(dec, tc.g);
-        inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gr), 3.402823466e38f);
-        inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__fdiv_rn(1.0f, gc), 3.402823466e38f);
+        inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__frcp_rn(gr), 3.402823466e38f);
+        inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__frcp_rn(gc), 3.402823466e38f);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();  // tile and tables in shared memory
