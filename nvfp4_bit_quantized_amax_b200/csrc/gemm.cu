@@ -95,25 +95,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "l"(map), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
-// The same tile load with an L2 eviction-priority hint (a policy from l2_policy).
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                                 uint32_t bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-        "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy)
-        : "memory");
-}
-// L2 policies: keep (evict last) the operand that is re-read across waves, let the
-// streamed one go first.
-__device__ __forceinline__ uint64_t l2_policy(bool keep) {
-    uint64_t pol;
-    if (keep)
-        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    else
-        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
     asm volatile(
@@ -904,12 +885,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0) {
             // ------------------------------------------------ A/B producer (each CTA its own)
             const uint32_t empty0 = smem_addr(&S.empty[0]);
-            // the operand that stays resident across waves (the smaller one in orders
-            // 0 / 1, the banded one in orders 2 / 3) is kept in L2, the other streams
-            const bool keep_a = p.group_mode == 0 && (order == 1 || order == 2);
-            const bool keep_b = p.group_mode == 0 && (order == 0 || order == 3);
-            const uint64_t pol_a = l2_policy(keep_a), pol_b = l2_policy(keep_b);
-            const bool hint = p.group_mode == 0;
             uint32_t s = 0, ph = 0;
             for (int64_t pt = cid; pt < tiles && !*(volatile int*)&timed_out; pt += ncl) {
                 const PairJob jb = job_of(pt);
@@ -922,17 +897,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     // this CTA's A and B boxes (rows past the tensors are zero-filled and count)
                     const uint32_t fb = smem_addr(&S.full[s]);
                     mbar_expect_tx(fb, 2u * 128u * kBKBytes);
-                    if (hint) {
-                        tma_load_2d_hint(smem_addr(S.a[s]), &tmA, (int)(kt * kBKBytes), (int)(jb.m0 + 128 * rank),
-                                         fb, pol_a);
-                        tma_load_2d_hint(smem_addr(S.b[s]), &tmB, (int)(kt * kBKBytes), (int)(jb.b_row + 128 * rank),
-                                         fb, pol_b);
-                    } else {
-                        tma_load_2d(smem_addr(S.a[s]), &tmA, (int)(jb.k0 / 2 + kt * kBKBytes),
-                                    (int)(jb.m0 + 128 * rank), fb);
-                        tma_load_2d(smem_addr(S.b[s]), &tmB, (int)((jb.bk0 + jb.k0) / 2 + kt * kBKBytes),
-                                    (int)(jb.b_row + 128 * rank), fb);
-                    }
+                    tma_load_2d(smem_addr(S.a[s]), &tmA, (int)(jb.k0 / 2 + kt * kBKBytes),
+                                (int)(jb.m0 + 128 * rank), fb);
+                    tma_load_2d(smem_addr(S.b[s]), &tmB, (int)((jb.bk0 + jb.k0) / 2 + kt * kBKBytes),
+                                (int)(jb.b_row + 128 * rank), fb);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -1247,7 +1215,10 @@ static void pair_tile_order(GemmParams& g, int64_t l2_bytes) {
         g.tile_band = 0;
         return;
     }
-    int64_t band = (l2_bytes * 2 / 5) / (256 * row_bytes);
+    // A fifth of L2 per resident band: at two fifths (a 50 MB band of the 8192 x 20480
+    // dgrad operand) the band thrashed (453 MB of DRAM traffic for a modelled 296 MB);
+    // at a fifth the measured 407 MB matches the model's 414 MB.
+    int64_t band = (l2_bytes / 5) / (256 * row_bytes);
     if (band < 1) band = 1;
     const int64_t bm = band < tiles_m ? band : tiles_m, bn = band < tiles_n ? band : tiles_n;
     const int64_t reads_m = a + (tiles_m + bm - 1) / bm * b;  // A bands resident, B streamed per band
