@@ -121,16 +121,12 @@ __device__ __forceinline__ Philox4 philox4x32_10_rk(uint32_t c0, uint32_t c1, ui
     return Philox4{c0, c1, c2, c3};
 }
 
-// Sixteen-bit draws of the 8 consecutive elements 8*group .. 8*group+7 of random
-// stream `stream`: counter (group lo, group hi, stream, 0); element j takes half
-// (j & 1) of word (j >> 1).
+// The Philox block of the 8 consecutive elements 8*group .. 8*group+7 of random
+// stream `stream`: counter (group lo, group hi, stream, 0).  Its words serve the
+// element pairs (0,2), (1,3), (4,6), (5,7), 16 bits per element (sr_codes8).
 __device__ __forceinline__ Philox4 sr_draws8(const uint32_t (&rk)[20], uint32_t stream,
                                              uint64_t group) {
     return philox4x32_10_rk((uint32_t)group, (uint32_t)(group >> 32), stream, 0u, rk);
-}
-__device__ __forceinline__ uint32_t draw16(const Philox4& p, int j) {
-    const uint32_t w = (j >> 1) == 0 ? p.x : (j >> 1) == 1 ? p.y : (j >> 1) == 2 ? p.z : p.w;
-    return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
 }
 
 // ---------------------------------------------------------------- scale layout

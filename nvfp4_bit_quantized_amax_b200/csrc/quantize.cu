@@ -529,42 +529,30 @@ __device__ __forceinline__ uint32_t block_code(float amax_b, const TensorScale& 
     return e4m3_rn_satfinite(__fmul_rn(div6_rn(amax_b), ts.enc));
 }
 
-// Stochastic rounding of eight values straight to packed E2M1 codes (element i in
-// bits [4i, 4i+4), the sign bit of y kept, zero included), the magnitude being
-// a = min(|y| * inv, 6).  With lo <= a <= hi the adjacent grid points the rule rounds
-// up iff r < p * 2^16, p = (a - lo) / (hi - lo), r the element's 16-bit draw.  The map
-// c(a) = min(2a, a + 2, a / 2 + 4) is affine between grid points and sends the grid
-// {0, .5, 1, 1.5, 2, 3, 4, 6} to the codes 0..7, so floor(c(a)) is the code of lo
-// and frac(c(a)) is p; hence code = floor(c) + [r < p * 2^16] =
-// (ceil(c * 2^16) + 65535 - r) >> 16, and grid points (p = 0) never move.  Each
-// line is an fp32 FMA rounded upward with 2^23 + offset * 2^16 + 65535 as its addend
-// (integers below 2^24, so the only rounding is the ceiling, which commutes with
-// the minimum), two elements per packed FMA; the float's bits minus r then carry
-// the code in byte 2.  Byte permutes gather the codes and the sign bits.
+// Stochastic rounding of eight values y * inv to packed E2M1 codes (element i in
+// bits [4i, 4i+4), the sign bit of y kept, zero included; |y * inv| > 6 gives 6)
+// with the B200's stochastic conversion, cvt.rs.satfinite.e2m1x4.f32.  Given
+// {0, b, 0, f} it writes f's code to nibble 0 and b's to nibble 2 and rounds each
+// up iff R + floor(p * 2^16) >= 2^16, p the position of |v| between its grid
+// neighbours, R = bytes 2:0 of the random word for f and bytes 3:1 for b: two
+// elements per conversion, 16 draw bits each (the other two lanes hold exact
+// zeros, which no draw moves).  Words x, y, z, w of the Philox block serve the
+// element pairs (0,2), (1,3), (4,6), (5,7); two shifted sums interleave the nibbles.
+__device__ __forceinline__ uint32_t cvt_rs_e2m1_pair(float b, float f, uint32_t rbits) {
+    uint16_t d;
+    asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %1, %3}, %4;"
+        : "=h"(d)
+        : "f"(0.0f), "f"(b), "f"(f), "r"(rbits));
+    return d;
+}
 __device__ __forceinline__ uint32_t sr_codes8(const float (&y)[8], float inv, const Philox4& rnd) {
-    const f32x2 k1 = pk(131072.0f, 131072.0f), k2 = pk(65536.0f, 65536.0f), k3 = pk(32768.0f, 32768.0f);
-    const f32x2 c1 = pk(8454143.0f, 8454143.0f), c2 = pk(8585215.0f, 8585215.0f), c3 = pk(8716287.0f, 8716287.0f);
-    uint32_t e[8];
+    const f32x2 iv = pk(inv, inv);
+    float v[8];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const f32x2 a = pk(fminf(__fmul_rn(fabsf(y[2 * m]), inv), 6.0f),
-                           fminf(__fmul_rn(fabsf(y[2 * m + 1]), inv), 6.0f));
-        float t1l, t1h, t2l, t2h, t3l, t3h;
-        unpk(fma2_ru(a, k1, c1), t1l, t1h);
-        unpk(fma2_ru(a, k2, c2), t2l, t2h);
-        unpk(fma2_ru(a, k3, c3), t3l, t3h);
-        e[2 * m] = __float_as_uint(fmin3(t1l, t2l, t3l)) - draw16(rnd, 2 * m);
-        e[2 * m + 1] = __float_as_uint(fmin3(t1h, t2h, t3h)) - draw16(rnd, 2 * m + 1);
-    }
-    const uint32_t ce = __byte_perm(__byte_perm(e[0], e[2], 0x0062), __byte_perm(e[4], e[6], 0x0062), 0x5410);
-    const uint32_t co = __byte_perm(__byte_perm(e[1], e[3], 0x0062), __byte_perm(e[5], e[7], 0x0062), 0x5410);
-    const uint32_t se = __byte_perm(__byte_perm(__float_as_uint(y[0]), __float_as_uint(y[2]), 0x0073),
-                                    __byte_perm(__float_as_uint(y[4]), __float_as_uint(y[6]), 0x0073), 0x5410);
-    const uint32_t so = __byte_perm(__byte_perm(__float_as_uint(y[1]), __float_as_uint(y[3]), 0x0073),
-                                    __byte_perm(__float_as_uint(y[5]), __float_as_uint(y[7]), 0x0073), 0x5410);
-    const uint32_t even = ce | ((se >> 4) & 0x08080808u);  // element 2k in byte k, sign in bit 3
-    const uint32_t odd = co | ((so >> 4) & 0x08080808u);
-    return even + (odd << 4);
+    for (int m = 0; m < 4; ++m) unpk(mul2(pk(y[2 * m], y[2 * m + 1]), iv), v[2 * m], v[2 * m + 1]);
+    const uint32_t c02 = cvt_rs_e2m1_pair(v[2], v[0], rnd.x), c13 = cvt_rs_e2m1_pair(v[3], v[1], rnd.y);
+    const uint32_t c46 = cvt_rs_e2m1_pair(v[6], v[4], rnd.z), c57 = cvt_rs_e2m1_pair(v[7], v[5], rnd.w);
+    return (c02 + (c13 << 4)) | ((c46 + (c57 << 4)) << 16);
 }
 
 // Round-to-nearest-even codes of y * inv, eight values.

@@ -27,8 +27,11 @@
  *  R7  RHT: y = x . diag(s) . H16 with the unnormalised Sylvester H16 (H H^T = 16 I);
  *      the quantizer sees the fp32 rounding of the exact sum.
  *  R8  stochastic rounding: lo <= |v| < hi adjacent E2M1 magnitudes,
- *      p = (|v| - lo) / (hi - lo); round up iff r < p * 2^16, with r the element's
- *      16-bit Philox draw (see ora_sr_draw16).
+ *      p = (|v| - lo) / (hi - lo); round up iff R + floor(p * 2^16) >= 2^16, with R
+ *      the element's 16-bit Philox draw (see ora_sr_draw16).  The round-up
+ *      probability floor(p * 2^16) / 2^16 is within 2^-16 of p and never above it.
+ *      (The B200's stochastic E2M1 conversion applies this rule to the draws it is
+ *      given, which the draw layout of ora_sr_draw16 follows.)
  *  R9  amax == 0 gives g = 0, enc = 0, all scales 0 and all codes +-0.
  *  R14 RHT on both backward GEMMs ([LTD] "Main findings", the Mosaic recipe): the
  *      dgrad operands dY and W^T are rotated along N, their shared reduction axis,
@@ -162,20 +165,29 @@ void ora_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t ou
 
 /* R8: element `idx` (row-major index in the quantized tensor V) takes 16 bits of
  * the Philox block with counter (idx>>3 low, idx>>3 high, stream, 0) and key
- * (seed low, seed high): word (idx&7)>>1, half (idx&1) (low half first).       */
+ * (seed low, seed high).  With j = idx & 7, the block's words pair the elements
+ * (0,2), (1,3), (4,6), (5,7): element j reads word (j & 1) + 2 * (j >> 2); the
+ * first element of a pair (bit 1 of j clear) takes bytes 2 (high) and 0 (low) of
+ * that word, the second bytes 3 (high) and 1 (low).  Every bit of the block serves
+ * exactly one element.                                                          */
 unsigned ora_sr_draw16(uint64_t seed, uint32_t stream, uint64_t idx) {
     uint64_t g = idx >> 3;
     uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), stream, 0u};
     uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
     uint32_t w[4];
     ora_philox4x32_10(ctr, key, w);
-    uint32_t word = w[(idx & 7u) >> 1];
-    return (unsigned)((word >> (16u * (unsigned)(idx & 1u))) & 0xFFFFu);
+    unsigned j = (unsigned)(idx & 7u);
+    uint32_t word = w[(j & 1u) + 2u * (j >> 2)];
+    unsigned h = (j >> 1) & 1u;
+    unsigned byte_lo = (word >> (8u * h)) & 0xFFu;
+    unsigned byte_hi = (word >> (8u * (2u + h))) & 0xFFu;
+    return (byte_hi << 8) | byte_lo;
 }
 
-/* R8: stochastic rounding onto the E2M1 grid.  The round-up probability is
- * p = (|v| - lo) / (hi - lo), realised as r < p * 65536 with r uniform in
- * [0, 65536).  All quantities are exact in fp64.                              */
+/* R8: stochastic rounding onto the E2M1 grid.  p = (|v| - lo) / (hi - lo) is exact
+ * in fp64 (|v| is a float, lo and hi are grid points); the element rounds up iff
+ * its draw R (uniform in [0, 65536)) satisfies R + floor(p * 65536) >= 65536, so
+ * floor(p * 65536) of the 65536 draws round up.                                */
 unsigned ora_e2m1_encode_sr(float v, unsigned r16) {
     unsigned sign = signbit(v) ? 8u : 0u;
     double a = fabs((double)v);
@@ -184,7 +196,8 @@ unsigned ora_e2m1_encode_sr(float v, unsigned r16) {
     while (c < 7 && ora_e2m1_decode(c + 1) <= a) ++c;
     double lo = ora_e2m1_decode(c), hi = ora_e2m1_decode(c + 1);
     double p = (a - lo) / (hi - lo);
-    unsigned up = ((double)r16 < p * 65536.0) ? 1u : 0u;
+    double t = floor(p * 65536.0);
+    unsigned up = ((double)r16 + t >= 65536.0) ? 1u : 0u;
     return sign | (c + up);
 }
 

@@ -99,13 +99,23 @@ def test_philox_known_answers(ora):
 
 
 def test_sr_draw_layout(ora):
+    """Each Philox block serves 8 consecutive elements; the words pair elements
+    (0,2), (1,3), (4,6), (5,7), the first of a pair taking bytes 2:0 of its word,
+    the second bytes 3:1; together the 8 draws use every bit of the block once."""
     seed = 0x0123456789ABCDEF
     for blk in (0, 1, 12345, (1 << 33) + 7):
-        words = ora.philox4x32_10([blk & 0xFFFFFFFF, blk >> 32, 1, 0],
-                                  [seed & 0xFFFFFFFF, seed >> 32])
+        words = [int(w) for w in ora.philox4x32_10([blk & 0xFFFFFFFF, blk >> 32, 1, 0],
+                                                   [seed & 0xFFFFFFFF, seed >> 32])]
+        pair_word = {0: 0, 2: 0, 1: 1, 3: 1, 4: 2, 6: 2, 5: 3, 7: 3}
+        used = [0, 0, 0, 0]
         for j in range(8):
-            half = (int(words[j // 2]) >> (16 * (j % 2))) & 0xFFFF
-            assert ora.sr_draw16(seed, 1, blk * 8 + j) == half
+            w = words[pair_word[j]]
+            second = j in (2, 3, 6, 7)
+            b = [(w >> (8 * k)) & 0xFF for k in range(4)]
+            expect = (b[3] << 8 | b[1]) if second else (b[2] << 8 | b[0])
+            assert ora.sr_draw16(seed, 1, blk * 8 + j) == expect
+            used[pair_word[j]] |= (0xFF00FF00 if second else 0x00FF00FF)
+        assert used == [0xFFFFFFFF] * 4
 
 
 # ---- stochastic rounding ------------------------------------------------------------
@@ -124,6 +134,33 @@ def test_sr_unbiased_1e6(ora, v):
     p = (a - lo) / (hi - lo)
     sigma = math.sqrt(p * (1 - p)) * (hi - lo)
     assert abs(vals.mean() - float(np.float32(v))) < 4 * sigma / math.sqrt(n) + 1e-12
+
+
+def _f32(bits):
+    return float(np.array([bits], dtype=np.uint32).view(np.float32)[0])
+
+
+@pytest.mark.parametrize("v", [_f32(0x3F800000 + 12345), _f32(0x3F800000 + (0xFF00 << 6) + 63),
+                               _f32(0x3F000000 + 2 * 777777), _f32(0x40800000 + (0x1234 << 6) + 9),
+                               _f32(0x3A000000 + 4321), 0.1, 0.3, 2.9, 5.99, -1.3, -0.05, 1e-20])
+def test_sr_exact_round_up_count(ora, v):
+    """Every one of the 65536 draws, for values whose p * 2^16 is not an integer:
+    the number of draws that round up is the one integer n with
+    p * 2^16 - 1 < n <= p * 2^16 (the probability is within 2^-16 of p and never
+    above it), and they are the n largest draws."""
+    from fractions import Fraction
+    grid = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3),
+            Fraction(4), Fraction(6)]
+    a = Fraction(abs(float(np.float32(v))))
+    c = max(i for i in range(8) if grid[i] <= a)
+    p = (a - grid[c]) / (grid[c + 1] - grid[c])
+    codes = np.array([ora.e2m1_encode_sr(v, r) for r in range(65536)])
+    sign = 8 if v < 0 else 0
+    assert set(np.unique(codes)) <= {sign | c, sign | (c + 1)}
+    up = codes == (sign | (c + 1))
+    n = int(up.sum())
+    assert p * 65536 - 1 < n <= p * 65536
+    assert up[65536 - n:].all() and not up[:65536 - n].any()
 
 
 def test_sr_grid_points_fixed_and_saturation(ora):
