@@ -41,45 +41,8 @@ namespace nvfp4 {
 constexpr int kBM = 128;         // rows of A per tile (MMA M)
 constexpr int kBKBytes = 128;    // bytes of K per stage per row (256 FP4)
 constexpr int kKStep = 64;       // FP4 elements per MMA
-constexpr long long kWaitCycles = 1ll << 31;
 
 // ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for the phase with the given parity to complete: false once
-// `budget` clock cycles have passed without it.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > budget) return false;
-    return true;
-}
-// Wait, at exit after a timeout, for this CTA's own asynchronous work (copies it
-// issued, MMAs it committed) to finish.  That work always completes, so the bound
-// is the long default, never the (possibly short) budget of the pipeline waits.
-__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
-    (void)mbar_wait(bar, parity, kWaitCycles);
-}
 // After a timeout: spin ~`cycles` so that mbarrier arrivals already on their way
 // between the two CTAs of a pair land before either CTA can leave.
 __device__ __forceinline__ void settle(long long cycles) {
@@ -93,14 +56,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(map), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
@@ -261,6 +216,33 @@ struct TmemLayout {
 };
 
 // ---------------------------------------------------------------- epilogue
+// 32 consecutive TMEM columns of this warp's 32 lanes (lane = row), one register
+// each; the values are valid after tmem_wait_ld.
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+// Wait for this thread's TMEM loads; the registers of `r` pass through the wait so
+// that no use of them is scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+                   "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+                   "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+                   "+r"(r[31])
+                 :
+                 : "memory");
+}
 // One epilogue warp's share of a finished tile: its 32 TMEM lanes (rows row0 ..
 // row0+31 of D, lane = row) by BN/2 columns from col0; nothing is stored unless
 // `store`, and `zero` writes zeros without reading the accumulator.  Drains the accumulator into
@@ -288,17 +270,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, 
             continue;
         }
         uint32_t r[32];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-            "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-              "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-              "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-              "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-              "=r"(r[31])
-            : "r"(lane_base + (uint32_t)(c * 32)));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        tmem_ld_32cols(lane_base + (uint32_t)(c * 32), r);
+        tmem_wait_ld(r);
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
@@ -978,7 +951,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint64_t ad = adesc0 + kStep * s, bd = bdesc0 + kStep * s;
                     const uint32_t t_sfa = tsf0 + (uint32_t)kRegion * s;
                     const uint32_t t_sfb = t_sfa + kSfaCols;
-                    if (kMx) {
+                    if (!kMx && kt < KT_full) {
+                        tc_mma_nvf4_pair_x4(tmem, ad, bd, kIdesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
+                    } else if (kMx) {
                         // an atom serves two K = 64 steps: steps 0, 1 read atom 0 (scale
                         // ids 0, 2), steps 2, 3 atom 1
                         const int nks = kt < KT_full ? 4 : (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
@@ -986,8 +961,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                             tc_mma_mx_pair(tmem, ad + 2u * j, bd + 2u * j, mx_sf_id(kIdesc, 2u * (j & 1)),
                                            t_sfa + 4 * (j >> 1), t_sfb + 4 * G * (j >> 1),
                                            (kt > 0 || j > 0) ? 1u : 0u);
-                    } else if (kt < KT_full) {
-                        tc_mma_nvf4_pair_x4(tmem, ad, bd, kIdesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
                     } else {  // K tail: 1 to 3 steps of 64
                         const int nks = (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
                         for (int j = 0; j < nks; ++j)

@@ -500,6 +500,220 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
 }
 
 // ============================================================================
+// amax prepass streamed through shared memory (the column-rotation and plain
+// cases).  Each warp walks a contiguous range of 16-row x 128-column units.  Lanes
+// 0-15 copy the 16 rows of the next unit (256 bytes each, cp.async.bulk, completing
+// on the warp's mbarrier for that slot) into the second of the warp's two slots
+// while the warp works on the unit in the first, so the DRAM latency of a unit
+// hides behind the previous unit's arithmetic and no register holds data in
+// flight.  Lane l then takes columns 4l .. 4l+3 of the 16 rows (two column pairs):
+// max |x| from the chunk statistics and, with kColRht, max |RHT16 down the rows|
+// (rht16_pair_absmax).  Rows past the tensor, padding rows and gathered rows with an
+// index past the source are not copied and count as zeros; so do columns past the
+// tensor.  Results, word layout and grouping are those of amax_kernel.
+// ============================================================================
+constexpr int kAmaxWarps = 8;
+constexpr int kAmaxUnitCols = 128;
+constexpr int kAmaxSlotBytes = 16 * kAmaxUnitCols * 2;                  // 4 KB
+constexpr int kAmaxSmemBytes = kAmaxWarps * 2 * kAmaxSlotBytes;         // 64 KB
+
+template <bool kColRht, bool kGrouped, bool kGather>
+__global__ void __launch_bounds__(kAmaxWarps * 32, 2)
+    amax_stream_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, uint32_t sign_mask,
+                       const RhtFlips flips, uint32_t* __restrict__ words, const int32_t* __restrict__ row_group,
+                       int64_t group_rows_uniform, const int32_t* __restrict__ row_src, int64_t src_rows,
+                       int* status) {
+    extern __shared__ __align__(128) uint8_t amax_smem[];
+    __shared__ __align__(8) uint64_t bars[kAmaxWarps][2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t full_mask = 0xFFFFFFFFu;
+    const uint32_t slot0 = smem_addr(amax_smem + warp * 2 * kAmaxSlotBytes);
+    const uint32_t bar0 = smem_addr(&bars[warp][0]);
+    if (lane == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar0 + 8, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    const int64_t col_units = (cols + kAmaxUnitCols - 1) / kAmaxUnitCols;
+    const int64_t units = ((rows + 15) >> 4) * col_units;
+    const int64_t nw = (int64_t)gridDim.x * kAmaxWarps;
+    const int64_t per = (units + nw - 1) / nw;
+    const int64_t u_begin = ((int64_t)blockIdx.x * kAmaxWarps + warp) * per;
+    const int64_t u_end = u_begin + per < units ? u_begin + per : units;
+
+    // Unit u is 16-row block u / col_units, 128-column block u % col_units; the warp's
+    // units are consecutive, so both indices advance by counting (one division).
+    // Copies of the unit at (ru, cu) into slot `slot`; returns the mask of rows copied.
+    auto issue = [&](int64_t ru, int64_t cu, int slot) -> uint32_t {
+        const int64_t r0 = ru * 16, c0 = cu * kAmaxUnitCols;
+        const int64_t ncol = cols - c0 < kAmaxUnitCols ? cols - c0 : kAmaxUnitCols;
+        const uint32_t bar = bar0 + 8u * slot;
+        const uint32_t dst = slot0 + slot * kAmaxSlotBytes + lane * (kAmaxUnitCols * 2);
+        uint32_t mask;
+        const uint16_t* src = nullptr;
+        if (!kGather && r0 + 16 <= rows) {  // every row present
+            mask = 0xFFFFu;
+            if (lane == 0) mbar_expect_tx(bar, (uint32_t)(16 * ncol * 2));
+            if (lane < 16) src = x + (r0 + lane) * cols + c0;
+        } else {
+            if (lane < 16 && r0 + lane < rows) {
+                int64_t sr = r0 + lane;
+                if (kGather) {
+                    sr = __ldg(row_src + sr);
+                    if (sr >= src_rows) {
+                        set_status(status, kStatusIndex);
+                        sr = -1;
+                    }
+                }
+                if (sr >= 0) src = x + sr * cols + c0;
+            }
+            mask = __ballot_sync(full_mask, src != nullptr);
+            if (lane == 0) mbar_expect_tx(bar, (uint32_t)(__popc(mask) * ncol * 2));
+        }
+        __syncwarp();
+        if (src != nullptr) {
+            // the slot was last read by this warp's generic loads, all complete
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            bulk_load(dst, src, (uint32_t)(ncol * 2), bar);
+        }
+        return mask;
+    };
+
+    uint32_t m_row = 0;  // two packed 16-bit magnitudes (the row orientation's max |x|)
+    uint32_t m_sg = 0x80008000u;  // !kColRht: signed packed maximum (see chunk_mag_stats)
+    float m_col = 0.0f;
+    int64_t g_cur = -1;   // kGrouped: the group the running maxima belong to
+    auto row_max = [&]() -> uint32_t {  // fp32 bits of the largest magnitude seen
+        const uint32_t m = kColRht ? m_row : vmax_u16x2(m_row & 0x7FFF7FFFu, m_sg & 0x7FFF7FFFu);
+        return max(m & 0xFFFFu, m >> 16) << 16;
+    };
+    auto flush_group = [&]() {
+        uint32_t ur = row_max();
+        uint32_t uc = kColRht ? __float_as_uint(m_col) : 0u;
+        ur = __reduce_max_sync(full_mask, ur);
+        uc = __reduce_max_sync(full_mask, uc);
+        if (lane == 0 && g_cur >= 0) {
+            if (ur) atomicMax(words + 2 * g_cur, ur);
+            if (kColRht && uc) atomicMax(words + 2 * g_cur + 1, uc);
+        }
+        m_row = 0;
+        m_sg = 0x80008000u;
+        m_col = 0.0f;
+    };
+
+    uint32_t phase = 0;  // bit s: parity of slot s's next completion
+    int64_t ru = u_begin / col_units, cu = u_begin % col_units;  // the unit being computed
+    int64_t ru_n = ru, cu_n = cu;                                // the next unit to copy
+    auto advance = [&](int64_t& r, int64_t& c) {
+        if (++c == col_units) {
+            c = 0;
+            ++r;
+        }
+    };
+    uint32_t mask_cur = 0u;
+    if (u_begin < u_end) {
+        mask_cur = issue(ru_n, cu_n, 0);
+        advance(ru_n, cu_n);
+    }
+    int slot = 0;
+    bool timed_out = false, next_issued = false;
+    for (int64_t u = u_begin; u < u_end; ++u) {
+        next_issued = u + 1 < u_end;
+        uint32_t mask_next = 0u;
+        if (next_issued) {
+            mask_next = issue(ru_n, cu_n, slot ^ 1);
+            advance(ru_n, cu_n);
+        }
+        // one decision for the whole warp (its lanes meet in collectives below)
+        if (!__all_sync(full_mask, mbar_wait(bar0 + 8u * slot, (phase >> slot) & 1u, kWaitCycles))) {
+            timed_out = true;
+            break;
+        }
+        phase ^= 1u << slot;
+        const int64_t r0 = ru * 16, c0 = cu * kAmaxUnitCols;
+        if (kGrouped) {
+            const int64_t g = row_group ? (int64_t)row_group[r0 >> 7] : r0 / group_rows_uniform;
+            if (g != g_cur) {
+                flush_group();
+                g_cur = g;
+            }
+        }
+        const bool lane_in = c0 + 4 * lane < cols;
+        const uint8_t* base = amax_smem + (warp * 2 + slot) * kAmaxSlotBytes + lane * 8;
+        uint32_t wa[16], wb[16];  // rows of column pairs (4l, 4l+1) and (4l+2, 4l+3)
+        if (mask_cur == 0xFFFFu && c0 + kAmaxUnitCols <= cols) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint2 q = *reinterpret_cast<const uint2*>(base + i * (kAmaxUnitCols * 2));
+                wa[i] = q.x;
+                wb[i] = q.y;
+            }
+        } else {  // rows or columns missing: zeros there (the slot holds stale data)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint2 q = *reinterpret_cast<const uint2*>(base + i * (kAmaxUnitCols * 2));
+                const bool ok = lane_in && ((mask_cur >> i) & 1u);
+                wa[i] = ok ? q.x : 0u;
+                wb[i] = ok ? q.y : 0u;
+            }
+        }
+        __syncwarp();  // every lane's reads of the slot are done before its next refill
+        if (kColRht) {
+            uint32_t mx, mn;
+            chunk_mag_stats<16>(wa, mx, mn);
+            m_row = vmax_u16x2(m_row, mx);
+            m_col = fmaxf(m_col, rht16_pair_absmax(wa, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
+            chunk_mag_stats<16>(wb, mx, mn);
+            m_row = vmax_u16x2(m_row, mx);
+            m_col = fmaxf(m_col, rht16_pair_absmax(wb, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
+        } else {  // max |x| only: the unsigned and signed packed maxima (chunk_mag_stats)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                m_row = vmax_u16x2(m_row, vmax_u16x2(wa[i], wb[i]));
+                m_sg = vmax_s16x2(m_sg, vmax_s16x2(wa[i], wb[i]));
+            }
+        }
+        advance(ru, cu);
+        slot ^= 1;
+        mask_cur = mask_next;
+    }
+    if (timed_out) {
+        // leave no copy in flight: wait (long bound) for the slot that timed out and
+        // for the other one if a copy went into it; the warp still joins the block's
+        // barrier below (its partial maxima stand beside the error status)
+        if (lane == 0) set_status(status, kStatusTimeout);
+        mbar_wait_drain(bar0 + 8u * slot, (phase >> slot) & 1u);
+        if (next_issued) mbar_wait_drain(bar0 + 8u * (slot ^ 1), (phase >> (slot ^ 1)) & 1u);
+    }
+    if (kGrouped) {
+        flush_group();
+        return;
+    }
+    uint32_t a_row = row_max();
+    uint32_t a_col = kColRht ? __float_as_uint(m_col) : 0u;
+    a_row = __reduce_max_sync(full_mask, a_row);
+    a_col = __reduce_max_sync(full_mask, a_col);
+    __shared__ uint32_t red[2][kAmaxWarps];
+    if (lane == 0) {
+        red[0][warp] = a_row;
+        red[1][warp] = a_col;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t r = 0, c = 0;
+#pragma unroll
+        for (int w = 0; w < kAmaxWarps; ++w) {
+            r = max(r, red[0][w]);
+            c = max(c, red[1][w]);
+        }
+        if (r) atomicMax(words + 0, r);
+        if (kColRht && c) atomicMax(words + 1, c);
+    }
+}
+
+// ============================================================================
 // Shared helpers of the quantize kernels.
 // ============================================================================
 __device__ __forceinline__ bool finite_bits(uint32_t b) { return (b & 0x7FFFFFFFu) < 0x7F800000u; }
@@ -1059,6 +1273,28 @@ static int grid_for(int64_t work_items, int per_block, int sm_count, int blocks_
     return (int)g;
 }
 
+// The streamed kernel: whole-SM residency (two CTAs of eight warps per SM) up to
+// the number of units.  The shared-memory size is set on every launch: it belongs
+// to the current context, which a device reset replaces.
+template <bool kColRht, bool kGrouped, bool kGather>
+static cudaError_t launch_amax_stream(const uint16_t* x, int64_t rows, int64_t cols, uint32_t sign_mask,
+                                      const RhtFlips& f, uint32_t* words, const int32_t* row_group,
+                                      int64_t group_rows_uniform, const int32_t* row_src, int64_t src_rows,
+                                      int* status, int sm_count, cudaStream_t st) {
+    const cudaError_t e = cudaFuncSetAttribute(amax_stream_kernel<kColRht, kGrouped, kGather>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kAmaxSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int64_t units = ((rows + 15) / 16) * ((cols + kAmaxUnitCols - 1) / kAmaxUnitCols);
+    const int grid = grid_for(units, kAmaxWarps, sm_count, 2);
+    amax_stream_kernel<kColRht, kGrouped, kGather><<<grid, kAmaxWarps * 32, kAmaxSmemBytes, st>>>(
+        x, rows, cols, sign_mask, f, words, row_group, group_rows_uniform, row_src, src_rows, status);
+    return cudaGetLastError();
+}
+// Bulk copies need 16-byte aligned rows.
+static bool stream_ok(const uint16_t* x, int64_t cols) {
+    return (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && cols % 8 == 0;
+}
+
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_rht,
                         uint32_t sign_mask, uint32_t* words, int sm_count, cudaStream_t st,
                         bool row_rht, int* status) {
@@ -1066,6 +1302,12 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
     const int grid = grid_for(units, 8, sm_count, 8);
     RhtFlips f;
     rht_flips(sign_mask, f);
+    // The column rotation's arithmetic hides the copies best when streamed; the plain
+    // max |x| is pure load throughput, where sixteen 16-byte loads per lane in flight
+    // (amax_kernel) beat the two-slot stream (W 20480 x 5120: 0.148 vs 0.158 ms).
+    if (col_rht && !row_rht && stream_ok(x, cols))
+        return launch_amax_stream<true, false, false>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0,
+                                                      status, sm_count, st);
     if (row_rht && col_rht)
         amax_kernel<true, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
     else if (row_rht)
@@ -1083,6 +1325,14 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
     uint32_t* words = const_cast<uint32_t*>(p.amax_words);
     RhtFlips f;
     rht_flips(p.sign_mask, f);
+    if (p.col_rht && stream_ok(p.x, p.cols)) {
+        if (p.row_src)
+            return launch_amax_stream<true, true, true>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
+                                                        p.group_rows_uniform, p.row_src, p.src_rows, p.status,
+                                                        sm_count, st);
+        return launch_amax_stream<true, true, false>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
+                                                     p.group_rows_uniform, nullptr, 0, p.status, sm_count, st);
+    }
     if (p.col_rht && p.row_src)
         amax_kernel<true, true, false, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
                                                                    p.row_group, p.group_rows_uniform, p.row_src,
