@@ -30,8 +30,13 @@
  * Numerics (fixed readings of points the pages leave open):
  *  - decode scale g = amax / (6 * 448) (fp32), encode factor 2688 / amax.
  *  - block scale s = E4M3_rne_satfinite((amax_b / 6) * enc); element
- *    v = x * (1 / (dec(s) * g)) rounded to E2M1 (RNE, or stochastic with a
- *    16-bit Philox4x32-10 draw keyed by (seed, element index)).
+ *    v = x * (1 / (dec(s) * g)) rounded to E2M1 (RNE, or stochastic: with p the
+ *    position of |v| between its two grid neighbours, v rounds up iff
+ *    R + floor(p * 2^16) >= 2^16, R the element's 16-bit draw from the
+ *    Philox4x32-10 block of counter (e/8 low, e/8 high, stream, 0) and key seed,
+ *    e the element's row-major index; the block's words serve the element pairs
+ *    (0,2), (1,3), (4,6), (5,7) of its 8 elements, the first of a pair taking
+ *    bytes 2:0 of its word and the second bytes 3:1).
  *  - scales are stored in the block-scaled MMA layout: 512-byte atoms of
  *    128 rows x 4 blocks, rows padded to 128 and blocks to 4 with zeros.
  *  - packed codes: [rows][cols/2] bytes, element 2j in the low nibble.

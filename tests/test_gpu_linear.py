@@ -147,8 +147,9 @@ def test_linear_mlp_12b_sampled(ora):
                 assert np.array_equal(gs[offs], sf[i]), f"operand {which} scales row {r0 + i}"
         rows_cache[which] = (gd, gs, gg, vc)
 
-    def sampled(out, a, b, alpha, nrows, ncols):
-        # a 32 x 32 grid of outputs: 32 sampled rows of each operand, all pairs
+    def sampled(out, a, b, alpha, nrows, ncols, bf16=True):
+        # a 32 x 32 grid of outputs: 32 sampled rows of each operand, all pairs; bf16
+        # outputs get the half-ulp of their rounding (8 significant bits: 2^-8 |r|)
         ra_idx = np.sort(rng.choice(nrows, 32, replace=False))
         rb_idx = np.sort(rng.choice(ncols, 32, replace=False))
         mi = np.repeat(ra_idx, 32)
@@ -174,9 +175,26 @@ def test_linear_mlp_12b_sampled(ora):
         ref, bound = ora.gemm_pairs(pa, sa, pb, sb, alpha * float(ga) * float(gb), ia, ib)
         got = out[torch.from_numpy(mi).to(DEV), torch.from_numpy(ni).to(DEV)].float().cpu().numpy()
         err = np.abs(got.astype(np.float64) - ref)
-        assert (err <= TOL * bound + BF16_REL * np.abs(ref) + 1e-30).all()
+        assert (err <= TOL * bound + (BF16_REL * np.abs(ref) if bf16 else 0.0) + 1e-30).all()
         assert Kred == pa.shape[1] * 2
 
     sampled(Y, capi.LIN_X_ROW, capi.LIN_W_ROW, 1.0, M, N)
     sampled(dX, capi.LIN_DY_ROW, capi.LIN_W_COL, 1.0, M, K)
     sampled(dW, capi.LIN_DY_COL, capi.LIN_X_COL, 1.0 / 16, N, K)
+
+    # the fp32 values before the bf16 rounding: nvfp4_gemm with an fp32 output on the
+    # step's own operands, at full size, sampled with the accumulation bound alone
+    lib = capi.load()
+    for a, b, alpha, shape in ((capi.LIN_X_ROW, capi.LIN_W_ROW, 1.0, (M, N)),
+                               (capi.LIN_DY_ROW, capi.LIN_W_COL, 1.0, (M, K)),
+                               (capi.LIN_DY_COL, capi.LIN_X_COL, 1.0 / 16, (N, K))):
+        va = capi.nvfp4_linear_operand(ws, M, K, N, a)
+        vb = capi.nvfp4_linear_operand(ws, M, K, N, b)
+        D = torch.empty(shape, dtype=torch.float32, device=DEV)
+        rc = lib.nvfp4_gemm(va.data, va.scales, vb.data, vb.scales, va.tensor_scale,
+                            vb.tensor_scale, alpha, va.rows, vb.rows, va.cols, None,
+                            D.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
+        assert rc == 0
+        torch.cuda.synchronize()
+        sampled(D, a, b, alpha, shape[0], shape[1], bf16=False)
+        del D
