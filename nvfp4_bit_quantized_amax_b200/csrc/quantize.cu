@@ -1085,23 +1085,37 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
 
     // ---- copies first (they do not depend on the scales): 1024 x 16 bytes, four per
-    // thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7
+    // thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7.  Gathered rows:
+    // the four source-row indices are all loaded before any is checked, so their
+    // latencies overlap.
+    int64_t sr[4];
+    bool in[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t r = r0 + ((k * 256 + tid) >> 4), c = c0 + ((k * 256 + tid) & 15) * 8;
+        sr[k] = r;
+        in[k] = r < p.rows && c < p.cols;
+    }
+    if (p.row_src != nullptr) {
+        int32_t idx[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) idx[k] = in[k] ? __ldg(p.row_src + sr[k]) : -1;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (in[k] && idx[k] >= p.src_rows) {
+                set_status(p.status, kStatusIndex);
+                in[k] = false;
+            }
+            in[k] = in[k] && idx[k] >= 0;
+            sr[k] = idx[k];
+        }
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int q = k * 256 + tid;
         const int lr = q >> 4, lc = (q & 15) * 8;
-        const int64_t r = r0 + lr, c = c0 + lc;
-        int64_t sr = r;
-        bool in = r < p.rows && c < p.cols;
-        if (p.row_src != nullptr && in) {  // gathered rows
-            sr = __ldg(p.row_src + r);
-            if (sr >= p.src_rows) {
-                set_status(p.status, kStatusIndex);
-                in = false;
-            }
-            in = in && sr >= 0;
-        }
-        cp_async16(&tile[lr][lc], in ? (const void*)(p.x + sr * p.cols + c) : (const void*)p.x, in ? 16u : 0u);
+        cp_async16(&tile[lr][lc], in[k] ? (const void*)(p.x + sr[k] * p.cols + c0 + lc) : (const void*)p.x,
+                   in[k] ? 16u : 0u);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 
