@@ -500,14 +500,14 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
 }
 
 // ============================================================================
-// amax prepass streamed through shared memory (the column-rotation and plain
-// cases).  Each warp walks a contiguous range of 16-row x 128-column units.  Lanes
+// amax prepass of the rotated column orientation, streamed through shared
+// memory.  Each warp walks a contiguous range of 16-row x 128-column units.  Lanes
 // 0-15 copy the 16 rows of the next unit (256 bytes each, cp.async.bulk, completing
 // on the warp's mbarrier for that slot) into the second of the warp's two slots
 // while the warp works on the unit in the first, so the DRAM latency of a unit
 // hides behind the previous unit's arithmetic and no register holds data in
 // flight.  Lane l then takes columns 4l .. 4l+3 of the 16 rows (two column pairs):
-// max |x| from the chunk statistics and, with kColRht, max |RHT16 down the rows|
+// max |x| from the chunk statistics and max |RHT16 down the rows|
 // (rht16_pair_absmax).  Rows past the tensor, padding rows and gathered rows with an
 // index past the source are not copied and count as zeros; so do columns past the
 // tensor.  Results, word layout and grouping are those of amax_kernel.
@@ -517,7 +517,7 @@ constexpr int kAmaxUnitCols = 128;
 constexpr int kAmaxSlotBytes = 16 * kAmaxUnitCols * 2;                  // 4 KB
 constexpr int kAmaxSmemBytes = kAmaxWarps * 2 * kAmaxSlotBytes;         // 64 KB
 
-template <bool kColRht, bool kGrouped, bool kGather>
+template <bool kGrouped, bool kGather>
 __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
     amax_stream_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, uint32_t sign_mask,
                        const RhtFlips flips, uint32_t* __restrict__ words, const int32_t* __restrict__ row_group,
@@ -582,24 +582,21 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
     };
 
     uint32_t m_row = 0;  // two packed 16-bit magnitudes (the row orientation's max |x|)
-    uint32_t m_sg = 0x80008000u;  // !kColRht: signed packed maximum (see chunk_mag_stats)
     float m_col = 0.0f;
     int64_t g_cur = -1;   // kGrouped: the group the running maxima belong to
     auto row_max = [&]() -> uint32_t {  // fp32 bits of the largest magnitude seen
-        const uint32_t m = kColRht ? m_row : vmax_u16x2(m_row & 0x7FFF7FFFu, m_sg & 0x7FFF7FFFu);
-        return max(m & 0xFFFFu, m >> 16) << 16;
+        return max(m_row & 0xFFFFu, m_row >> 16) << 16;
     };
     auto flush_group = [&]() {
         uint32_t ur = row_max();
-        uint32_t uc = kColRht ? __float_as_uint(m_col) : 0u;
+        uint32_t uc = __float_as_uint(m_col);
         ur = __reduce_max_sync(full_mask, ur);
         uc = __reduce_max_sync(full_mask, uc);
         if (lane == 0 && g_cur >= 0) {
             if (ur) atomicMax(words + 2 * g_cur, ur);
-            if (kColRht && uc) atomicMax(words + 2 * g_cur + 1, uc);
+            if (uc) atomicMax(words + 2 * g_cur + 1, uc);
         }
         m_row = 0;
-        m_sg = 0x80008000u;
         m_col = 0.0f;
     };
 
@@ -660,21 +657,13 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
             }
         }
         __syncwarp();  // every lane's reads of the slot are done before its next refill
-        if (kColRht) {
-            uint32_t mx, mn;
-            chunk_mag_stats<16>(wa, mx, mn);
-            m_row = vmax_u16x2(m_row, mx);
-            m_col = fmaxf(m_col, rht16_pair_absmax(wa, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
-            chunk_mag_stats<16>(wb, mx, mn);
-            m_row = vmax_u16x2(m_row, mx);
-            m_col = fmaxf(m_col, rht16_pair_absmax(wb, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
-        } else {  // max |x| only: the unsigned and signed packed maxima (chunk_mag_stats)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                m_row = vmax_u16x2(m_row, vmax_u16x2(wa[i], wb[i]));
-                m_sg = vmax_s16x2(m_sg, vmax_s16x2(wa[i], wb[i]));
-            }
-        }
+        uint32_t mx, mn;
+        chunk_mag_stats<16>(wa, mx, mn);
+        m_row = vmax_u16x2(m_row, mx);
+        m_col = fmaxf(m_col, rht16_pair_absmax(wa, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
+        chunk_mag_stats<16>(wb, mx, mn);
+        m_row = vmax_u16x2(m_row, mx);
+        m_col = fmaxf(m_col, rht16_pair_absmax(wb, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
         advance(ru, cu);
         slot ^= 1;
         mask_cur = mask_next;
@@ -692,7 +681,7 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
         return;
     }
     uint32_t a_row = row_max();
-    uint32_t a_col = kColRht ? __float_as_uint(m_col) : 0u;
+    uint32_t a_col = __float_as_uint(m_col);
     a_row = __reduce_max_sync(full_mask, a_row);
     a_col = __reduce_max_sync(full_mask, a_col);
     __shared__ uint32_t red[2][kAmaxWarps];
@@ -709,7 +698,7 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
             c = max(c, red[1][w]);
         }
         if (r) atomicMax(words + 0, r);
-        if (kColRht && c) atomicMax(words + 1, c);
+        if (c) atomicMax(words + 1, c);
     }
 }
 
@@ -1394,17 +1383,17 @@ static int grid_for(int64_t work_items, int per_block, int sm_count, int blocks_
 // The streamed kernel: whole-SM residency (two CTAs of eight warps per SM) up to
 // the number of units.  The shared-memory size is set on every launch: it belongs
 // to the current context, which a device reset replaces.
-template <bool kColRht, bool kGrouped, bool kGather>
+template <bool kGrouped, bool kGather>
 static cudaError_t launch_amax_stream(const uint16_t* x, int64_t rows, int64_t cols, uint32_t sign_mask,
                                       const RhtFlips& f, uint32_t* words, const int32_t* row_group,
                                       int64_t group_rows_uniform, const int32_t* row_src, int64_t src_rows,
                                       int* status, int sm_count, cudaStream_t st) {
-    const cudaError_t e = cudaFuncSetAttribute(amax_stream_kernel<kColRht, kGrouped, kGather>,
+    const cudaError_t e = cudaFuncSetAttribute(amax_stream_kernel<kGrouped, kGather>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kAmaxSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t units = ((rows + 15) / 16) * ((cols + kAmaxUnitCols - 1) / kAmaxUnitCols);
     const int grid = grid_for(units, kAmaxWarps, sm_count, 2);
-    amax_stream_kernel<kColRht, kGrouped, kGather><<<grid, kAmaxWarps * 32, kAmaxSmemBytes, st>>>(
+    amax_stream_kernel<kGrouped, kGather><<<grid, kAmaxWarps * 32, kAmaxSmemBytes, st>>>(
         x, rows, cols, sign_mask, f, words, row_group, group_rows_uniform, row_src, src_rows, status);
     return cudaGetLastError();
 }
@@ -1424,7 +1413,7 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
     // max |x| is pure load throughput, where sixteen 16-byte loads per lane in flight
     // (amax_kernel) beat the two-slot stream (W 20480 x 5120: 0.148 vs 0.158 ms).
     if (col_rht && !row_rht && stream_ok(x, cols))
-        return launch_amax_stream<true, false, false>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0,
+        return launch_amax_stream<false, false>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0,
                                                       status, sm_count, st);
     if (row_rht && col_rht)
         amax_kernel<true, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
@@ -1445,10 +1434,10 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
     rht_flips(p.sign_mask, f);
     if (p.col_rht && stream_ok(p.x, p.cols)) {
         if (p.row_src)
-            return launch_amax_stream<true, true, true>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
+            return launch_amax_stream<true, true>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
                                                         p.group_rows_uniform, p.row_src, p.src_rows, p.status,
                                                         sm_count, st);
-        return launch_amax_stream<true, true, false>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
+        return launch_amax_stream<true, false>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
                                                      p.group_rows_uniform, nullptr, 0, p.status, sm_count, st);
     }
     if (p.col_rht && p.row_src)
