@@ -1070,7 +1070,7 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     __shared__ __align__(16) uint8_t col_atom[512];
     __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
 
     // ---- copies first (they do not depend on the scales): 1024 x 16 bytes, four per
