@@ -1014,8 +1014,9 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
                 const bool inside = c < p.cols && rin;
                 if (inside)
                     *reinterpret_cast<uint2*>(p.col_data + c * (p.rows >> 1) + ((r0 + 16 * j) >> 1)) = codes;
-                // atom byte of (column lc, block j): line lc % 32, group lc / 32
-                col_atom[(lc & 31) * 16 + (lc >> 5) * 4 + j] = inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
+                // staged block-major (byte j * 128 + lc: a warp's stores are consecutive
+                // bytes); the atom store below reorders them into the atom's lines
+                col_atom[j * 128 + lc] = inside ? (uint8_t)(h ? s1 : s0) : (uint8_t)0;
             }
         }
     }
@@ -1033,8 +1034,13 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
     if (want_col && warp == 0) {
         const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
         const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
-        *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) =
-            *reinterpret_cast<const uint4*>(col_atom + lane * 16);
+        // line l of the atom: byte 4w + j holds (column l + 32w, block j)
+        uint32_t line[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            line[w] = (uint32_t)col_atom[lane + 32 * w] | ((uint32_t)col_atom[128 + lane + 32 * w] << 8) |
+                      ((uint32_t)col_atom[256 + lane + 32 * w] << 16) | ((uint32_t)col_atom[384 + lane + 32 * w] << 24);
+        *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) = make_uint4(line[0], line[1], line[2], line[3]);
     }
     if (want_row && (warp == 2 || warp == 3)) {
         const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
@@ -1065,8 +1071,9 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     __shared__ float tile_inv[kTR / 16][kTC / 16];
     // The tile's scales, staged so that they leave in wide stores instead of one
     // byte each: the column orientation's 128 columns x 4 blocks are exactly one
-    // 512-byte atom; the row orientation's 64 rows x 8 blocks are 8 bytes of each
-    // of the 32 lines of two atoms.  Entries past the tensor hold 0 (the padding).
+    // 512-byte atom (staged block-major, reordered into lines when stored); the row
+    // orientation's 64 rows x 8 blocks are 8 bytes of each of the 32 lines of two
+    // atoms.  Entries past the tensor hold 0 (the padding).
     __shared__ __align__(16) uint8_t col_atom[512];
     __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
 
