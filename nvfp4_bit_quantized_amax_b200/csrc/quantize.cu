@@ -854,17 +854,36 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
     const int64_t nblocks = p.rows * bpr;
     const int64_t katoms = (bpr + 3) >> 2;
     const bool al32 = (reinterpret_cast<uintptr_t>(p.x) & 31u) == 0;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks;
-         b += (int64_t)gridDim.x * blockDim.x) {
-        uint32_t w[8];
-        ld_block16(p.x + b * 16, al32, w);
+    // grid-stride over blocks; the next block's 32 bytes are loaded while this one is
+    // encoded, and its (row, block) position advances by counting
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    const int64_t stride_r = stride / bpr, stride_kb = stride % bpr;
+    int64_t r = b / bpr, kb = b % bpr;
+    uint32_t w[8];
+    ld_block16(p.x + b * 16, al32, w);
+    for (;;) {
+        const int64_t bn = b + stride;
+        uint32_t wn[8];
+        if (bn < nblocks) ld_block16(p.x + bn * 16, al32, wn);
         const uint32_t s = block_code(absmax16(w), tr);
         const float inv = inv_tab[s];
         float v[16];
         unpack16(w, v);
         const uint2 codes = encode16(v, inv, p.row_sr, p.rk, 0u, (uint64_t)b * 16);
         reinterpret_cast<uint2*>(p.row_data)[b] = codes;
-        p.row_sf[sf_offset(b / bpr, b % bpr, katoms)] = (uint8_t)s;
+        p.row_sf[sf_offset(r, kb, katoms)] = (uint8_t)s;
+        if (bn >= nblocks) break;
+        b = bn;
+        r += stride_r;
+        kb += stride_kb;
+        if (kb >= bpr) {
+            kb -= bpr;
+            ++r;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) w[k] = wn[k];
     }
 }
 
@@ -1539,7 +1558,7 @@ cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStrea
     QuantParams p = params;
     philox_round_keys(p.seed, p.rk);
     const int64_t nblocks = p.rows * (p.cols / 16);
-    const int grid = grid_for(nblocks, 256, sm_count, 8);
+    const int grid = grid_for(nblocks, 256, sm_count, 4);  // the CTAs resident at 62 registers
     quant_rows_kernel<<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
