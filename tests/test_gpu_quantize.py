@@ -59,6 +59,18 @@ def test_quantize_1x16(ora, shape, rounding, kind):
     assert_same(got, oracle_full(ora, x, 0, False, None, 0, rounding, 1234), f"{shape} {kind}")
 
 
+@pytest.mark.parametrize("rounding", [0, 1])
+def test_quantize_1x16_many_blocks_per_thread(ora, rounding):
+    """The row quantizer walks its blocks grid-stride and advances each block's (row,
+    block) position by counting: with 65 blocks per row (1040 columns), which no grid
+    stride of 256-thread CTAs divides, and 266k blocks, every thread handles several
+    blocks and the position wraps across rows.  Full comparison with the oracle."""
+    x = syn.normal_bf16((4099, 1040), 31, outlier_prob=0.01)
+    got = gpu_quantize(x, 0, rounding, seed=4321)
+    assert got[3] == 0
+    assert_same(got, oracle_full(ora, x, 0, False, None, 0, rounding, 4321), f"4099x1040 r{rounding}")
+
+
 @pytest.mark.parametrize("shape", SHAPES_2D)
 @pytest.mark.parametrize("rounding", [0, 1])
 @pytest.mark.parametrize("kind", ["normal", "laplace", "tiny"])
@@ -146,6 +158,20 @@ def test_quantize_2d_orientations(ora, shape, recipe):
     if recipe == "w":  # 16x16: the two orientations are exact transposes
         from test_oracle_quantize import unpack
         assert np.array_equal(unpack(r[0]), unpack(c[0]).T)
+
+
+@pytest.mark.parametrize("shape,recipe", [((16384, 272), "dy"), ((8208, 1040), "w")])
+def test_quantize_2d_many_units_ragged(ora, shape, recipe):
+    """Enough work that every warp of the streamed amax pass walks several 16 x 128
+    units (crossing rows, the last column unit partial: 272 columns) and every CTA of
+    the persistent 16x16 kernel several tiles (the last tile row and column partial:
+    8208 rows, 1040 columns).  Full comparison with the oracle, both orientations."""
+    signs = syn.rht_signs(5)
+    x = syn.normal_bf16(shape, 23, outlier_prob=0.01)
+    bm, rr, cr, rht = {"dy": (0, 1, 1, True), "w": (1, 0, 0, False)}[recipe]
+    r, c = gpu_quantize_2d(x, bm, rr, cr, 987, rht, signs)
+    assert_same(r, oracle_full(ora, x, 0, False, signs, bm, rr, 987), f"{recipe} {shape} row")
+    assert_same(c, oracle_full(ora, x, 1, rht, signs, bm, cr, 987), f"{recipe} {shape} col")
 
 
 @pytest.mark.parametrize("axis", [0, 1])
