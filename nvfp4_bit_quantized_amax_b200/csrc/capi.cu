@@ -4,6 +4,7 @@
 // and the order of kernel launches for each entry point.  Every step of the
 // computation runs in the kernels of quantize.cu and gemm.cu.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -11,6 +12,16 @@
 #include "internal.h"
 
 using namespace nvfp4;
+
+// NVTX range over one C-ABI call (a no-op unless a profiler is attached), so that
+// timelines show each entry point around its kernels.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define NVFP4_RANGE(name) NvtxRange nvfp4_range_(name)
 
 namespace {
 
@@ -217,6 +228,7 @@ size_t nvfp4_quantize_workspace_bytes(void) { return (size_t)kCtrlBytes; }
 int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int block_mode, int rounding,
                    uint64_t seed, uint8_t* packed, uint8_t* scales, float* tensor_scale,
                    void* workspace, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_quantize");
     if (!x || !packed || !scales || !tensor_scale) return NVFP4_ERR_ARG;
     if (!workspace) return NVFP4_ERR_WORKSPACE;
     if (block_mode != NVFP4_BLOCK_1X16 && block_mode != NVFP4_BLOCK_16X16) return NVFP4_ERR_ARG;
@@ -241,6 +253,7 @@ int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int block_mode, in
 int nvfp4_quantize_2d(const void* x, int64_t rows, int64_t cols, const nvfp4_quantize_opts* o,
                       nvfp4_tensor* row_out, nvfp4_tensor* col_out, void* workspace,
                       nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_quantize_2d");
     if (!x || !o || (!row_out && !col_out)) return NVFP4_ERR_ARG;
     if (!workspace) return NVFP4_ERR_WORKSPACE;
     if (o->block_mode != NVFP4_BLOCK_1X16 && o->block_mode != NVFP4_BLOCK_16X16) return NVFP4_ERR_ARG;
@@ -285,6 +298,7 @@ int nvfp4_quantize_2d(const void* x, int64_t rows, int64_t cols, const nvfp4_qua
 
 int nvfp4_rht(const void* x, int64_t rows, int64_t cols, int axis, const int8_t* signs, int n,
               float* y, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_rht");
     if (!x || !y) return NVFP4_ERR_ARG;
     if (n != 16 || (axis != 0 && axis != 1)) return NVFP4_ERR_ARG;
     uint32_t mask = 0;
@@ -303,6 +317,7 @@ int nvfp4_rht(const void* x, int64_t rows, int64_t cols, int axis, const int8_t*
 int nvfp4_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB,
                const float* scale_a, const float* scale_b, float alpha, int64_t M, int64_t N,
                int64_t K, void* D_bf16, float* D_f32, int* status, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_gemm");
     return nvfp4_gemm_wait_limit(A, sfA, B, sfB, scale_a, scale_b, alpha, M, N, K, D_bf16, D_f32,
                                  status, 0, stream);
 }
@@ -311,6 +326,7 @@ int nvfp4_gemm_wait_limit(const uint8_t* A, const uint8_t* sfA, const uint8_t* B
                           const float* scale_a, const float* scale_b, float alpha, int64_t M,
                           int64_t N, int64_t K, void* D_bf16, float* D_f32, int* status,
                           long long wait_cycles, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_gemm_wait_limit");
     if (!A || !sfA || !B || !sfB || (!D_bf16 && !D_f32)) return NVFP4_ERR_ARG;
     if (wait_cycles < 0) return NVFP4_ERR_ARG;
     if (M < 1 || N < 8 || K < 64 || K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_SHAPE;
@@ -369,6 +385,7 @@ static int opts_check(const nvfp4_linear_opts* o) {
 int nvfp4_linear_fprop_ex(const void* X, const void* W, void* Y, int64_t M, int64_t K, int64_t N,
                           const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
                           size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_linear_fprop_ex");
     if (!X || !W || !Y) return NVFP4_ERR_ARG;
     uint32_t mask = 0;
     if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
@@ -412,6 +429,7 @@ int nvfp4_linear_fprop(const void* X, const void* W, void* Y, int64_t M, int64_t
 int nvfp4_linear_dgrad_ex(const void* dY, void* dX, int64_t M, int64_t K, int64_t N, uint64_t seed,
                           const int8_t* rht_signs, const nvfp4_linear_opts* opts, void* ws,
                           size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_linear_dgrad_ex");
     if (!dY || !dX) return NVFP4_ERR_ARG;
     uint32_t mask = 0;
     if (sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
@@ -447,6 +465,7 @@ int nvfp4_linear_dgrad(const void* dY, void* dX, int64_t M, int64_t K, int64_t N
 
 int nvfp4_linear_wgrad(const void* dY, void* dW, int64_t M, int64_t K, int64_t N, uint64_t seed,
                        const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_linear_wgrad");
     if (!dW) return NVFP4_ERR_ARG;
     uint32_t mask = 0;
     if (dY && sign_mask_of(rht_signs, &mask)) return NVFP4_ERR_ARG;
@@ -497,6 +516,7 @@ int nvfp4_moe_linear_fprop(const void* X_perm, const void* W, void* Y_perm,
                            const int64_t* group_rows, int E, int64_t K, int64_t N,
                            const int8_t* rht_signs, void* ws, size_t ws_bytes,
                            nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_linear_fprop");
     if (!X_perm || !W || !Y_perm) return NVFP4_ERR_ARG;
     return moe_for_each(group_rows, E, K, N, ws, ws_bytes, [&](int e, int64_t row, void* w, size_t b) {
         return nvfp4_linear_fprop(static_cast<const uint16_t*>(X_perm) + row * K,
@@ -509,6 +529,7 @@ int nvfp4_moe_linear_fprop(const void* X_perm, const void* W, void* Y_perm,
 int nvfp4_moe_linear_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
                            int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
                            size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_linear_dgrad");
     if (!dY_perm || !dX_perm) return NVFP4_ERR_ARG;
     return moe_for_each(group_rows, E, K, N, ws, ws_bytes, [&](int e, int64_t row, void* w, size_t b) {
         return nvfp4_linear_dgrad(static_cast<const uint16_t*>(dY_perm) + row * N,
@@ -520,6 +541,7 @@ int nvfp4_moe_linear_dgrad(const void* dY_perm, void* dX_perm, const int64_t* gr
 int nvfp4_moe_linear_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,
                            uint64_t seed, const int8_t* rht_signs, void* ws, size_t ws_bytes,
                            nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_linear_wgrad");
     if (!dW) return NVFP4_ERR_ARG;
     return moe_for_each(group_rows, E, K, N, ws, ws_bytes, [&](int e, int64_t row, void* w, size_t b) {
         (void)row;
@@ -530,6 +552,7 @@ int nvfp4_moe_linear_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K
 
 int nvfp4_moe_gather(const void* src, const int32_t* row_src, int64_t rows, int64_t cols,
                      void* dst, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_gather");
     if (!src || !row_src || !dst) return NVFP4_ERR_ARG;
     if (rows < 1 || cols < 8 || cols % 8) return NVFP4_ERR_SHAPE;
     if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(row_src, 4)) return NVFP4_ERR_ALIGN;
@@ -543,6 +566,7 @@ int nvfp4_moe_gather(const void* src, const int32_t* row_src, int64_t rows, int6
 
 int nvfp4_moe_combine(const void* src, const int32_t* slots, int64_t tokens, int topk,
                       int64_t cols, void* dst, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_combine");
     if (!src || !slots || !dst || topk < 1) return NVFP4_ERR_ARG;
     if (tokens < 1 || cols < 8 || cols % 8) return NVFP4_ERR_SHAPE;
     if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(slots, 4)) return NVFP4_ERR_ALIGN;
@@ -748,6 +772,7 @@ size_t nvfp4_mx_scale_bytes(int64_t rows, int64_t cols) {
 
 int nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* scales,
                       nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_mx_quantize");
     if (!x || !packed || !scales) return NVFP4_ERR_ARG;
     if (rows < 1 || cols < 32 || cols % 32 || rows > (1ll << 40) / cols) return NVFP4_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(packed, 16)) return NVFP4_ERR_ALIGN;
@@ -763,6 +788,7 @@ int nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, uint8_t* packed
 int nvfp4_mx_gemm(const uint8_t* A, const uint8_t* sfA, const uint8_t* B, const uint8_t* sfB, float alpha,
                   int64_t M, int64_t N, int64_t K, void* D_bf16, float* D_f32, int* status,
                   nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_mx_gemm");
     if (!A || !sfA || !B || !sfB || (!D_bf16 && !D_f32)) return NVFP4_ERR_ARG;
     if (M < 1 || N < 8 || K < 128 || K % 128 != 0 || N % 8 != 0) return NVFP4_ERR_SHAPE;
     if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K / 2 > (1ll << 31)) return NVFP4_ERR_SHAPE;
@@ -861,6 +887,7 @@ extern "C" {
 int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, const int64_t* group_rows,
                             int E, int64_t K, int64_t N, const int8_t* rht_signs, void* ws,
                             size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_grouped_fprop");
     return moe_grouped_fprop(X_perm, nullptr, 0, W, Y_perm, group_rows, E, K, N, rht_signs, ws, ws_bytes,
                              stream);
 }
@@ -868,6 +895,7 @@ int nvfp4_moe_grouped_fprop(const void* X_perm, const void* W, void* Y_perm, con
 int nvfp4_moe_grouped_fprop_gather(const void* X_tok, const int32_t* row_src, int64_t tokens, const void* W,
                                    void* Y_perm, const int64_t* group_rows, int E, int64_t K, int64_t N,
                                    const int8_t* rht_signs, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_grouped_fprop_gather");
     if (!row_src) return NVFP4_ERR_ARG;
     if (tokens < 1 || tokens > (1ll << 31) - 1) return NVFP4_ERR_SHAPE;
     if (!aligned(row_src, 4)) return NVFP4_ERR_ALIGN;
@@ -878,6 +906,7 @@ int nvfp4_moe_grouped_fprop_gather(const void* X_tok, const int32_t* row_src, in
 int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* group_rows, int E,
                             int64_t K, int64_t N, uint64_t seed, const int8_t* rht_signs, void* ws,
                             size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_grouped_dgrad");
     if (!dY_perm || !dX_perm) return NVFP4_ERR_ARG;
     if (!aligned(dY_perm, 16) || !aligned(dX_perm, 16)) return NVFP4_ERR_ALIGN;
     uint32_t mask = 0;
@@ -909,6 +938,7 @@ int nvfp4_moe_grouped_dgrad(const void* dY_perm, void* dX_perm, const int64_t* g
 
 int nvfp4_moe_grouped_wgrad(void* dW, const int64_t* group_rows, int E, int64_t K, int64_t N,
                             void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    NVFP4_RANGE("nvfp4_moe_grouped_wgrad");
     if (!dW) return NVFP4_ERR_ARG;
     if (!aligned(dW, 16)) return NVFP4_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
