@@ -384,24 +384,23 @@ __device__ __forceinline__ void rht16_lane_pair(const uint4& w, uint32_t sign_ma
 // x 8 columns (sixteen 16-byte loads).  Word 0 receives max |x| (fp32 bits of a
 // bf16 magnitude; NaN patterns sort above Inf), word 1 max |RHT16 down the
 // rows| (column orientation), as fp32 bits.  Both are combined with atomicMax.
+// Launched for the plain max |x| and for the rotated row orientation; the rotated
+// column orientation alone goes through amax_stream_kernel.
 // ============================================================================
 // Grouped (kGrouped): the rows of a unit lie in one group, whose words are
 // words[2g] and words[2g+1]; each unit is folded into them by the warp.
 // kRowRht: word 0 (or 2g) is max |RHT16 along the rows| instead of max |x| (the
 // row orientation is rotated); a non-finite input still makes it non-finite.
-// row_src (nullable): row r of the tensor is row row_src[r] of x (see QuantParams).
 template <bool kColRht, bool kRowRht>
 constexpr int amax_min_blocks() {
     return (kColRht && kRowRht) ? 1 : 2;  // both rotations: registers for one CTA per SM
 }
-template <bool kColRht, bool kGrouped, bool kRowRht, bool kGather>
+template <bool kColRht, bool kGrouped, bool kRowRht>
 __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, uint32_t sign_mask, const RhtFlips flips,
                                                    uint32_t* __restrict__ words,
                                                    const int32_t* __restrict__ row_group,
-                                                   int64_t group_rows_uniform,
-                                                   const int32_t* __restrict__ row_src, int64_t src_rows,
-                                                   int* status) {
+                                                   int64_t group_rows_uniform, int* status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t col_units = (cols + 255) >> 8;
     const int64_t units = ((rows + 15) >> 4) * col_units;
@@ -419,17 +418,8 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
         uint4 v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            bool in = c0 < cols && r0 + i < rows;
-            int64_t sr = r0 + i;
-            if (kGather && in) {
-                sr = __ldg(row_src + r0 + i);
-                if (sr >= src_rows) {
-                    if (lane == 0) set_status(status, kStatusIndex);
-                    in = false;
-                }
-                in = in && sr >= 0;
-            }
-            v[i] = in ? ld_stream_v4(x + sr * cols + c0) : make_uint4(0, 0, 0, 0);
+            const bool in = c0 < cols && r0 + i < rows;
+            v[i] = in ? ld_stream_v4(x + (r0 + i) * cols + c0) : make_uint4(0, 0, 0, 0);
         }
         if (kRowRht) {  // every lane takes part (zeros past the columns)
 #pragma unroll
@@ -1437,18 +1427,19 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, bool col_
     rht_flips(sign_mask, f);
     // The column rotation's arithmetic hides the copies best when streamed; the plain
     // max |x| is pure load throughput, where sixteen 16-byte loads per lane in flight
-    // (amax_kernel) beat the two-slot stream (W 20480 x 5120: 0.148 vs 0.158 ms).
-    if (col_rht && !row_rht && stream_ok(x, cols))
+    // (amax_kernel) beat the two-slot stream (W 20480 x 5120: 0.148 vs 0.158 ms).  The
+    // C ABI refuses rows that are not 16-byte aligned before any launch.
+    if (col_rht && !row_rht) {
+        if (!stream_ok(x, cols)) return cudaErrorInvalidValue;
         return launch_amax_stream<false, false>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0,
-                                                      status, sm_count, st);
+                                                status, sm_count, st);
+    }
     if (row_rht && col_rht)
-        amax_kernel<true, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
+        amax_kernel<true, false, true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, status);
     else if (row_rht)
-        amax_kernel<false, false, true, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
-    else if (col_rht)
-        amax_kernel<true, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
+        amax_kernel<false, false, true><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, status);
     else
-        amax_kernel<false, false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, nullptr, 0, status);
+        amax_kernel<false, false, false><<<grid, 256, 0, st>>>(x, rows, cols, sign_mask, f, words, nullptr, 0, status);
     return cudaGetLastError();
 }
 
@@ -1458,26 +1449,18 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
     uint32_t* words = const_cast<uint32_t*>(p.amax_words);
     RhtFlips f;
     rht_flips(p.sign_mask, f);
-    if (p.col_rht && stream_ok(p.x, p.cols)) {
+    if (p.col_rht) {
+        if (!stream_ok(p.x, p.cols)) return cudaErrorInvalidValue;
         if (p.row_src)
             return launch_amax_stream<true, true>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
-                                                        p.group_rows_uniform, p.row_src, p.src_rows, p.status,
-                                                        sm_count, st);
+                                                  p.group_rows_uniform, p.row_src, p.src_rows, p.status,
+                                                  sm_count, st);
         return launch_amax_stream<true, false>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
-                                                     p.group_rows_uniform, nullptr, 0, p.status, sm_count, st);
+                                               p.group_rows_uniform, nullptr, 0, p.status, sm_count, st);
     }
-    if (p.col_rht && p.row_src)
-        amax_kernel<true, true, false, true><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
-                                                                   p.row_group, p.group_rows_uniform, p.row_src,
-                                                                   p.src_rows, p.status);
-    else if (p.col_rht)
-        amax_kernel<true, true, false, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
-                                                                    p.row_group, p.group_rows_uniform, nullptr, 0,
-                                                                    p.status);
-    else
-        amax_kernel<false, true, false, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words,
-                                                                     p.row_group, p.group_rows_uniform, nullptr,
-                                                                     0, p.status);
+    if (p.row_src) return cudaErrorInvalidValue;  // gathered rows come with the column rotation only
+    amax_kernel<false, true, false><<<grid, 256, 0, st>>>(p.x, p.rows, p.cols, p.sign_mask, f, words, p.row_group,
+                                                          p.group_rows_uniform, p.status);
     return cudaGetLastError();
 }
 
