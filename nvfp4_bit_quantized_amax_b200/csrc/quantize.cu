@@ -1552,16 +1552,16 @@ static cudaError_t launch_tile(const QuantParams& p, int sm_count, cudaStream_t 
     // 20480 x 5120 0.1475 -> 0.1421 ms); for the rotated and SR passes its
     // lockstep tiles issue less well than independent CTAs (dY 0.423 -> 0.432 ms).
     if constexpr (k2D && !kGrouped) {
-        if (p.row_src == nullptr) {
-            const int64_t tiles = ((p.cols + kTC - 1) / kTC) * ((p.rows + kTR - 1) / kTR);
-            const int grid = grid_for(tiles, 1, sm_count, 4);
-            quant_tile_persistent_kernel<k2D, kRht, kRowRht><<<grid, 256, 0, st>>>(p);
-            return cudaGetLastError();
-        }
+        if (p.row_src != nullptr) return cudaErrorInvalidValue;  // gathered rows come grouped only
+        const int64_t tiles = ((p.cols + kTC - 1) / kTC) * ((p.rows + kTR - 1) / kTR);
+        const int grid = grid_for(tiles, 1, sm_count, 4);
+        quant_tile_persistent_kernel<k2D, kRht, kRowRht><<<grid, 256, 0, st>>>(p);
+        return cudaGetLastError();
+    } else {
+        const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
+        quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, 0, st>>>(p);
+        return cudaGetLastError();
     }
-    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
-    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, 0, st>>>(p);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, int sm_count, cudaStream_t st) {
