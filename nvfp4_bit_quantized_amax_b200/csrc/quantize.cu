@@ -51,10 +51,10 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-// a * b + c rounded once, upward (toward +inf)
-__device__ __forceinline__ f32x2 fma2_ru(f32x2 a, f32x2 b, f32x2 c) {
+// a + b rounded upward (toward +inf)
+__device__ __forceinline__ f32x2 add2_ru(f32x2 a, f32x2 b) {
     f32x2 d;
-    asm("fma.rp.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    asm("add.rp.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
 __device__ __forceinline__ float fmin3(float a, float b, float c) {
@@ -306,6 +306,25 @@ __device__ __forceinline__ float rht16_pair_absmax(const uint32_t (&w)[16], cons
     return m;
 }
 
+// Upper bounds of max_j |y_j| for the two columns of a column pair (w as in
+// rht16_pair), and the pair's magnitudes folded into m_row (two packed 16-bit
+// maxima, the same as chunk_mag_stats' largest magnitude).  Every entry of H16 is
+// +-1, so |y_j| <= sum_i |x_i|.  The sums round upward, so each bound is a float at
+// or above the exact sum, hence at or above RN32(|y_j|) for every j.  The high value
+// of a word is read as fp32 with the low value's magnitude bits below its mantissa,
+// which can only raise it.  An Inf or NaN input makes the bound Inf or NaN.
+__device__ __forceinline__ f32x2 pair_l1_up(const uint32_t (&w)[16], uint32_t& m_row) {
+    f32x2 s[4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t t = w[i] & 0x7FFF7FFFu;
+        m_row = vmax_u16x2(m_row, t);
+        const f32x2 v = pk_bits(t << 16, t);
+        s[i & 3] = i < 4 ? v : add2_ru(s[i & 3], v);
+    }
+    return add2_ru(add2_ru(s[0], s[1]), add2_ru(s[2], s[3]));
+}
+
 // Rotation of one row block held by one thread: w[k] holds elements 2k, 2k+1 of the
 // block (16 values).  Scalar fp32 butterfly under the same span test, else fp64.
 __device__ __forceinline__ void rht16_row(const uint32_t (&w)[8], uint32_t sign_mask, float (&y)[16],
@@ -491,40 +510,55 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
 
 // ============================================================================
 // amax prepass of the rotated column orientation, streamed through shared
-// memory.  Each warp walks a contiguous range of 16-row x 128-column units.  Lanes
-// 0-15 copy the 16 rows of the next unit (256 bytes each, cp.async.bulk, completing
-// on the warp's mbarrier for that slot) into the second of the warp's two slots
-// while the warp works on the unit in the first, so the DRAM latency of a unit
-// hides behind the previous unit's arithmetic and no register holds data in
-// flight.  Lane l then takes columns 4l .. 4l+3 of the 16 rows (two column pairs):
-// max |x| from the chunk statistics and max |RHT16 down the rows|
-// (rht16_pair_absmax).  Rows past the tensor, padding rows and gathered rows with an
-// index past the source are not copied and count as zeros; so do columns past the
-// tensor.  Results, word layout and grouping are those of amax_kernel.
+// memory.  Each warp walks a contiguous range of 16-row x 128-column units.  The
+// whole warp copies a unit into one of its two slots with 16-byte cp.async (eight
+// per lane; rows past the tensor, padding rows, gathered rows with an index past
+// the source and columns past the tensor are zero-filled, so they count as
+// zeros) while it works on the unit in the other slot: the DRAM latency hides
+// behind the arithmetic and no register holds data in flight.  Lane l then takes
+// columns 4l .. 4l+3 of the 16 rows (two column pairs): max |x|, and max |RHT16 down
+// the rows| (rht16_pair_absmax) for the column pairs that can still raise it.
+// Results, word layout and grouping are those of amax_kernel.
+//
+// The rotation is skipped where it cannot change the result.  The warp keeps a
+// threshold: the largest rotated magnitude that it, or any warp that has published to
+// the output word (or the group's word), computed.  A column whose rounded-up sum of
+// |x| (pair_l1_up) is at most the threshold has no rotated value above it.  The word
+// ends at least at the threshold, so skipping such a column leaves the word unchanged.
+// A warp publishes its maximum to the word (atomicMax) when the maximum passes the
+// threshold.  It reads the word back when it starts the unit after one in which it
+// rotated (and on a new group), after that unit's data has landed, so that the read
+// sees what the other warps published meanwhile.  Only a rotated chunk records the
+// fp64-domain status; the quantizer's tile pass rotates every chunk, so it records
+// that status for the same input.
 // ============================================================================
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// 16-byte copy global -> shared, `src_bytes` of it read (the rest zero-filled).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
 constexpr int kAmaxWarps = 8;
 constexpr int kAmaxUnitCols = 128;
 constexpr int kAmaxSlotBytes = 16 * kAmaxUnitCols * 2;                  // 4 KB
 constexpr int kAmaxSmemBytes = kAmaxWarps * 2 * kAmaxSlotBytes;         // 64 KB
+constexpr int kAmaxCtasPerSm = 2;
 
 template <bool kGrouped, bool kGather>
-__global__ void __launch_bounds__(kAmaxWarps * 32, 2)
+__global__ void __launch_bounds__(kAmaxWarps * 32, kAmaxCtasPerSm)
     amax_stream_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, uint32_t sign_mask,
                        const RhtFlips flips, uint32_t* __restrict__ words, const int32_t* __restrict__ row_group,
                        int64_t group_rows_uniform, const int32_t* __restrict__ row_src, int64_t src_rows,
                        int* status) {
     extern __shared__ __align__(128) uint8_t amax_smem[];
-    __shared__ __align__(8) uint64_t bars[kAmaxWarps][2];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t full_mask = 0xFFFFFFFFu;
-    const uint32_t slot0 = smem_addr(amax_smem + warp * 2 * kAmaxSlotBytes);
-    const uint32_t bar0 = smem_addr(&bars[warp][0]);
-    if (lane == 0) {
-        mbar_init(bar0, 1);
-        mbar_init(bar0 + 8, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
+    uint8_t* const slots = amax_smem + warp * 2 * kAmaxSlotBytes;
 
     const int64_t col_units = (cols + kAmaxUnitCols - 1) / kAmaxUnitCols;
     const int64_t units = ((rows + 15) >> 4) * col_units;
@@ -535,44 +569,40 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
 
     // Unit u is 16-row block u / col_units, 128-column block u % col_units; the warp's
     // units are consecutive, so both indices advance by counting (one division).
-    // Copies of the unit at (ru, cu) into slot `slot`; returns the mask of rows copied.
-    auto issue = [&](int64_t ru, int64_t cu, int slot) -> uint32_t {
-        const int64_t r0 = ru * 16, c0 = cu * kAmaxUnitCols;
-        const int64_t ncol = cols - c0 < kAmaxUnitCols ? cols - c0 : kAmaxUnitCols;
-        const uint32_t bar = bar0 + 8u * slot;
-        const uint32_t dst = slot0 + slot * kAmaxSlotBytes + lane * (kAmaxUnitCols * 2);
-        uint32_t mask;
-        const uint16_t* src = nullptr;
-        if (!kGather && r0 + 16 <= rows) {  // every row present
-            mask = 0xFFFFu;
-            if (lane == 0) mbar_expect_tx(bar, (uint32_t)(16 * ncol * 2));
-            if (lane < 16) src = x + (r0 + lane) * cols + c0;
-        } else {
-            if (lane < 16 && r0 + lane < rows) {
-                int64_t sr = r0 + lane;
-                if (kGather) {
-                    sr = __ldg(row_src + sr);
-                    if (sr >= src_rows) {
-                        set_status(status, kStatusIndex);
-                        sr = -1;
-                    }
-                }
-                if (sr >= 0) src = x + sr * cols + c0;
+    // Copies of the unit at (ru, cu) into slot `slot`: 16 rows x 16 chunks of 16
+    // bytes, chunk lane + 32k of the unit being row 2k + lane / 16, chunk lane % 16.
+    // One commit group per unit and lane.
+    auto issue = [&](int64_t ru, int64_t cu, int slot) {
+        const int64_t r0 = ru * 16;
+        const int64_t col = cu * kAmaxUnitCols + (lane & 15) * 8;
+        int64_t sr = -1;  // kGather: the source row of unit row `lane` (lanes 0-15)
+        if (kGather && lane < 16 && r0 + lane < rows) {
+            sr = __ldg(row_src + r0 + lane);
+            if (sr >= src_rows) {
+                set_status(status, kStatusIndex);
+                sr = -1;
             }
-            mask = __ballot_sync(full_mask, src != nullptr);
-            if (lane == 0) mbar_expect_tx(bar, (uint32_t)(__popc(mask) * ncol * 2));
         }
-        __syncwarp();
-        if (src != nullptr) {
-            // the slot was last read by this warp's generic loads, all complete
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            bulk_load(dst, src, (uint32_t)(ncol * 2), bar);
+        uint8_t* const dst = slots + slot * kAmaxSlotBytes + (lane & 15) * 16;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int row = 2 * k + (lane >> 4);
+            int64_t src_row = r0 + row;
+            bool in = col < cols && src_row < rows;
+            if (kGather) {
+                src_row = __shfl_sync(full_mask, sr, row);
+                in = col < cols && src_row >= 0;
+            }
+            cp_async16(dst + row * (kAmaxUnitCols * 2), in ? (const void*)(x + src_row * cols + col) : (const void*)x,
+                       in ? 16u : 0u);
         }
-        return mask;
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
     uint32_t m_row = 0;  // two packed 16-bit magnitudes (the row orientation's max |x|)
     float m_col = 0.0f;
+    float thr = 0.0f;     // warp-uniform skip threshold (a rotated magnitude computed for this word)
+    bool reread = false;  // read the word again for this unit (the last one rotated, or a new group)
     int64_t g_cur = -1;   // kGrouped: the group the running maxima belong to
     auto row_max = [&]() -> uint32_t {  // fp32 bits of the largest magnitude seen
         return max(m_row & 0xFFFFu, m_row >> 16) << 16;
@@ -590,7 +620,6 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
         m_col = 0.0f;
     };
 
-    uint32_t phase = 0;  // bit s: parity of slot s's next completion
     int64_t ru = u_begin / col_units, cu = u_begin % col_units;  // the unit being computed
     int64_t ru_n = ru, cu_n = cu;                                // the next unit to copy
     auto advance = [&](int64_t& r, int64_t& c) {
@@ -599,73 +628,73 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, 2)
             ++r;
         }
     };
-    uint32_t mask_cur = 0u;
     if (u_begin < u_end) {
-        mask_cur = issue(ru_n, cu_n, 0);
+        issue(ru_n, cu_n, 0);
         advance(ru_n, cu_n);
     }
     int slot = 0;
-    bool timed_out = false, next_issued = false;
     for (int64_t u = u_begin; u < u_end; ++u) {
-        next_issued = u + 1 < u_end;
-        uint32_t mask_next = 0u;
-        if (next_issued) {
-            mask_next = issue(ru_n, cu_n, slot ^ 1);
+        if (u + 1 < u_end) {
+            issue(ru_n, cu_n, slot ^ 1);  // the slot computed last; every lane's reads of it are done
             advance(ru_n, cu_n);
+        } else {
+            asm volatile("cp.async.commit_group;" ::: "memory");  // an empty group keeps the count
         }
-        // one decision for the whole warp (its lanes meet in collectives below)
-        if (!__all_sync(full_mask, mbar_wait(bar0 + 8u * slot, (phase >> slot) & 1u, kWaitCycles))) {
-            timed_out = true;
-            break;
-        }
-        phase ^= 1u << slot;
-        const int64_t r0 = ru * 16, c0 = cu * kAmaxUnitCols;
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this lane's copies of the unit landed
+        __syncwarp();                                          // and every other lane's
+        const int64_t r0 = ru * 16;
         if (kGrouped) {
             const int64_t g = row_group ? (int64_t)row_group[r0 >> 7] : r0 / group_rows_uniform;
             if (g != g_cur) {
                 flush_group();
                 g_cur = g;
+                thr = 0.0f;  // the threshold belonged to the last group
+                reread = true;
             }
         }
-        const bool lane_in = c0 + 4 * lane < cols;
-        const uint8_t* base = amax_smem + (warp * 2 + slot) * kAmaxSlotBytes + lane * 8;
+        uint32_t* const col_word = kGrouped ? words + 2 * g_cur + 1 : words + 1;
+        const bool lane_in = cu * kAmaxUnitCols + 4 * lane < cols;
+        const uint8_t* base = slots + slot * kAmaxSlotBytes + lane * 8;
         uint32_t wa[16], wb[16];  // rows of column pairs (4l, 4l+1) and (4l+2, 4l+3)
-        if (mask_cur == 0xFFFFu && c0 + kAmaxUnitCols <= cols) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint2 q = *reinterpret_cast<const uint2*>(base + i * (kAmaxUnitCols * 2));
-                wa[i] = q.x;
-                wb[i] = q.y;
-            }
-        } else {  // rows or columns missing: zeros there (the slot holds stale data)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint2 q = *reinterpret_cast<const uint2*>(base + i * (kAmaxUnitCols * 2));
-                const bool ok = lane_in && ((mask_cur >> i) & 1u);
-                wa[i] = ok ? q.x : 0u;
-                wb[i] = ok ? q.y : 0u;
+        for (int i = 0; i < 16; ++i) {
+            const uint2 q = *reinterpret_cast<const uint2*>(base + i * (kAmaxUnitCols * 2));
+            wa[i] = q.x;
+            wb[i] = q.y;
+        }
+        __syncwarp();  // every lane's reads of the slot are done before its refill
+        // the word as other warps have left it (read after the wait, used after the
+        // first bound, so that the read has time to return)
+        const uint32_t seen = reread ? ld_relaxed_u32(col_word) : 0u;
+        float a0, a1, b0, b1;
+        unpk(pair_l1_up(wa, m_row), a0, a1);
+        thr = fmaxf(thr, __uint_as_float(seen));
+        const float t_lane = fmaxf(thr, m_col);
+        const bool need_a = !(a0 <= t_lane && a1 <= t_lane);  // a NaN bound is rotated
+        if (need_a) {
+            uint32_t mx, mn;
+            chunk_mag_stats<16>(wa, mx, mn);
+            m_col = fmaxf(m_col, rht16_pair_absmax(wa, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
+        }
+        unpk(pair_l1_up(wb, m_row), b0, b1);
+        const bool need_b = !(b0 <= t_lane && b1 <= t_lane);
+        if (need_b) {
+            uint32_t mx, mn;
+            chunk_mag_stats<16>(wb, mx, mn);
+            m_col = fmaxf(m_col, rht16_pair_absmax(wb, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
+        }
+        reread = __any_sync(full_mask, need_a || need_b);
+        if (reread) {
+            const float wmax = __uint_as_float(__reduce_max_sync(full_mask, __float_as_uint(m_col)));
+            if (wmax > thr) {
+                thr = wmax;
+                if (lane == 0) atomicMax(col_word, __float_as_uint(wmax));
             }
         }
-        __syncwarp();  // every lane's reads of the slot are done before its next refill
-        uint32_t mx, mn;
-        chunk_mag_stats<16>(wa, mx, mn);
-        m_row = vmax_u16x2(m_row, mx);
-        m_col = fmaxf(m_col, rht16_pair_absmax(wa, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
-        chunk_mag_stats<16>(wb, mx, mn);
-        m_row = vmax_u16x2(m_row, mx);
-        m_col = fmaxf(m_col, rht16_pair_absmax(wb, flips, sign_mask, mx, mn, lane_in ? status : nullptr));
         advance(ru, cu);
         slot ^= 1;
-        mask_cur = mask_next;
     }
-    if (timed_out) {
-        // leave no copy in flight: wait (long bound) for the slot that timed out and
-        // for the other one if a copy went into it; the warp still joins the block's
-        // barrier below (its partial maxima stand beside the error status)
-        if (lane == 0) set_status(status, kStatusTimeout);
-        mbar_wait_drain(bar0 + 8u * slot, (phase >> slot) & 1u);
-        if (next_issued) mbar_wait_drain(bar0 + 8u * (slot ^ 1), (phase >> (slot ^ 1)) & 1u);
-    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     if (kGrouped) {
         flush_group();
         return;
@@ -893,13 +922,6 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 // rows the amax pass read last (still in L2).
 // ============================================================================
 constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;  // +16 bytes per row: conflict-free column reads
-
-// 16-byte copy global -> shared, `src_bytes` of it read (the rest zero-filled).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src), "r"(src_bytes)
-                 : "memory");
-}
 
 // The work on one tile whose bf16 values are in `tile` (rows r0.., columns c0..)
 // with the multiplier tables filled: row orientation, column orientation and the
@@ -1408,7 +1430,7 @@ static cudaError_t launch_amax_stream(const uint16_t* x, int64_t rows, int64_t c
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kAmaxSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t units = ((rows + 15) / 16) * ((cols + kAmaxUnitCols - 1) / kAmaxUnitCols);
-    const int grid = grid_for(units, kAmaxWarps, sm_count, 2);
+    const int grid = grid_for(units, kAmaxWarps, sm_count, kAmaxCtasPerSm);
     amax_stream_kernel<kGrouped, kGather><<<grid, kAmaxWarps * 32, kAmaxSmemBytes, st>>>(
         x, rows, cols, sign_mask, f, words, row_group, group_rows_uniform, row_src, src_rows, status);
     return cudaGetLastError();
