@@ -511,11 +511,12 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
 // ============================================================================
 // amax prepass of the rotated column orientation, streamed through shared
 // memory.  Each warp walks a contiguous range of 16-row x 128-column units.  The
-// whole warp copies a unit into one of its two slots with 16-byte cp.async (eight
-// per lane; rows past the tensor, padding rows, gathered rows with an index past
-// the source and columns past the tensor are zero-filled, so they count as
-// zeros) while it works on the unit in the other slot: the DRAM latency hides
-// behind the arithmetic and no register holds data in flight.  Lane l then takes
+// whole warp copies a unit into one of its kAmaxSlots slots with 16-byte cp.async
+// (eight per lane; rows past the tensor, padding rows, gathered rows with an index
+// past the source and columns past the tensor are zero-filled, so they count as
+// zeros); the copies of the next kAmaxSlots - 1 units are in flight while it works
+// on one, so the DRAM latency hides behind the arithmetic and no register holds
+// data in flight.  Lane l then takes
 // columns 4l .. 4l+3 of the 16 rows (two column pairs): max |x|, and max |RHT16 down
 // the rows| (rht16_pair_absmax) for the column pairs that can still raise it.
 // Results, word layout and grouping are those of amax_kernel.
@@ -546,7 +547,8 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
 constexpr int kAmaxWarps = 8;
 constexpr int kAmaxUnitCols = 128;
 constexpr int kAmaxSlotBytes = 16 * kAmaxUnitCols * 2;                  // 4 KB
-constexpr int kAmaxSmemBytes = kAmaxWarps * 2 * kAmaxSlotBytes;         // 64 KB
+constexpr int kAmaxSlots = 2;                                           // units in flight + 1
+constexpr int kAmaxSmemBytes = kAmaxWarps * kAmaxSlots * kAmaxSlotBytes;  // 64 KB
 constexpr int kAmaxCtasPerSm = 2;
 
 template <bool kGrouped, bool kGather>
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, kAmaxCtasPerSm)
     extern __shared__ __align__(128) uint8_t amax_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t full_mask = 0xFFFFFFFFu;
-    uint8_t* const slots = amax_smem + warp * 2 * kAmaxSlotBytes;
+    uint8_t* const slots = amax_smem + warp * kAmaxSlots * kAmaxSlotBytes;
 
     const int64_t col_units = (cols + kAmaxUnitCols - 1) / kAmaxUnitCols;
     const int64_t units = ((rows + 15) >> 4) * col_units;
@@ -584,6 +586,14 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, kAmaxCtasPerSm)
             }
         }
         uint8_t* const dst = slots + slot * kAmaxSlotBytes + (lane & 15) * 16;
+        if (!kGather && r0 + 16 <= rows && cu * kAmaxUnitCols + kAmaxUnitCols <= cols) {  // a whole unit
+            const uint16_t* src = x + (r0 + (lane >> 4)) * cols + col;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                cp_async16(dst + (2 * k + (lane >> 4)) * (kAmaxUnitCols * 2), src + 2 * k * cols, 16u);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            return;
+        }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int row = 2 * k + (lane >> 4);
@@ -628,20 +638,29 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, kAmaxCtasPerSm)
             ++r;
         }
     };
-    if (u_begin < u_end) {
-        issue(ru_n, cu_n, 0);
-        advance(ru_n, cu_n);
+    // kAmaxSlots - 1 units in flight ahead of the one being computed (one commit group
+    // per unit, empty past the warp's range, so that the group count stays fixed)
+#pragma unroll
+    for (int k = 0; k < kAmaxSlots - 1; ++k) {
+        if (u_begin + k < u_end) {
+            issue(ru_n, cu_n, k);
+            advance(ru_n, cu_n);
+        } else {
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
     }
     int slot = 0;
     for (int64_t u = u_begin; u < u_end; ++u) {
-        if (u + 1 < u_end) {
-            issue(ru_n, cu_n, slot ^ 1);  // the slot computed last; every lane's reads of it are done
+        if (u + kAmaxSlots - 1 < u_end) {
+            // the slot computed last; every lane's reads of it are done
+            issue(ru_n, cu_n, slot == 0 ? kAmaxSlots - 1 : slot - 1);
             advance(ru_n, cu_n);
         } else {
-            asm volatile("cp.async.commit_group;" ::: "memory");  // an empty group keeps the count
+            asm volatile("cp.async.commit_group;" ::: "memory");
         }
-        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this lane's copies of the unit landed
-        __syncwarp();                                          // and every other lane's
+        // this lane's copies of the unit landed, then every other lane's
+        asm volatile("cp.async.wait_group %0;" ::"n"(kAmaxSlots - 1) : "memory");
+        __syncwarp();
         const int64_t r0 = ru * 16;
         if (kGrouped) {
             const int64_t g = row_group ? (int64_t)row_group[r0 >> 7] : r0 / group_rows_uniform;
@@ -692,7 +711,7 @@ __global__ void __launch_bounds__(kAmaxWarps * 32, kAmaxCtasPerSm)
             }
         }
         advance(ru, cu);
-        slot ^= 1;
+        slot = slot + 1 == kAmaxSlots ? 0 : slot + 1;
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     if (kGrouped) {
