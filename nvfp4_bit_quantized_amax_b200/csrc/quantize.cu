@@ -1513,51 +1513,95 @@ cudaError_t launch_amax_grouped(const QuantParams& p, int sm_count, cudaStream_t
 struct GroupSizes {
     int64_t rows[kMaxGroups];
 };
-__global__ void group_tables_kernel(GroupSizes gs, int E, int32_t* __restrict__ block_group,
-                                    int64_t* __restrict__ row0, int64_t* __restrict__ nrows,
-                                    int64_t* __restrict__ pair_row0, int32_t* __restrict__ pair_group,
-                                    int32_t* __restrict__ pair_rows) {
-    __shared__ int64_t start[kMaxGroups + 1];
-    __shared__ int32_t tstart[kMaxGroups];  // first 256-row tile of every group
-    if (threadIdx.x == 0) {
-        int64_t r = 0;
-        int32_t t = 0;
-        for (int e = 0; e < E; ++e) {
-            start[e] = r;
-            tstart[e] = t;
-            r += gs.rows[e];
-            t += (int32_t)((gs.rows[e] + 255) / 256);
+constexpr int kGroupTableThreads = 1024;  // one thread per group in the scan
+static_assert(kMaxGroups <= kGroupTableThreads, "one scan thread per group");
+
+// Largest e < n with v[e] <= x (v nondecreasing, v[0] <= x).  A group with no rows
+// shares its start with the next group, so the largest index found is never an
+// empty group while x lies below the total.
+template <typename T>
+__device__ __forceinline__ int last_at_or_below(const T* v, int n, int64_t x) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)v[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kGroupTableThreads)
+    group_tables_kernel(GroupSizes gs, int E, int32_t* __restrict__ block_group, int64_t* __restrict__ row0,
+                        int64_t* __restrict__ nrows, int64_t* __restrict__ pair_row0,
+                        int32_t* __restrict__ pair_group, int32_t* __restrict__ pair_rows) {
+    __shared__ int64_t start[kMaxGroups + 1];  // first row of every group; start[E] = all rows
+    __shared__ int32_t tstart[kMaxGroups + 1]; // first 256-row tile of every group
+    __shared__ int64_t warp_rows[32];
+    __shared__ int32_t warp_tiles[32];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    // exclusive scans of the row counts and of the 256-row tile counts
+    const int64_t r = e < E ? gs.rows[e] : 0;
+    const int32_t t = (int32_t)((r + 255) / 256);
+    int64_t ir = r;
+    int32_t it = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t ur = __shfl_up_sync(0xFFFFFFFFu, ir, o);
+        const int32_t ut = __shfl_up_sync(0xFFFFFFFFu, it, o);
+        if (lane >= o) {
+            ir += ur;
+            it += ut;
         }
-        start[E] = r;
+    }
+    if (lane == 31) {
+        warp_rows[warp] = ir;
+        warp_tiles[warp] = it;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    if (warp == 0) {
+        int64_t wr = warp_rows[lane];
+        int32_t wt = warp_tiles[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t ur = __shfl_up_sync(0xFFFFFFFFu, wr, o);
+            const int32_t ut = __shfl_up_sync(0xFFFFFFFFu, wt, o);
+            if (lane >= o) {
+                wr += ur;
+                wt += ut;
+            }
+        }
+        warp_rows[lane] = wr - warp_rows[lane];  // rows / tiles of the warps before
+        warp_tiles[lane] = wt - warp_tiles[lane];
+    }
+    __syncthreads();
+    if (e < E) {
+        start[e] = warp_rows[warp] + ir - r;
+        tstart[e] = warp_tiles[warp] + it - t;
+        if (e == E - 1) {  // the totals
+            start[E] = warp_rows[warp] + ir;
+            tstart[E] = warp_tiles[warp] + it;
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && e < E) {
         row0[e] = start[e];
         nrows[e] = gs.rows[e];
     }
-    // the 256-row tiles of every group (block 0 writes them): a group of 128 * odd
-    // rows ends with a tile whose second half lies past the group
-    if (pair_row0 && blockIdx.x == 0) {
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            const int32_t n = (int32_t)((gs.rows[e] + 255) / 256);
-            for (int32_t t = 0; t < n; ++t) {
-                pair_row0[tstart[e] + t] = start[e] + 256 * (int64_t)t;
-                pair_group[tstart[e] + t] = e;
-                pair_rows[tstart[e] + t] = (int32_t)(gs.rows[e] - 256 * (int64_t)t < 256 ? gs.rows[e] - 256 * (int64_t)t : 256);
-            }
+    // the 256-row tiles of every group: a group of 128 * odd rows ends with a tile
+    // whose second half lies past the group
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (pair_row0) {
+        for (int64_t q = (int64_t)blockIdx.x * blockDim.x + e; q < tstart[E]; q += stride) {
+            const int g = last_at_or_below(tstart, E, q);
+            const int64_t first = start[g] + 256 * (q - tstart[g]);
+            const int64_t left = start[g + 1] - first;
+            pair_row0[q] = first;
+            pair_group[q] = g;
+            pair_rows[q] = (int32_t)(left < 256 ? left : 256);
         }
     }
     const int64_t blocks = start[E] / 128;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < blocks;
-         b += (int64_t)gridDim.x * blockDim.x) {
-        int lo = 0, hi = E - 1;  // last group whose start is <= the block's first row
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (start[mid] <= b * 128) lo = mid; else hi = mid - 1;
-        }
-        while (lo < E - 1 && start[lo + 1] <= b * 128) ++lo;
-        block_group[b] = lo;
-    }
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + e; b < blocks; b += stride)
+        block_group[b] = last_at_or_below(start, E, b * 128);
 }
 
 cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block_group, int64_t* row0,
@@ -1572,9 +1616,9 @@ cudaError_t launch_group_tables(const int64_t* group_rows, int E, int32_t* block
         total += group_rows[e];
     }
     const int64_t blocks = total / 128;
-    const int grid = (int)((blocks + 255) / 256 < 64 ? (blocks + 255) / 256 : 64);
-    group_tables_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(gs, E, block_group, row0, nrows, pair_row0,
-                                                               pair_group, pair_rows);
+    const int64_t grid = (blocks + kGroupTableThreads - 1) / kGroupTableThreads;
+    group_tables_kernel<<<grid < 1 ? 1 : (grid > 16 ? 16 : (int)grid), kGroupTableThreads, 0, st>>>(
+        gs, E, block_group, row0, nrows, pair_row0, pair_group, pair_rows);
     return cudaGetLastError();
 }
 

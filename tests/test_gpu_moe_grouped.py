@@ -69,10 +69,19 @@ def expert_slice(kind, gv, gdata, gsf, e, off, m, N):
             atoms(gsf, gv.rows, gv.cols)[:, c0 // 64: c1 // 64].ravel())
 
 
+def _many_groups():
+    """1024 groups (the most a grouped call takes), nearly all empty: the group
+    tables' scans cross every warp of their block, and the last group is used."""
+    g = [0] * 1024
+    g[3], g[517], g[1000], g[1023] = 128, 384, 256, 128
+    return g
+
+
 @pytest.mark.parametrize("group_rows,K,N", [
     ([256, 0, 128, 384, 128], 256, 384),
     ([128], 128, 128),
     ([0, 1152, 128, 0, 256, 640, 128, 128], 512, 256),
+    (_many_groups(), 128, 128),
 ])
 def test_grouped_equals_per_expert(group_rows, K, N):
     g = np.array(group_rows, dtype=np.int64)
