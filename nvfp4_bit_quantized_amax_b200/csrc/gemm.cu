@@ -144,6 +144,29 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint6
 __device__ __forceinline__ uint32_t mx_sf_id(uint32_t idesc, uint32_t id) {
     return idesc | (id << 29) | (id << 4);
 }
+// The four K = 64 steps of one MX k-tile in one statement: scale ids 0, 2, 0, 2
+// (idesc0 / idesc2), A scales advancing by 4 and B scales by 4 * G columns after the
+// second step.
+template <int G>
+__device__ __forceinline__ void tc_mma_mx_x4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc0,
+                                             uint32_t idesc2, uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        ".reg .b32 sa2, sb2;\n\t"
+        "setp.ne.b32 p, %7, 0;\n\t"
+        "setp.eq.b32 q, %3, %3;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.u32 sa2, %5, 4;\n\tadd.u32 sb2, %6, %8;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], a1, b1, %4, [%5], [%6], q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], a2, b2, %3, [sa2], [sb2], q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], a3, b3, %4, [sa2], [sb2], q;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc0), "r"(idesc2), "r"(sfa), "r"(sfb), "r"(accumulate), "n"(4 * G)
+        : "memory");
+}
 
 // Bulk tensor store of a shared-memory box to global memory (async proxy), and
 // its completion groups: .read waits until the source buffer may be reused.
@@ -486,8 +509,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint64_t ad = adesc0 + kAStep * s, bd = bdesc0 + kBStep * s;
                     const uint32_t t_sfa = tsf0 + (uint32_t)TL::kRegion * s;
                     const uint32_t t_sfb = t_sfa + TL::kSfaCols;
-                    if (kMx) {
-                        const int nks = kt < KT_full ? 4 : (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
+                    if (kMx && kt < KT_full) {
+                        tc_mma_mx_x4<G>(tmem, ad, bd, mx_sf_id(idesc, 0u), mx_sf_id(idesc, 2u), t_sfa, t_sfb,
+                                        kt > 0 ? 1u : 0u);
+                    } else if (kMx) {  // K tail: 1 to 3 steps of 64
+                        const int nks = (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
                         for (int j = 0; j < nks; ++j)
                             tc_mma_mx(tmem, ad + 2u * j, bd + 2u * j, mx_sf_id(idesc, 2u * (j & 1)),
                                       t_sfa + 4 * (j >> 1), t_sfb + 4 * G * (j >> 1),
@@ -741,6 +767,30 @@ __device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t adesc, 
         : "memory");
 }
 
+// The four K = 64 steps of one MX k-tile: an E8M0 scale atom column serves two
+// steps (scale ids 0 and 2 of the same columns), so the A scales advance by 4 and
+// the B scales by 8 columns every second step.  idesc0 / idesc2 carry scale ids 0 / 2.
+__device__ __forceinline__ void tc_mma_mx_pair_x4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                  uint32_t idesc0, uint32_t idesc2, uint32_t sfa, uint32_t sfb,
+                                                  uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        ".reg .b32 sa2, sb2;\n\t"
+        "setp.ne.b32 p, %7, 0;\n\t"
+        "setp.eq.b32 q, %3, %3;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.u32 sa2, %5, 4;\n\tadd.u32 sb2, %6, 8;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], a1, b1, %4, [%5], [%6], q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], a2, b2, %3, [sa2], [sb2], q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], a3, b3, %4, [sa2], [sb2], q;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc0), "r"(idesc2), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+
 template <int STAGES, bool kMx>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -953,10 +1003,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint32_t t_sfb = t_sfa + kSfaCols;
                     if (!kMx && kt < KT_full) {
                         tc_mma_nvf4_pair_x4(tmem, ad, bd, kIdesc, t_sfa, t_sfb, kt > 0 ? 1u : 0u);
-                    } else if (kMx) {
+                    } else if (kMx && kt < KT_full) {
+                        tc_mma_mx_pair_x4(tmem, ad, bd, mx_sf_id(kIdesc, 0u), mx_sf_id(kIdesc, 2u), t_sfa, t_sfb,
+                                          kt > 0 ? 1u : 0u);
+                    } else if (kMx) {  // K tail: 1 to 3 steps of 64
                         // an atom serves two K = 64 steps: steps 0, 1 read atom 0 (scale
                         // ids 0, 2), steps 2, 3 atom 1
-                        const int nks = kt < KT_full ? 4 : (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
+                        const int nks = (int)((jb.k_len - (int64_t)kt * 256) / kKStep);
                         for (int j = 0; j < nks; ++j)
                             tc_mma_mx_pair(tmem, ad + 2u * j, bd + 2u * j, mx_sf_id(kIdesc, 2u * (j & 1)),
                                            t_sfa + 4 * (j >> 1), t_sfb + 4 * G * (j >> 1),
