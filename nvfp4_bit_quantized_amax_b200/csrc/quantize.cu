@@ -516,10 +516,10 @@ __global__ void __launch_bounds__(256, (amax_min_blocks<kColRht, kRowRht>())) am
 // past the source and columns past the tensor are zero-filled, so they count as
 // zeros); the copies of the next kAmaxSlots - 1 units are in flight while it works
 // on one, so the DRAM latency hides behind the arithmetic and no register holds
-// data in flight.  Lane l then takes
-// columns 4l .. 4l+3 of the 16 rows (two column pairs): max |x|, and max |RHT16 down
-// the rows| (rht16_pair_absmax) for the column pairs that can still raise it.
-// Results, word layout and grouping are those of amax_kernel.
+// data in flight.  Lane l then takes columns 4l .. 4l+3 of the 16 rows (two column
+// pairs): max |x|, and max |RHT16 down the rows| (rht16_pair_absmax) for the column
+// pairs that can still raise it.  Results, word layout and grouping are those of
+// amax_kernel.
 //
 // The rotation is skipped where it cannot change the result.  The warp keeps a
 // threshold: the largest rotated magnitude that it, or any warp that has published to

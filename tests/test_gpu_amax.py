@@ -135,6 +135,22 @@ def test_amax_subnormal_inputs(ora):
     check(ora, x, signs, status_ok=False)   # the quantizer may report the tiny scale
 
 
+@pytest.mark.parametrize("bits", [0x7F80, 0xFF80, 0x7FC1])
+def test_amax_late_nonfinite(bits):
+    """An Inf or NaN in the last unit of a large tensor, after every warp's threshold
+    is set: the row word holds its pattern, the quantizer reports it, and an Inf's
+    column (whose bound is Inf) is rotated, so the column word is Inf as well."""
+    signs = syn.rht_signs(7)
+    x = syn.normal_bf16(SHAPE, 26)
+    x[SHAPE[0] - 3, SHAPE[1] - 5] = bits
+    got_row, got_col, st = gpu_amax_words(x, signs)
+    assert st == capi.ERR_NONFINITE
+    if bits & 0x7F:  # NaN: its magnitude pattern sorts above Inf in the row word
+        assert got_row == (bits & 0x7FFF) << 16
+    else:
+        assert got_row == 0x7F800000 and got_col == 0x7F800000
+
+
 @pytest.mark.parametrize("gather", [False, True])
 def test_grouped_amax_alternating_scales(ora, gather):
     """170 experts of 128 rows, hidden 1024: 10880 units, several per warp, so many
