@@ -37,8 +37,8 @@ FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
 # DRAM bytes (read + write) of one launch of each GEMM of the step, from one-pass ncu
 # captures of that launch; reported only while the GEMM source is the one that was
 # captured.
-GEMM_TRAFFIC = {"gemm_cu_sha256_16": "0852f031f72d16b5", "bytes": {
-    "fprop": 87717632 + 296744448, "dgrad": 427576320 + 71228416, "wgrad": 118264064 + 179698176}}
+GEMM_TRAFFIC = {"gemm_cu_sha256_16": "61acdbb0feaffc48", "bytes": {
+    "fprop": 89231616 + 296627968, "dgrad": 427509760 + 71016448, "wgrad": 118325248 + 180209664}}
 
 
 def env_rank():
