@@ -62,13 +62,16 @@ def plant(x, r0, col, chunk):
     x[r0:r0 + 16, col] = chunk
 
 
-def check(ora, x, signs, *, status_ok=True):
-    got_row, got_col, st = gpu_amax_words(x, signs)
+def check(ora, x, signs, *, status_ok=True, repeats=3):
+    """Which columns a warp rotates depends on when the other warps publish, so the
+    pass runs several times; every run must give the oracle's words."""
     ref_row, ref_col = oracle_words(ora, x, signs)
-    if status_ok:
-        assert st == 0
-    assert got_row == ref_row, (hex(got_row), hex(ref_row))
-    assert got_col == ref_col, (hex(got_col), hex(ref_col))
+    for _ in range(repeats):
+        got_row, got_col, st = gpu_amax_words(x, signs)
+        if status_ok:
+            assert st == 0
+        assert got_row == ref_row, (hex(got_row), hex(ref_row))
+        assert got_col == ref_col, (hex(got_col), hex(ref_col))
 
 
 @pytest.mark.parametrize("kind", ["normal", "t3", "outlier"])
