@@ -926,12 +926,14 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 }
 
 // ============================================================================
-// Tile kernel: a CTA quantizes one 64 x 128 bf16 tile.  The tile goes straight
-// from global to shared memory (cp.async, 16 bytes per copy, four per thread; rows
-// and columns past the tensor and gathered padding rows are zero-filled by the copy
-// itself), so no register holds it in flight.  Then one thread per 16-element row
-// block writes the row orientation, and one thread per column pair and 16-row chunk
-// writes the column orientation.  k2D: 16x16 blocks, the tile scale is found by the
+// Tile kernel: a CTA quantizes one TR x 128 bf16 tile (TR = 64 rows; 128 for grouped
+// tensors, whose group boundaries are multiples of 128 rows, so that the per-tile
+// group lookup, tensor scales and tables serve twice the rows).  The tile goes
+// straight from global to shared memory (cp.async, 16 bytes per copy, TR / 16 per
+// thread; rows and columns past the tensor and gathered padding rows are zero-filled
+// by the copy itself), so no register holds it in flight.  Then one thread per
+// 16-element row block writes the row orientation, and one thread per column pair
+// and 16-row chunk writes the column orientation.  k2D: 16x16 blocks, the tile scale is found by the
 // column pass and shared by both orientations.  kRht: the 16-point RHT down each
 // column chunk before the column orientation is quantized.  kRowRht: the row
 // orientation is rotated along each row block (the Mosaic recipe's dgrad operands).
@@ -945,11 +947,12 @@ constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;  // +16 bytes per row: conf
 // The work on one tile whose bf16 values are in `tile` (rows r0.., columns c0..)
 // with the multiplier tables filled: row orientation, column orientation and the
 // scale atoms.  Every thread of the CTA calls it (it meets the CTA's barriers).
-template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
+// TR: the tile's rows (64 or 128; a multiple of 64, r0 a multiple of TR).
+template <bool k2D, bool kRht, bool kGrouped, bool kRowRht, int TR = kTR>
 __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, int64_t c0,
                                             const uint16_t (*tile)[kPitch], const float (*inv_tab)[256],
                                             uint32_t (*tile_s)[kTC / 16], float (*tile_inv)[kTC / 16],
-                                            uint8_t* col_atom, uint8_t (*row_half_atoms)[32][8],
+                                            uint8_t* col_atom, uint8_t (*row_half_atoms)[32][TR / 8],
                                             const TensorScale& tr, const TensorScale& tc,
                                             const uint32_t (&rk)[20], int64_t g_row0, int64_t g_rows) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -960,7 +963,7 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
     // ---- row pass: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
     auto row_pass = [&]() {
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < TR / 32; ++k) {
             const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
             const int64_t r = r0 + lr, c = c0 + lc;
             // two 16-byte reads, the lane quads of a row taking the halves in opposite
@@ -993,15 +996,18 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
             const uint2 codes =
                 encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
             if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
-            // (row lr, block bc): half-atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
+            // (row lr, block bc): (half-)atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
             row_half_atoms[bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)sc : (uint8_t)0;
         }
     };
     if (want_row && !k2D) row_pass();
 
-    // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunk j
+    // ---- column pass: thread -> column pair cp (columns 2cp, 2cp+1), 16-row chunks
+    // j = tid / 64 + 4 i
     if (want_col || k2D) {
-        const int cp = tid & 63, j = tid >> 6;
+#pragma unroll 1
+    for (int jj = 0; jj < TR / 64; ++jj) {
+        const int cp = tid & 63, j = (tid >> 6) + 4 * jj;
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = *reinterpret_cast<const uint32_t*>(&tile[16 * j + e][2 * cp]);
@@ -1070,35 +1076,44 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
             }
         }
     }
+    }
     if (want_row && k2D) {
         __syncthreads();  // tile scales written
         row_pass();
     }
 
-    // ---- scale stores.  Every entry written lies inside the scale buffer: the
-    // column atom is (128-column group c0 / 128, blocks r0 / 16 .. + 3) with r0 a
-    // multiple of 64 below the rows; the row half-atoms cover 64 rows below
-    // pad128(rows), and the second is skipped when its blocks start past the
-    // padded block count.
+    // ---- scale stores.  Every entry written lies inside the scale buffer: a
+    // column atom is (128-column group c0 / 128, blocks 4a .. 4a+3 of rows) for the
+    // tile's 64-row groups a that start below the padded block count; the row
+    // (half-)atoms cover TR rows below pad128(rows), and the second is skipped when
+    // its blocks start past the padded block count.
     __syncthreads();
-    if (want_col && warp == 0) {
+    if (want_col && warp < TR / 64) {
         const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
-        const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6);
-        // line l of the atom: byte 4w + j holds (column l + 32w, block j)
-        uint32_t line[4];
+        if ((r0 >> 6) + warp < katoms_c) {
+            const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6) + warp;
+            const uint8_t* ca = col_atom + warp * 512;
+            // line l of the atom: byte 4w + j holds (column l + 32w, block j)
+            uint32_t line[4];
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-            line[w] = (uint32_t)col_atom[lane + 32 * w] | ((uint32_t)col_atom[128 + lane + 32 * w] << 8) |
-                      ((uint32_t)col_atom[256 + lane + 32 * w] << 16) | ((uint32_t)col_atom[384 + lane + 32 * w] << 24);
-        *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) = make_uint4(line[0], line[1], line[2], line[3]);
+            for (int w = 0; w < 4; ++w)
+                line[w] = (uint32_t)ca[lane + 32 * w] | ((uint32_t)ca[128 + lane + 32 * w] << 8) |
+                          ((uint32_t)ca[256 + lane + 32 * w] << 16) | ((uint32_t)ca[384 + lane + 32 * w] << 24);
+            *reinterpret_cast<uint4*>(p.col_sf + atom * 512 + lane * 16) = make_uint4(line[0], line[1], line[2], line[3]);
+        }
     }
     if (want_row && (warp == 2 || warp == 3)) {
         const int64_t katoms_r = (p.cols / 16 + 3) >> 2;
         const int a = warp - 2;
         if ((c0 >> 6) + a < katoms_r) {
             const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
-            *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
-                *reinterpret_cast<const uint2*>(row_half_atoms[a][lane]);
+            if constexpr (TR == 128) {
+                *reinterpret_cast<uint4*>(p.row_sf + atom * 512 + lane * 16) =
+                    *reinterpret_cast<const uint4*>(row_half_atoms[a][lane]);
+            } else {
+                *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
+                    *reinterpret_cast<const uint2*>(row_half_atoms[a][lane]);
+            }
         }
     }
 }
@@ -1112,42 +1127,43 @@ constexpr int quant_tile_min_blocks() {
     return 4;
 }
 
-template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
+template <bool k2D, bool kRht, bool kGrouped, bool kRowRht, int TR = kTR>
 __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGrouped>()))
     quant_tile_kernel(const QuantParams p) {
-    __shared__ __align__(16) uint16_t tile[kTR][kPitch];
+    __shared__ __align__(16) uint16_t tile[TR][kPitch];
     __shared__ float inv_tab[2][256];  // element multipliers of every scale code: rows, columns
-    __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
-    __shared__ float tile_inv[kTR / 16][kTC / 16];
+    __shared__ uint32_t tile_s[TR / 16][kTC / 16];
+    __shared__ float tile_inv[TR / 16][kTC / 16];
     // The tile's scales, staged so that they leave in wide stores instead of one
     // byte each: the column orientation's 128 columns x 4 blocks are exactly one
     // 512-byte atom (staged block-major, reordered into lines when stored); the row
     // orientation's 64 rows x 8 blocks are 8 bytes of each of the 32 lines of two
     // atoms.  Entries past the tensor hold 0 (the padding).
-    __shared__ __align__(16) uint8_t col_atom[512];
-    __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
+    __shared__ __align__(16) uint8_t col_atom[TR / 16 * 128];
+    __shared__ __align__(16) uint8_t row_half_atoms[2][32][TR / 8];
 
     const int tid = threadIdx.x;
-    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
+    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * TR, c0 = (int64_t)blockIdx.x * kTC;
 
-    // ---- copies first (they do not depend on the scales): 1024 x 16 bytes, four per
-    // thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7.  Gathered rows:
-    // the four source-row indices are all loaded before any is checked, so their
-    // latencies overlap.
-    int64_t sr[4];
-    bool in[4];
+    // ---- copies first (they do not depend on the scales): TR * 16 x 16 bytes, TR / 16
+    // per thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7.  Gathered rows:
+    // the source-row indices of a thread are all loaded before any is checked, so
+    // their latencies overlap.
+    constexpr int kCopies = TR / 16;
+    int64_t sr[kCopies];
+    bool in[kCopies];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kCopies; ++k) {
         const int64_t r = r0 + ((k * 256 + tid) >> 4), c = c0 + ((k * 256 + tid) & 15) * 8;
         sr[k] = r;
         in[k] = r < p.rows && c < p.cols;
     }
     if (p.row_src != nullptr) {
-        int32_t idx[4];
+        int32_t idx[kCopies];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) idx[k] = in[k] ? __ldg(p.row_src + sr[k]) : -1;
+        for (int k = 0; k < kCopies; ++k) idx[k] = in[k] ? __ldg(p.row_src + sr[k]) : -1;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < kCopies; ++k) {
             if (in[k] && idx[k] >= p.src_rows) {
                 set_status(p.status, kStatusIndex);
                 in[k] = false;
@@ -1157,7 +1173,7 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
         }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kCopies; ++k) {
         const int q = k * 256 + tid;
         const int lr = q >> 4, lc = (q & 15) * 8;
         cp_async16(&tile[lr][lc], in[k] ? (const void*)(p.x + sr[k] * p.cols + c0 + lc) : (const void*)p.x,
@@ -1225,8 +1241,8 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();  // tile and tables in shared memory
 
-    tile_passes<k2D, kRht, kGrouped, kRowRht>(p, r0, c0, tile, inv_tab, tile_s, tile_inv, col_atom,
-                                              row_half_atoms, tr, tc, rk, g_row0, g_rows);
+    tile_passes<k2D, kRht, kGrouped, kRowRht, TR>(p, r0, c0, tile, inv_tab, tile_s, tile_inv, col_atom,
+                                                  row_half_atoms, tr, tc, rk, g_row0, g_rows);
 }
 
 // Persistent form for ungrouped 16x16 tensors: four CTAs per SM walk the tiles (bottom
@@ -1643,8 +1659,9 @@ static cudaError_t launch_tile(const QuantParams& p, int sm_count, cudaStream_t 
         quant_tile_persistent_kernel<k2D, kRht, kRowRht><<<grid, 256, 0, st>>>(p);
         return cudaGetLastError();
     } else {
-        const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
-        quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, 0, st>>>(p);
+        constexpr int TR = kGrouped ? 128 : kTR;  // grouped: the tile's fixed costs over twice the rows
+        const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + TR - 1) / TR));
+        quant_tile_kernel<k2D, kRht, kGrouped, kRowRht, TR><<<grid, 256, 0, st>>>(p);
         return cudaGetLastError();
     }
 }
