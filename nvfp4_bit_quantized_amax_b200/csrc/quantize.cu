@@ -927,8 +927,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 
 // ============================================================================
 // Tile kernel: a CTA quantizes one TR x 128 bf16 tile (TR = 64 rows; 128 for grouped
-// tensors, whose group boundaries are multiples of 128 rows, so that the per-tile
-// group lookup, tensor scales and tables serve twice the rows).  The tile goes
+// tensors, whose group boundaries are multiples of 128 rows, and for 16x16 blocks, so
+// that the per-tile group lookup, tensor scales and tables serve twice the rows).  The tile goes
 // straight from global to shared memory (cp.async, 16 bytes per copy, TR / 16 per
 // thread; rows and columns past the tensor and gathered padding rows are zero-filled
 // by the copy itself), so no register holds it in flight.  Then one thread per
@@ -1243,91 +1243,6 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
 
     tile_passes<k2D, kRht, kGrouped, kRowRht, TR>(p, r0, c0, tile, inv_tab, tile_s, tile_inv, col_atom,
                                                   row_half_atoms, tr, tc, rk, g_row0, g_rows);
-}
-
-// Persistent form for ungrouped 16x16 tensors: four CTAs per SM walk the tiles (bottom
-// tile row first, as above), each computing the tensor scales and the multiplier
-// tables once and copying the next tile into the second of two shared-memory
-// buffers while it works on the current one.  Same per-tile work (tile_passes), so
-// the same bytes.
-template <bool k2D, bool kRht, bool kRowRht>
-__global__ void __launch_bounds__(256, 4) quant_tile_persistent_kernel(const QuantParams p) {
-    __shared__ __align__(16) uint16_t tile[2][kTR][kPitch];
-    __shared__ float inv_tab[2][256];
-    __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
-    __shared__ float tile_inv[kTR / 16][kTC / 16];
-    __shared__ __align__(16) uint8_t col_atom[512];
-    __shared__ __align__(16) uint8_t row_half_atoms[2][32][8];
-    __shared__ float sh_scales[4];
-    const int tid = threadIdx.x;
-    const int64_t tiles_x = (p.cols + kTC - 1) / kTC, tiles_y = (p.rows + kTR - 1) / kTR;
-    const int64_t tiles = tiles_x * tiles_y;
-    // copies of tile t into buffer b (one commit group): 1024 x 16 bytes, four per
-    // thread; rows and columns past the tensor are zero-filled by the copy
-    auto issue = [&](int64_t t, int b) {
-        const int64_t r0 = (tiles_y - 1 - t / tiles_x) * kTR, c0 = (t % tiles_x) * kTC;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int q = k * 256 + tid;
-            const int lr = q >> 4, lc = (q & 15) * 8;
-            const int64_t r = r0 + lr, c = c0 + lc;
-            const bool in = r < p.rows && c < p.cols;
-            cp_async16(&tile[b][lr][lc], in ? (const void*)(p.x + r * p.cols + c) : (const void*)p.x, in ? 16u : 0u);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    int64_t t = blockIdx.x;
-    if (t < tiles) issue(t, 0);
-
-    const uint32_t wr = p.amax_words[0];
-    const uint32_t wc = p.col_rht ? p.amax_words[1] : wr;
-    const bool first = tid == 0 && blockIdx.x == 0;
-    if (!finite_bits(wr) || !finite_bits(wc)) {  // the same for the whole CTA
-        if (first) {
-            set_status(p.status, kStatusNonFinite);
-            if (p.row_g) p.row_g[0] = __uint_as_float(0x7FC00000u);
-            if (p.col_g) p.col_g[0] = __uint_as_float(0x7FC00000u);
-        }
-        asm volatile("cp.async.wait_group 0;" ::: "memory");  // let the copies land before leaving
-        return;
-    }
-    if (tid == 0) {
-        const TensorScale a = tensor_scale_from_amax(__uint_as_float(wr));
-        const TensorScale b = tensor_scale_from_amax(__uint_as_float(wc));
-        sh_scales[0] = a.g;
-        sh_scales[1] = a.enc;
-        sh_scales[2] = b.g;
-        sh_scales[3] = b.enc;
-        if (first) {
-            if (p.row_g) p.row_g[0] = a.g;
-            if (p.col_g) p.col_g[0] = b.g;
-        }
-    }
-    __syncthreads();
-    const TensorScale tr{sh_scales[0], sh_scales[1]}, tc{sh_scales[2], sh_scales[3]};
-    {
-        const float dec = e4m3_to_f32((uint32_t)tid);
-        const float gr = __fmul_rn(dec, tr.g), gc = __fmul_rn(dec, tc.g);
-        inv_tab[0][tid] = (gr == 0.0f) ? 0.0f : fminf(__frcp_rn(gr), 3.402823466e38f);
-        inv_tab[1][tid] = (gc == 0.0f) ? 0.0f : fminf(__frcp_rn(gc), 3.402823466e38f);
-    }
-    int b = 0;
-    for (; t < tiles; t += gridDim.x) {
-        // the next tile's copies go into the other buffer, last read by the previous
-        // tile's passes (the barrier at the end of the loop); an empty group past the end
-        if (t + gridDim.x < tiles)
-            issue(t + gridDim.x, b ^ 1);
-        else
-            asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's copies have landed
-        __syncthreads();                                       // ... for every thread (and the tables)
-        const int64_t r0 = (tiles_y - 1 - t / tiles_x) * kTR, c0 = (t % tiles_x) * kTC;
-        tile_passes<k2D, kRht, false, kRowRht>(p, r0, c0, tile[b], inv_tab, tile_s, tile_inv, col_atom,
-                                               row_half_atoms, tr, tc, p.rk, 0, p.rows);
-        __syncthreads();  // buffer b and the staged scales are free again
-        b ^= 1;
-    }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ============================================================================
@@ -1649,21 +1564,17 @@ cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStrea
 
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
 static cudaError_t launch_tile(const QuantParams& p, int sm_count, cudaStream_t st) {
-    // The persistent form pays where the per-tile setup weighs most (16x16: W
-    // 20480 x 5120 0.1475 -> 0.1421 ms); for the rotated and SR passes its
-    // lockstep tiles issue less well than independent CTAs (dY 0.423 -> 0.432 ms).
-    if constexpr (k2D && !kGrouped) {
-        if (p.row_src != nullptr) return cudaErrorInvalidValue;  // gathered rows come grouped only
-        const int64_t tiles = ((p.cols + kTC - 1) / kTC) * ((p.rows + kTR - 1) / kTR);
-        const int grid = grid_for(tiles, 1, sm_count, 4);
-        quant_tile_persistent_kernel<k2D, kRht, kRowRht><<<grid, 256, 0, st>>>(p);
-        return cudaGetLastError();
-    } else {
-        constexpr int TR = kGrouped ? 128 : kTR;  // grouped: the tile's fixed costs over twice the rows
-        const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + TR - 1) / TR));
-        quant_tile_kernel<k2D, kRht, kGrouped, kRowRht, TR><<<grid, 256, 0, st>>>(p);
-        return cudaGetLastError();
-    }
+    (void)sm_count;
+    // 128-row tiles for grouped tensors and 16x16 blocks: a tile's fixed costs (group
+    // lookup, tensor scales, multiplier tables, the 16x16 tile scales' exchange and
+    // the barriers) over twice the rows (W 20480 x 5120 0.1439 -> 0.1296 ms against
+    // a persistent double-buffered 64-row kernel; MoE step 1.002 -> 0.984 ms); 64 rows
+    // for the dense 1x16 passes, where 128 measured 1% slower.
+    if (!kGrouped && p.row_src != nullptr) return cudaErrorInvalidValue;  // gathered rows come grouped only
+    constexpr int TR = (kGrouped || k2D) ? 128 : kTR;
+    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + TR - 1) / TR));
+    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht, TR><<<grid, 256, 0, st>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_tile(const QuantParams& params, bool two_d, int sm_count, cudaStream_t st) {

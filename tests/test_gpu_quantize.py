@@ -163,9 +163,9 @@ def test_quantize_2d_orientations(ora, shape, recipe):
 @pytest.mark.parametrize("shape,recipe", [((16384, 272), "dy"), ((8208, 1040), "w")])
 def test_quantize_2d_many_units_ragged(ora, shape, recipe):
     """Enough work that every warp of the streamed amax pass walks several 16 x 128
-    units (crossing rows, the last column unit partial: 272 columns) and every CTA of
-    the persistent 16x16 kernel several tiles (the last tile row and column partial:
-    8208 rows, 1040 columns).  Full comparison with the oracle, both orientations."""
+    units (crossing rows, the last column unit partial: 272 columns), and many
+    128 x 128 tiles of the 16x16 tile kernel with the last tile row and column partial
+    (8208 rows, 1040 columns).  Full comparison with the oracle, both orientations."""
     signs = syn.rht_signs(5)
     x = syn.normal_bf16(shape, 23, outlier_prob=0.01)
     bm, rr, cr, rht = {"dy": (0, 1, 1, True), "w": (1, 0, 0, False)}[recipe]
