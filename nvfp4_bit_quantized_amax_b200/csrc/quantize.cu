@@ -926,10 +926,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 }
 
 // ============================================================================
-// Tile kernel: a CTA quantizes one TR x 128 bf16 tile (TR = 64 rows; 128 for grouped
-// tensors, whose group boundaries are multiples of 128 rows, and for 16x16 blocks, so
-// that the per-tile group lookup, tensor scales and tables serve twice the rows).  The tile goes
-// straight from global to shared memory (cp.async, 16 bytes per copy, TR / 16 per
+// Tile kernel: a CTA quantizes one 128 x 128 bf16 tile (a grouped tensor's group
+// boundaries are multiples of 128 rows, so a tile lies in one group).  The tile goes
+// straight from global to shared memory (cp.async, 16 bytes per copy, eight per
 // thread; rows and columns past the tensor and gathered padding rows are zero-filled
 // by the copy itself), so no register holds it in flight.  Then one thread per
 // 16-element row block writes the row orientation, and one thread per column pair
@@ -942,17 +941,16 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
 // Tiles run bottom-up (the grid's y extent reversed), so the first tiles re-read the
 // rows the amax pass read last (still in L2).
 // ============================================================================
-constexpr int kTR = 64, kTC = 128, kPitch = kTC + 8;  // +16 bytes per row: conflict-free column reads
+constexpr int kTR = 128, kTC = 128, kPitch = kTC + 8;  // +16 bytes per row: conflict-free column reads
 
 // The work on one tile whose bf16 values are in `tile` (rows r0.., columns c0..)
 // with the multiplier tables filled: row orientation, column orientation and the
 // scale atoms.  Every thread of the CTA calls it (it meets the CTA's barriers).
-// TR: the tile's rows (64 or 128; a multiple of 64, r0 a multiple of TR).
-template <bool k2D, bool kRht, bool kGrouped, bool kRowRht, int TR = kTR>
+template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
 __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, int64_t c0,
                                             const uint16_t (*tile)[kPitch], const float (*inv_tab)[256],
                                             uint32_t (*tile_s)[kTC / 16], float (*tile_inv)[kTC / 16],
-                                            uint8_t* col_atom, uint8_t (*row_half_atoms)[32][TR / 8],
+                                            uint8_t* col_atom, uint8_t (*row_atoms)[32][16],
                                             const TensorScale& tr, const TensorScale& tc,
                                             const uint32_t (&rk)[20], int64_t g_row0, int64_t g_rows) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -963,7 +961,7 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
     // ---- row pass: row block b = k * 256 + tid is row b / 8, columns (b % 8) * 16 .. + 15
     auto row_pass = [&]() {
 #pragma unroll
-        for (int k = 0; k < TR / 32; ++k) {
+        for (int k = 0; k < kTR / 32; ++k) {
             const int lr = (k * 256 + tid) >> 3, bc = tid & 7, lc = bc * 16;
             const int64_t r = r0 + lr, c = c0 + lc;
             // two 16-byte reads, the lane quads of a row taking the halves in opposite
@@ -996,8 +994,8 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
             const uint2 codes =
                 encode16(v, inv, p.row_sr, rk, 0u, (uint64_t)(r - g_row0) * (uint64_t)p.cols + (uint64_t)c);
             if (inside) *reinterpret_cast<uint2*>(p.row_data + r * (p.cols >> 1) + (c >> 1)) = codes;
-            // (row lr, block bc): (half-)atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
-            row_half_atoms[bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)sc : (uint8_t)0;
+            // (row lr, block bc): atom bc / 4, line lr % 32, byte 4 * (lr / 32) + bc % 4
+            row_atoms[bc >> 2][lr & 31][(lr >> 5) * 4 + (bc & 3)] = inside ? (uint8_t)sc : (uint8_t)0;
         }
     };
     if (want_row && !k2D) row_pass();
@@ -1006,7 +1004,7 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
     // j = tid / 64 + 4 i
     if (want_col || k2D) {
 #pragma unroll 1
-    for (int jj = 0; jj < TR / 64; ++jj) {
+    for (int jj = 0; jj < kTR / 64; ++jj) {
         const int cp = tid & 63, j = (tid >> 6) + 4 * jj;
         uint32_t w[16];
 #pragma unroll
@@ -1084,11 +1082,11 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
 
     // ---- scale stores.  Every entry written lies inside the scale buffer: a
     // column atom is (128-column group c0 / 128, blocks 4a .. 4a+3 of rows) for the
-    // tile's 64-row groups a that start below the padded block count; the row
-    // (half-)atoms cover TR rows below pad128(rows), and the second is skipped when
-    // its blocks start past the padded block count.
+    // tile's 64-row groups a that start below the padded block count; the row atoms
+    // cover the tile's 128 rows below pad128(rows), and the second is skipped when its
+    // blocks start past the padded block count.
     __syncthreads();
-    if (want_col && warp < TR / 64) {
+    if (want_col && warp < kTR / 64) {
         const int64_t katoms_c = (p.rows / 16 + 3) >> 2;
         if ((r0 >> 6) + warp < katoms_c) {
             const int64_t atom = (c0 >> 7) * katoms_c + (r0 >> 6) + warp;
@@ -1107,49 +1105,45 @@ __device__ __forceinline__ void tile_passes(const QuantParams& p, int64_t r0, in
         const int a = warp - 2;
         if ((c0 >> 6) + a < katoms_r) {
             const int64_t atom = (r0 >> 7) * katoms_r + (c0 >> 6) + a;
-            if constexpr (TR == 128) {
-                *reinterpret_cast<uint4*>(p.row_sf + atom * 512 + lane * 16) =
-                    *reinterpret_cast<const uint4*>(row_half_atoms[a][lane]);
-            } else {
-                *reinterpret_cast<uint2*>(p.row_sf + atom * 512 + lane * 16 + ((r0 & 127) >> 5) * 4) =
-                    *reinterpret_cast<const uint2*>(row_half_atoms[a][lane]);
-            }
+            *reinterpret_cast<uint4*>(p.row_sf + atom * 512 + lane * 16) =
+                *reinterpret_cast<const uint4*>(row_atoms[a][lane]);
         }
     }
 }
 
 // Resident CTAs per SM the register budget is sized for (each CTA quantizes one tile,
 // so more resident CTAs keep more copies and more independent arithmetic in flight).
-// Four for every variant: the grouped rotated variant spills at 64 registers, and is
-// still faster than at 80 registers and three CTAs (MoE step 1.110 -> 1.077 ms).
+// Three (80 registers) for the dense rotated passes, which spill 20 B there and run
+// 3% faster than at four; four (64 registers) for the others, the grouped rotated
+// variant included (three measured the same).
 template <bool k2D, bool kRht, bool kGrouped>
 constexpr int quant_tile_min_blocks() {
-    return 4;
+    return (kRht && !kGrouped) ? 3 : 4;
 }
 
-template <bool k2D, bool kRht, bool kGrouped, bool kRowRht, int TR = kTR>
+template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
 __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGrouped>()))
     quant_tile_kernel(const QuantParams p) {
-    __shared__ __align__(16) uint16_t tile[TR][kPitch];
+    __shared__ __align__(16) uint16_t tile[kTR][kPitch];
     __shared__ float inv_tab[2][256];  // element multipliers of every scale code: rows, columns
-    __shared__ uint32_t tile_s[TR / 16][kTC / 16];
-    __shared__ float tile_inv[TR / 16][kTC / 16];
+    __shared__ uint32_t tile_s[kTR / 16][kTC / 16];
+    __shared__ float tile_inv[kTR / 16][kTC / 16];
     // The tile's scales, staged so that they leave in wide stores instead of one
-    // byte each: the column orientation's 128 columns x 4 blocks are exactly one
-    // 512-byte atom (staged block-major, reordered into lines when stored); the row
-    // orientation's 64 rows x 8 blocks are 8 bytes of each of the 32 lines of two
-    // atoms.  Entries past the tensor hold 0 (the padding).
-    __shared__ __align__(16) uint8_t col_atom[TR / 16 * 128];
-    __shared__ __align__(16) uint8_t row_half_atoms[2][32][TR / 8];
+    // byte each: each 64-row half of the column orientation's 128 columns x 8 blocks
+    // is exactly one 512-byte atom (staged block-major, reordered into lines when
+    // stored); the row orientation's 128 rows x 8 blocks are exactly two atoms.
+    // Entries past the tensor hold 0 (the padding).
+    __shared__ __align__(16) uint8_t col_atom[kTR / 16 * 128];
+    __shared__ __align__(16) uint8_t row_atoms[2][32][16];
 
     const int tid = threadIdx.x;
-    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * TR, c0 = (int64_t)blockIdx.x * kTC;
+    const int64_t r0 = (int64_t)(gridDim.y - 1 - blockIdx.y) * kTR, c0 = (int64_t)blockIdx.x * kTC;
 
-    // ---- copies first (they do not depend on the scales): TR * 16 x 16 bytes, TR / 16
-    // per thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7.  Gathered rows:
+    // ---- copies first (they do not depend on the scales): 2048 x 16 bytes, eight per
+    // thread; copy q covers row q / 16, columns (q % 16) * 8 .. + 7.  Gathered rows:
     // the source-row indices of a thread are all loaded before any is checked, so
     // their latencies overlap.
-    constexpr int kCopies = TR / 16;
+    constexpr int kCopies = kTR / 16;
     int64_t sr[kCopies];
     bool in[kCopies];
 #pragma unroll
@@ -1241,8 +1235,8 @@ __global__ void __launch_bounds__(256, (quant_tile_min_blocks<k2D, kRht, kGroupe
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();  // tile and tables in shared memory
 
-    tile_passes<k2D, kRht, kGrouped, kRowRht, TR>(p, r0, c0, tile, inv_tab, tile_s, tile_inv, col_atom,
-                                                  row_half_atoms, tr, tc, rk, g_row0, g_rows);
+    tile_passes<k2D, kRht, kGrouped, kRowRht>(p, r0, c0, tile, inv_tab, tile_s, tile_inv, col_atom, row_atoms,
+                                              tr, tc, rk, g_row0, g_rows);
 }
 
 // ============================================================================
@@ -1565,15 +1559,9 @@ cudaError_t launch_quant_rows(const QuantParams& params, int sm_count, cudaStrea
 template <bool k2D, bool kRht, bool kGrouped, bool kRowRht>
 static cudaError_t launch_tile(const QuantParams& p, int sm_count, cudaStream_t st) {
     (void)sm_count;
-    // 128-row tiles for grouped tensors and 16x16 blocks: a tile's fixed costs (group
-    // lookup, tensor scales, multiplier tables, the 16x16 tile scales' exchange and
-    // the barriers) over twice the rows (W 20480 x 5120 0.1439 -> 0.1296 ms against
-    // a persistent double-buffered 64-row kernel; MoE step 1.002 -> 0.984 ms); 64 rows
-    // for the dense 1x16 passes, where 128 measured 1% slower.
     if (!kGrouped && p.row_src != nullptr) return cudaErrorInvalidValue;  // gathered rows come grouped only
-    constexpr int TR = (kGrouped || k2D) ? 128 : kTR;
-    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + TR - 1) / TR));
-    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht, TR><<<grid, 256, 0, st>>>(p);
+    const dim3 grid((unsigned)((p.cols + kTC - 1) / kTC), (unsigned)((p.rows + kTR - 1) / kTR));
+    quant_tile_kernel<k2D, kRht, kGrouped, kRowRht><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
