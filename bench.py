@@ -229,6 +229,33 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_tflops(world, FLOPS_PER_STEP, ms)
 
     out = {}
+    # ---- the same step, its three C-ABI calls captured once as a CUDA graph and
+    # replayed (the launch gaps between the calls' kernels go away); one rank only, so
+    # that a capture failure cannot leave other ranks waiting in a collective
+    def graph_step_ms():
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        g_ms = timed(graph.replay, args.steps, max(args.warmup, 3))
+        del graph
+        return g_ms
+
+    if world > 1:
+        out["step_graph"] = {"skipped": "measured on one GPU only"}
+    else:
+        try:
+            g_ms = graph_step_ms()
+            out["step_graph"] = {"ms_per_step": round(g_ms, 4),
+                                 "value": round(whole_job_tflops(world, FLOPS_PER_STEP, g_ms), 2),
+                                 "note": "the timed step's three C-ABI calls replayed as one CUDA graph"}
+        except Exception as exc:  # reported, not fatal: the eager number stands
+            out["step_graph"] = {"error": str(exc)[:200]}
+    assert capi.nvfp4_read_status(ws) == 0
     out["in_step"] = in_step_breakdown(capi, syn, X, W, dY, Y, dX, dW, ws, signs, seed, stream,
                                        barrier, iters=max(5, min(20, args.steps)))
     # ---- per-kernel timing on the same stream (each launch alone, back to back); every
