@@ -57,11 +57,6 @@ __device__ __forceinline__ f32x2 add2_ru(f32x2 a, f32x2 b) {
     asm("add.rp.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-__device__ __forceinline__ float fmin3(float a, float b, float c) {
-    float d;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
 // Two 16-bit lanes: signed minimum, unsigned maximum.
 __device__ __forceinline__ uint32_t vmin_s16x2(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -173,16 +168,6 @@ __device__ __forceinline__ bool span_ok_mag(uint32_t mx, uint32_t mn) {
     if (mx == 0u) return true;  // all inputs zero
     if (mn == 0u) return false;
     const int emax = (int)(mx >> 7), emin = (int)(mn >> 7);
-    return emax <= 251 && emax - max(emin, 1) <= 13;
-}
-
-// The exponent-span test above for one 16-bit lane of the chunk statistics: with
-// v = |x| + 0x7FFF per bf16 (0x7FFF for a zero, >= 0x8000 otherwise), vmx is the
-// unsigned maximum of v and vmn its signed minimum (the smallest nonzero |x|).
-__device__ __forceinline__ bool span_ok(uint32_t vmx, uint32_t vmn) {
-    if (vmx == 0x7FFFu) return true;  // all inputs zero
-    const int emax = (int)((vmx - 0x7FFFu) >> 7);
-    const int emin = (int)((vmn - 0x7FFFu) >> 7);
     return emax <= 251 && emax - max(emin, 1) <= 13;
 }
 
