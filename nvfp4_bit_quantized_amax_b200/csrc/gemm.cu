@@ -267,7 +267,7 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
                  : "memory");
 }
 // One epilogue warp's share of a finished tile: its 32 TMEM lanes (rows row0 ..
-// row0+31 of D, lane = row) by BN/2 columns from col0; nothing is stored unless
+// row0+31 of D, lane = row) by CW columns from col0; nothing is stored unless
 // `store`, and `zero` writes zeros without reading the accumulator.  Drains the accumulator into
 // registers (times alpha, rounded to bf16; the fp32 checking output is stored
 // before the release), arrives on the accumulator-empty barrier (local, or the
@@ -276,12 +276,12 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
 // j ^ ((row / 4) % 2), the 32-byte swizzle the store's tensor map undoes
 // (conflict-free), one bulk tensor store each; rows and columns past M and N are
 // clipped by the tensor map.
-template <int BN>
+template <int CW>
 __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, int64_t row0, int64_t col0,
                                               const GemmParams& p, float alpha, bool store, bool zero,
                                               uint32_t acc_empty, uint32_t remote, uint32_t buf,
                                               const CUtensorMap* tmD) {
-    constexpr int HC = BN / 2;
+    constexpr int HC = CW;
     const int lane = threadIdx.x & 31;
     const int64_t row = row0 + lane;
     uint32_t packed[HC / 2];  // bf16 pairs of this thread's row
@@ -609,7 +609,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // after a timeout the accumulator is neither read nor stored
             const bool bad = *(volatile int*)&timed_out != 0;
             const int64_t m_in = (jb.d_row - (jb.group >= 0 && p.group_mode == 2 ? (int64_t)jb.group * p.M : 0)) + 32 * q;
-            epilogue_tile<BN>(lane_base, jb.d_row + 32 * q, jb.n0 + half * HC, p, alpha,
+            epilogue_tile<HC>(lane_base, jb.d_row + 32 * q, jb.n0 + half * HC, p, alpha,
                               !bad && m_in < p.M, bad || jb.k_len == 0, smem_addr(&S.acc_empty), 0u,
                               smem_addr(S.dstage[warp - 6]), &tmD);
         }
@@ -720,11 +720,22 @@ __device__ __forceinline__ void tc_mma_nvf4_pair_x4(uint32_t d_tmem, uint64_t ad
 constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
                                 ((uint32_t)(256 >> 4) << 24);
 
-template <int STAGES>
+// Epilogue warps of the pair kernel (EW, a template parameter): EW / 4 per TMEM lane
+// quarter, each draining 256 / (EW / 4) columns of its 32 rows.  Sixteen release the
+// accumulator sooner, which pays where tiles are short (the grouped GEMMs, 4-8 k-tiles
+// per tile: MoE step 0.986 -> 0.976 ms); on the long dense tiles the extra waiting
+// warps cost more than they save (MLP GEMMs 0.996 -> 1.020 ms), so those keep eight.
+constexpr int kPairEpiWarpsMax = 16;
+template <int EW>
+constexpr int pair_threads() {
+    return (6 + EW + 1) * 32;  // producer, issuer, 4 scale writers, epilogue, scale producer
+}
+
+template <int STAGES, int EW>
 struct __align__(1024) PairSmem {
     uint8_t a[STAGES][128 * kBKBytes];       // this CTA's 128 rows of A, 16 KB / stage
     uint8_t b[STAGES][128 * kBKBytes];       // this CTA's 128 rows of B, 16 KB / stage
-    uint8_t dstage[8][32 * 32];              // per epilogue warp: 32 rows x 16 bf16, 32B-swizzled
+    uint8_t dstage[EW][32 * 32];             // per epilogue warp: 32 rows x 16 bf16, 32B-swizzled
     uint8_t sfa[STAGES][4 * 512];            // scales of this CTA's A rows
     uint8_t sfb[STAGES][2][4 * 512];         // scales of all 256 B rows of the tile
     uint64_t full[STAGES];       // this CTA's A/B boxes landed
@@ -737,7 +748,6 @@ struct __align__(1024) PairSmem {
     uint32_t tmem_base;
 };
 
-constexpr int kPairThreads = 480;  // the warps of the one-SM kernel + a scale-copy producer
 
 // Operands and result of one 256 x 256 output tile of the pair kernel (the group
 // modes of GemmParams; mode 1 walks the 256-row tiles of every group, whose second
@@ -791,12 +801,15 @@ __device__ __forceinline__ void tc_mma_mx_pair_x4(uint32_t d_tmem, uint64_t ades
         : "memory");
 }
 
-template <int STAGES, bool kMx>
-__global__ void __launch_bounds__(kPairThreads, 1)
+template <int STAGES, bool kMx, int EW>
+__global__ void __launch_bounds__(pair_threads<EW>(), 1)
     gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-    using Smem = PairSmem<STAGES>;
-    constexpr int BN = 256, G = 2, HC = BN / 2;
+    using Smem = PairSmem<STAGES, EW>;
+    constexpr int BN = 256, G = 2;
+    constexpr int kEpiCols = BN / (EW / 4);  // columns per epilogue warp
+    constexpr int kScaleW = 6 + EW;          // the scale-atom producer, after the epilogue warps
+    static_assert(EW % 4 == 0 && EW <= kPairEpiWarpsMax, "epilogue warps: a multiple of 4, at most 16");
     constexpr int kSfaCols = 16, kRegion = 48;              // per stage: A scales, then B scales
     constexpr int kUsed = BN + STAGES * kRegion;
     static_assert(kUsed <= 512, "TMEM holds 512 columns");
@@ -883,7 +896,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             mbar_init(smem_addr(&S.sf_full[s]), 8);
         }
         mbar_init(smem_addr(&S.acc_full), 1);
-        mbar_init(smem_addr(&S.acc_empty), 16);
+        mbar_init(smem_addr(&S.acc_empty), 2 * EW);
         mbar_init(smem_addr(&S.drain), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -932,7 +945,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 14) {
+    } else if (warp == kScaleW) {
         if (lane == 0) {
             // ------------------------------------------------ scale-atom producer (both CTAs)
             // One thread issuing every copy of a stage was the pipeline's limit;
@@ -1093,10 +1106,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------- epilogue (warps 6-13, both CTAs)
-        const int q = warp & 3;
-        const int half = (warp - 6) >> 2;
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * HC);
+        // ---------------------------------------------------- epilogue (warps 6 .. 5 + EW, both CTAs)
+        const int q = warp & 3;                // TMEM lane quarter
+        const int part = (warp - 6) >> 2;      // columns [part * kEpiCols, + kEpiCols)
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(part * kEpiCols);
         const uint32_t acc_empty_l = leader ? smem_addr(&S.acc_empty) : mapa_shared(smem_addr(&S.acc_empty), 0);
         uint32_t local = 0;
         for (int64_t pt = cid; pt < tiles; pt += ncl, ++local) {
@@ -1113,7 +1126,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             // after a timeout the accumulator is neither read nor stored
             const bool bad = *(volatile int*)&timed_out != 0;
             const int64_t r_in = 128 * rank + 32 * q;  // this warp's first row inside the tile
-            epilogue_tile<BN>(lane_base, jb.d_row + r_in, jb.n0 + half * HC, p, alpha, !bad && r_in < jb.rows,
+            epilogue_tile<kEpiCols>(lane_base, jb.d_row + r_in, jb.n0 + part * kEpiCols, p, alpha,
+                                        !bad && r_in < jb.rows,
                               bad || jb.k_len == 0, acc_empty_l, leader ? 0u : 1u,
                               smem_addr(S.dstage[warp - 6]), &tmD);
         }
@@ -1133,7 +1147,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (warp == 0 && lane == 0)
             for (int64_t k = (issued_ab > STAGES ? issued_ab - STAGES : 0); k < issued_ab; ++k)
                 mbar_wait_drain(smem_addr(&S.full[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
-        if (warp == 14 && lane == 0)
+        if (warp == kScaleW && lane == 0)
             for (int64_t k = (issued_sf > STAGES ? issued_sf - STAGES : 0); k < issued_sf; ++k)
                 mbar_wait_drain(smem_addr(&S.sf_loaded[k % STAGES]), (uint32_t)(k / STAGES) & 1u);
         if (warp == 1 && lane == 0 && leader) {
@@ -1253,7 +1267,7 @@ static void pair_tile_order(GemmParams& g, int64_t l2_bytes) {
     g.tile_band = reads_m <= reads_n ? bm : bn;
 }
 
-template <int STAGES, bool kMx>
+template <int STAGES, bool kMx, int EW>
 static cudaError_t launch_gemm_pair(const GemmParams& params, int sm_count, cudaStream_t st) {
     GemmParams p = params;
     if (p.group_mode == 0) {
@@ -1274,10 +1288,10 @@ static cudaError_t launch_gemm_pair(const GemmParams& params, int sm_count, cuda
     memset(&md, 0, sizeof(md));
     const int64_t d_rows = p.group_mode == 2 ? p.M * p.num_groups : p.M;
     if (p.D_bf16 && !make_output_map(&md, p.D_bf16, d_rows, p.N)) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(PairSmem<STAGES>) + 1024;
+    const size_t smem = sizeof(PairSmem<STAGES, EW>) + 1024;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<STAGES, kMx>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_pair_kernel<STAGES, kMx, EW>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -1287,7 +1301,7 @@ static cudaError_t launch_gemm_pair(const GemmParams& params, int sm_count, cuda
                         : p.group_mode == 2 ? tiles_m * tiles_n * p.num_groups
                                             : tiles_m * tiles_n;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kPairThreads);
+    cfg.blockDim = dim3(pair_threads<EW>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -1302,13 +1316,13 @@ static cudaError_t launch_gemm_pair(const GemmParams& params, int sm_count, cuda
     static int resident = 0;
     if (resident == 0) {
         cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
-        if (cudaOccupancyMaxActiveClusters(&resident, gemm_nvf4_pair_kernel<STAGES, kMx>, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&resident, gemm_nvf4_pair_kernel<STAGES, kMx, EW>, &cfg) != cudaSuccess ||
             resident < 1)
             resident = sm_count / 2;
     }
     const int64_t clusters = tiles < resident ? (tiles > 0 ? tiles : 1) : resident;
     cfg.gridDim = dim3((unsigned)(2 * clusters));
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<STAGES, kMx>, ma, mb, md, p);
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<STAGES, kMx, EW>, ma, mb, md, p);
 }
 
 cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
@@ -1316,7 +1330,11 @@ cudaError_t launch_gemm(const GemmParams& p, int sm_count, cudaStream_t st) {
     // problems (mode 1 needs its table of 256-row group tiles)
     const bool pair = sm_count >= 2 && (p.group_mode == 0 ? p.M > 128
                                         : p.group_mode == 2 || p.pair_row0 != nullptr);
-    if (pair) return p.mx ? launch_gemm_pair<5, true>(p, sm_count, st) : launch_gemm_pair<5, false>(p, sm_count, st);
+    if (pair) {
+        if (p.mx) return launch_gemm_pair<5, true, 8>(p, sm_count, st);
+        return p.group_mode != 0 ? launch_gemm_pair<5, false, 16>(p, sm_count, st)
+                                 : launch_gemm_pair<5, false, 8>(p, sm_count, st);
+    }
     if (p.mx) return launch_gemm_cfg<256, 4, true>(p, sm_count, st);
     return launch_gemm_cfg<256, 4, false>(p, sm_count, st);
 }
