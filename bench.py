@@ -37,8 +37,8 @@ FP4_OVER_BF16 = 4.0   # nominal dense FP4 9 PFLOP/s over bf16 2.25 PFLOP/s
 # DRAM bytes (read + write) of one launch of each GEMM of the step, from one-pass ncu
 # captures of that launch; reported only while the GEMM source is the one that was
 # captured.
-GEMM_TRAFFIC = {"gemm_cu_sha256_16": "61acdbb0feaffc48", "bytes": {
-    "fprop": 89231616 + 296627968, "dgrad": 427509760 + 71016448, "wgrad": 118325248 + 180209664}}
+GEMM_TRAFFIC = {"gemm_cu_sha256_16": "30f8c6ccc064eacd", "bytes": {
+    "fprop": 87166208 + 296675584, "dgrad": 428784128 + 71357440, "wgrad": 118288128 + 178921984}}
 
 
 def env_rank():
